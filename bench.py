@@ -1,0 +1,390 @@
+#!/usr/bin/env python
+"""Benchmark of the Gated DeltaNet mixer hot path on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+  prefill: gdn_conv1d_silu + gdn_chunk_prefill over a Qwen3.5-27B-shaped layer
+           (16 key heads, 48 value heads of 128, conv over 10240 channels) at T = 65536,
+           returning the final 48 x 128 x 128 fp32 state;
+  decode : gdn_decode_step for 256 sequences x 1 token, 27B-shaped fp32 states
+           (256 x 48 x 128 x 128, 805 MB) and 3-tap conv states updated in place.
+
+value  = prefill tokens/s for the layer (device time of the prefill phase, events on the
+         launching stream); the decode phase is reported in "decode" as state GB/s.
+Inputs (1.34 GB x, 805 MB state) exceed the 126 MB L2, so no flush is needed.
+
+``--impl reference`` times the fp64 CPU oracle on the host cores instead (bounded sample).
+Run with torchrun for N > 1: every rank runs its own independent 64K sequence and decode
+batch (no data-path collective; weak scaling); timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gated_deltanet_mixer_causal_b200 import workloads as W  # noqa: E402
+
+METRIC = "GDN prefill tokens/s/layer @64K + decode state GB/s, % of roofline"
+UNIT = "tokens/s/layer"
+SHAPE = W.QWEN35_27B
+T_PREFILL = 65536
+B_DECODE = 256
+
+# algorithmic work (chunked form counted at C = 64; see the design notes)
+def prefill_flops_per_token(sh=SHAPE, C=64):
+    d, G = sh.dk, sh.Hv // sh.Hk
+    return sh.Hv * (6 * d * d + 6 * C * d + C * C / 3 + 4 * C * d / G)
+
+
+def prefill_bytes_per_token(sh=SHAPE):
+    # q|k|v in (post-conv y for the chunked call, pre-conv x for the layer), o out, g, beta
+    return sh.conv_channels * 2 + sh.Hv * sh.dv * 2 + 2 * sh.Hv * 4
+
+
+def conv_bytes(T, sh=SHAPE):
+    return 2 * T * sh.conv_channels * 2 + sh.conv_channels * 4 * 2
+
+
+def decode_bytes(B, sh=SHAPE):
+    Cc = sh.conv_channels
+    state = B * sh.Hv * sh.dv * sh.dk * 4
+    return (2 * state + B * Cc * 2 + 2 * B * 3 * Cc * 2 + B * sh.Hv * sh.dv * 2
+            + 2 * B * sh.Hv * 4 + Cc * 4 * 2)
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p["hbm_gbs"], p["bf16_tflops"], p.get("bf16_tflops_sustained", p["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1])); smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------- CPU oracle leg
+
+def cpu_oracle_prefill(p: W.PrefillInputs, target_s: float = 12.0, max_tokens: int = 4096):
+    """Time the fp64 oracle on the first tokens of the same 64K sequence (all 48 heads,
+    conv included), sized to about ``target_s`` seconds. Returns (tok/s, threads, sample)."""
+    import oracle
+    sh = p.shape
+    threads = oracle.default_threads()
+
+    def run(n):
+        x = p.x[:n].float().numpy(); w = p.conv_w.float().numpy()
+        t0 = time.perf_counter()
+        oracle.layer_prefill(x, w, p.g[:n].numpy(), p.beta[:n].numpy(), sh.Hk, sh.Hv, sh.dk,
+                             sh.dv, n_threads=threads)
+        return time.perf_counter() - t0
+
+    n0 = 64
+    t_cal = run(n0)
+    n = int(min(max_tokens, max(n0, n0 * target_s / max(t_cal, 1e-6))))
+    dt = run(n)
+    return n / dt, threads, f"first {n} tokens of the 65536-token 27B-shaped sequence, all 48 heads, conv included"
+
+
+# --------------------------------------------------------------------------- main
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="gdn", choices=["gdn", "reference"])
+    ap.add_argument("--T", type=int, default=T_PREFILL)
+    ap.add_argument("--decode-batch", type=int, default=B_DECODE)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    return ap.parse_args()
+
+
+def dist_setup(n_gpus):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def max_over_ranks(v: float, world: int, dev) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    p = W.qwen35_27b_prefill(args.T)
+    vals, threads, sample = [], 0, ""
+    for i in range(args.warmup + args.steps):
+        v, threads, sample = cpu_oracle_prefill(p, target_s=3.0, max_tokens=1024)
+        if i >= args.warmup:
+            vals.append(v)
+    value = statistics.median(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, 27B-shaped)",
+            "config": {"workload": f"Qwen3.5-27B-shaped GDN layer prefill, T={args.T} (oracle sample)"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_setup(args.gpus)
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+
+    import gated_deltanet_mixer_causal_b200 as gdn
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    sh = SHAPE
+    hbm_gbs, tc_tflops, tc_sust, peak_src = measured_peaks()
+
+    # ---- inputs, resident in HBM before timing (each rank: its own seed offset)
+    p = W.make_prefill(sh, args.T, seed=2 + 1000 * rank, g_low=-0.3)
+    dcd = W.make_decode(sh, args.decode_batch, 1, seed=3 + 1000 * rank, g_low=-0.3)
+    x = p.x.to(dev); w = p.conv_w.to(dev); g = p.g.to(dev); beta = p.beta.to(dev)
+    T, Cc = x.shape
+    y = torch.empty_like(x)
+    o = torch.empty((T, sh.Hv, sh.dv), dtype=x.dtype, device=dev)
+    fin = torch.empty((1, sh.Hv, sh.dv, sh.dk), dtype=torch.float32, device=dev)
+    ws_n = gdn.gdn_chunk_prefill_workspace_size(T, 1, sh.Hk, sh.Hv, sh.dk, sh.dv, x.dtype)
+    ws = torch.empty(max(ws_n, 1), dtype=torch.uint8, device=dev)
+    dx = dcd.xs[0].to(dev); dg = dcd.gs[0].to(dev); db = dcd.betas[0].to(dev)
+    dcs = dcd.conv_state.to(dev); dst = dcd.state.to(dev); dw = dcd.conv_w.to(dev)
+    do = torch.empty((args.decode_batch, sh.Hv, sh.dv), dtype=x.dtype, device=dev)
+    q, k, v = gdn.qkv_views(y, sh.Hk, sh.Hv, sh.dk)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev):
+        ev[0].record(stream)
+        gdn.gdn_conv1d_silu(x, w, None, None, None, y)
+        ev[1].record(stream)
+        gdn.gdn_chunk_prefill(q, k, v, g, beta, None, None, fin, 1.0, True, o, ws)
+        ev[2].record(stream)
+        gdn.gdn_decode_step(dx, dw, dcs, dg, db, dst, sh.Hk, do)
+        ev[3].record(stream)
+
+    # launches of this library's kernels per step: conv 1, prefill (per path), decode 1
+    launches_per_step = 1 + gdn_prefill_launches() + 1
+
+    for _ in range(args.warmup):
+        step([torch.cuda.Event(enable_timing=True) for _ in range(4)])
+    torch.cuda.synchronize(dev)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    t_start = torch.cuda.Event(enable_timing=True); t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clk = clocks.stop()
+
+    total_ms = t_start.elapsed_time(t_end)
+    conv_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    pre_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    dec_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    total_ms = max_over_ranks(total_ms, world, dev)
+    layer_ms = max_over_ranks(sum(c + p_ for c, p_ in zip(conv_ms, pre_ms)), world, dev)
+    dec_sum = max_over_ranks(sum(dec_ms), world, dev)
+
+    value = world * T * args.steps / (layer_ms / 1e3)
+    conv_avg, pre_avg, dec_avg = (statistics.mean(conv_ms), statistics.mean(pre_ms),
+                                  statistics.mean(dec_ms))
+    dec_gbs = decode_bytes(args.decode_batch) / (dec_avg / 1e3) / 1e9
+    conv_gbs = conv_bytes(T) / (conv_avg / 1e3) / 1e9
+    pre_tflops = prefill_flops_per_token() * T / (pre_avg / 1e3) / 1e12
+
+    # dominant kernel: the prefill call (the chunked gated delta rule)
+    kernels = {"prefill": pre_avg, "conv": conv_avg, "decode": dec_avg}
+    dominant = max(kernels, key=kernels.get)
+    if dominant == "prefill":
+        roof = {"kernel": "gdn_chunk_prefill", "bound": "tensor", "achieved": pre_tflops,
+                "peak": tc_sust, "unit": "TFLOP/s", "frac": pre_tflops / tc_sust,
+                "peak_kind": f"bf16 dense sustained ({peak_src})",
+                "algorithmic_per_launch": prefill_flops_per_token() * T,
+                "traffic": TRAFFIC.get("prefill")}
+    elif dominant == "decode":
+        roof = {"kernel": "gdn_decode_step", "bound": "hbm", "achieved": dec_gbs, "peak": hbm_gbs,
+                "unit": "GB/s", "frac": dec_gbs / hbm_gbs, "peak_kind": f"HBM copy ({peak_src})",
+                "algorithmic_per_launch": decode_bytes(args.decode_batch),
+                "traffic": TRAFFIC.get("decode")}
+    else:
+        roof = {"kernel": "gdn_conv1d_silu", "bound": "hbm", "achieved": conv_gbs, "peak": hbm_gbs,
+                "unit": "GB/s", "frac": conv_gbs / hbm_gbs, "peak_kind": f"HBM copy ({peak_src})",
+                "algorithmic_per_launch": conv_bytes(T), "traffic": TRAFFIC.get("conv")}
+
+    # ---- end to end: host buffers in pinned memory, copies inside the timed region
+    e2e = None
+    if args.e2e_steps > 0:
+        hx = p.x.pin_memory(); hg = p.g.pin_memory(); hb = p.beta.pin_memory()
+        ho = torch.empty((T, sh.Hv, sh.dv), dtype=x.dtype).pin_memory()
+        hfin = torch.empty_like(fin, device="cpu").pin_memory()
+        hdx = dcd.xs[0].pin_memory(); hdg = dcd.gs[0].pin_memory(); hdb = dcd.betas[0].pin_memory()
+        hdo = torch.empty_like(do, device="cpu").pin_memory()
+
+        def e2e_step():
+            x.copy_(hx, non_blocking=True); g.copy_(hg, non_blocking=True)
+            beta.copy_(hb, non_blocking=True)
+            gdn.prefill_layer(x, w, g, beta, sh.Hk, sh.Hv, sh.dk, final_state=fin, y=y, o=o,
+                              workspace=ws)
+            ho.copy_(o, non_blocking=True); hfin.copy_(fin, non_blocking=True)
+            dx.copy_(hdx, non_blocking=True); dg.copy_(hdg, non_blocking=True)
+            db.copy_(hdb, non_blocking=True)
+            gdn.gdn_decode_step(dx, dw, dcs, dg, db, dst, sh.Hk, do)
+            hdo.copy_(do, non_blocking=True)
+
+        e2e_step(); torch.cuda.synchronize(dev)
+        barrier(world)
+        a = torch.cuda.Event(enable_timing=True); b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(a.elapsed_time(b), world, dev)
+        h2d = hx.numel() * 2 + hg.numel() * 4 + hb.numel() * 4 + hdx.numel() * 2 + hdg.numel() * 4 + hdb.numel() * 4
+        d2h = ho.numel() * 2 + hfin.numel() * 4 + hdo.numel() * 2
+        e2e = {"value": world * T * args.e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "note": "prefill tokens/s with the step's x, g, beta copied in from pinned host "
+                       "memory and o + final state copied out, decode step included"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v_cpu, threads, sample = cpu_oracle_prefill(p)
+        cpu = {"value": v_cpu, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; x~N(0,1), conv w~N(0,0.5), g~U[-0.3,0], beta=sigmoid(N(0,1)), decode state~N(0,0.02))",
+            "config": {"workload": f"Qwen3.5-27B-shaped GDN layer: prefill T={T} (Hk 16, Hv 48, d 128, "
+                                   f"conv 10240 ch) + decode step B={args.decode_batch}",
+                       "global_batch": world, "seq_len": T, "parallelism": f"dp{world}",
+                       "l2": "inputs larger than L2 (126 MB); no flush"},
+            "prefill": {"tokens_per_s": value, "conv_ms": conv_avg, "chunk_prefill_ms": pre_avg,
+                        "chunk_prefill_tflops": pre_tflops,
+                        "flops_per_token": prefill_flops_per_token(),
+                        "layer_ms": (conv_avg + pre_avg),
+                        "conv_gbs": conv_gbs, "conv_frac_hbm": conv_gbs / hbm_gbs},
+            "decode": {"value": dec_gbs, "unit": "GB/s", "us_per_step": dec_avg * 1e3,
+                       "frac_hbm": dec_gbs / hbm_gbs, "bytes_per_step": decode_bytes(args.decode_batch),
+                       "tokens_per_s": world * args.decode_batch / (dec_avg / 1e3)},
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def gdn_prefill_launches() -> int:
+    """Kernels one gdn_chunk_prefill call enqueues on the benchmark's path."""
+    return 1
+
+
+# DRAM traffic per launch from an ncu capture of the same kernel (bytes), or None when
+# the kernel changed since the counters were taken.
+TRAFFIC = {"prefill": None, "conv": None, "decode": None}
+
+if __name__ == "__main__":
+    main()

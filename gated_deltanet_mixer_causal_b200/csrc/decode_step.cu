@@ -1,0 +1,211 @@
+// decode_step.cu -- one token for each of B sequences, conv taps and fp32 states in place.
+//
+// Workload (Qwen3.5 page, section 8): decode is a state-update stream -- every token reads,
+// modifies and writes each fixed-size fp32 state. It is HBM-bound: per (sequence, value
+// head) the 128 x 128 state (64 KB) is read once and written once; nothing else is large.
+//
+// One CTA owns one (sequence b, key head hk): the conv channels of that key head's q and k
+// and of its G = Hv/Hk value heads. Owning the channels makes the in-place tap shift
+// race-free without a second kernel. After the conv, SiLU and the q/k L2 norm (in shared
+// memory), each warp streams whole state rows (value index i): a row is 128 floats, one
+// float4 per lane, so a warp access is 512 contiguous bytes. Per row, with s the old row:
+//   sk = s.k, sq = s.q                  (one two-value warp reduction)
+//   u  = beta (v_i - alpha sk)          (delta write strength for this row)
+//   s' = alpha s + u k                  (decay, then the write along k)
+//   o_i = scale (alpha sq + u (k.q))    (= s'.q without a second pass)
+#include "common.cuh"
+#include "launch.h"
+
+namespace gdn {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kRowUnroll = 4;      // rows per warp iteration (loads in flight)
+constexpr float kEps = 1e-6f;
+
+template <int VEC> struct RowIO;
+template <> struct RowIO<4> {
+  static __device__ __forceinline__ void load(const float* p, float (&s)[4]) {
+    float4 v = __ldcs(reinterpret_cast<const float4*>(p));
+    s[0] = v.x; s[1] = v.y; s[2] = v.z; s[3] = v.w;
+  }
+  static __device__ __forceinline__ void store(float* p, const float (&s)[4]) {
+    __stcs(reinterpret_cast<float4*>(p), make_float4(s[0], s[1], s[2], s[3]));
+  }
+};
+template <> struct RowIO<2> {
+  static __device__ __forceinline__ void load(const float* p, float (&s)[2]) {
+    float2 v = __ldcs(reinterpret_cast<const float2*>(p));
+    s[0] = v.x; s[1] = v.y;
+  }
+  static __device__ __forceinline__ void store(float* p, const float (&s)[2]) {
+    __stcs(reinterpret_cast<float2*>(p), make_float2(s[0], s[1]));
+  }
+};
+template <> struct RowIO<1> {
+  static __device__ __forceinline__ void load(const float* p, float (&s)[1]) { s[0] = __ldcs(p); }
+  static __device__ __forceinline__ void store(float* p, const float (&s)[1]) { __stcs(p, s[0]); }
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads)
+decode_step_kernel(const T* __restrict__ x, const T* __restrict__ conv_w, T* __restrict__ conv_state,
+                   const float* __restrict__ g, const float* __restrict__ beta,
+                   float* __restrict__ state, T* __restrict__ o, int32_t Hk, int32_t Hv,
+                   float scale) {
+  constexpr int VEC = D >= 32 ? D / 32 : 1;
+  const int G = Hv / Hk;
+  const int32_t Cc = 2 * Hk * D + Hv * D;
+  const int64_t b = blockIdx.x / Hk;
+  const int hk = blockIdx.x % Hk;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+
+  extern __shared__ float smem[];
+  float* ys = smem;                       // [(2 + G) * D]: q | k | v of the G heads
+  float* os = smem + (2 + G) * D;         // [G * D] outputs
+
+  // 1. conv + SiLU over this CTA's channels; shift the taps in place.
+  const int n_local = (2 + G) * D;
+  for (int lv = threadIdx.x; lv < n_local / 8; lv += kThreads) {
+    const int lc = lv * 8;
+    int gc;
+    if (lc < D) gc = hk * D + lc;
+    else if (lc < 2 * D) gc = Hk * D + hk * D + (lc - D);
+    else gc = 2 * Hk * D + hk * G * D + (lc - 2 * D);
+    float xv[8], t0[8], t1[8], t2[8], wr[32];
+    VecIO<T, 8>::load(x + b * Cc + gc, xv);
+    T* cs = conv_state + b * 3 * Cc + gc;
+    VecIO<T, 8>::load(cs, t0);
+    VecIO<T, 8>::load(cs + Cc, t1);
+    VecIO<T, 8>::load(cs + 2 * Cc, t2);
+    VecIO<T, 32>::load(conv_w + (int64_t)gc * 4, wr);
+    float yv[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float z = wr[i * 4 + 0] * t0[i];
+      z = fmaf(wr[i * 4 + 1], t1[i], z);
+      z = fmaf(wr[i * 4 + 2], t2[i], z);
+      z = fmaf(wr[i * 4 + 3], xv[i], z);
+      yv[i] = silu(z);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ys[lc + i] = yv[i];
+    VecIO<T, 8>::store(cs, t1);
+    VecIO<T, 8>::store(cs + Cc, t2);
+    VecIO<T, 8>::store(cs + 2 * Cc, xv);
+  }
+  __syncthreads();
+
+  // 2. L2-normalised q and k, per warp, in registers (VEC columns per lane).
+  const bool active = lane * VEC < D;
+  float qh[VEC], kh[VEC];
+  float qq = 0.f, kk = 0.f, kq = 0.f;
+#pragma unroll
+  for (int j = 0; j < VEC; ++j) {
+    qh[j] = active ? ys[lane * VEC + j] : 0.f;
+    kh[j] = active ? ys[D + lane * VEC + j] : 0.f;
+    qq = fmaf(qh[j], qh[j], qq);
+    kk = fmaf(kh[j], kh[j], kk);
+    kq = fmaf(kh[j], qh[j], kq);
+  }
+  qq = warp_sum(qq); kk = warp_sum(kk); kq = warp_sum(kq);
+  const float iq = 1.0f / sqrtf(qq + kEps), ik = 1.0f / sqrtf(kk + kEps);
+#pragma unroll
+  for (int j = 0; j < VEC; ++j) { qh[j] *= iq; kh[j] *= ik; }
+  const float kqh = kq * iq * ik;
+
+  // 3. stream the G * D state rows of this CTA.
+  const int rows = G * D;
+  for (int r0 = warp * kRowUnroll; r0 < rows; r0 += kWarps * kRowUnroll) {
+    float s[kRowUnroll][VEC];
+    float* ptr[kRowUnroll];
+#pragma unroll
+    for (int u = 0; u < kRowUnroll; ++u) {
+      const int r = r0 + u;
+      const int h = hk * G + r / D, i = r % D;
+      ptr[u] = state + ((b * Hv + h) * (int64_t)D + i) * D + lane * VEC;
+      if (r < rows && active) RowIO<VEC>::load(ptr[u], s[u]);
+      else {
+#pragma unroll
+        for (int j = 0; j < VEC; ++j) s[u][j] = 0.f;
+      }
+    }
+    float sk[kRowUnroll], sq[kRowUnroll];
+#pragma unroll
+    for (int u = 0; u < kRowUnroll; ++u) {
+      float a = 0.f, c = 0.f;
+#pragma unroll
+      for (int j = 0; j < VEC; ++j) { a = fmaf(s[u][j], kh[j], a); c = fmaf(s[u][j], qh[j], c); }
+      sk[u] = a; sq[u] = c;
+    }
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1)
+#pragma unroll
+      for (int u = 0; u < kRowUnroll; ++u) {
+        sk[u] += __shfl_xor_sync(0xffffffffu, sk[u], m);
+        sq[u] += __shfl_xor_sync(0xffffffffu, sq[u], m);
+      }
+#pragma unroll
+    for (int u = 0; u < kRowUnroll; ++u) {
+      const int r = r0 + u;
+      if (r >= rows) break;
+      const int h = hk * G + r / D;
+      const float alpha = expf(g[b * Hv + h]);
+      const float bt = beta[b * Hv + h];
+      const float uu = bt * (ys[2 * D + r] - alpha * sk[u]);
+#pragma unroll
+      for (int j = 0; j < VEC; ++j) s[u][j] = fmaf(alpha, s[u][j], uu * kh[j]);
+      if (active) RowIO<VEC>::store(ptr[u], s[u]);
+      if (lane == 0) os[r] = scale * fmaf(alpha, sq[u], uu * kqh);
+    }
+  }
+  __syncthreads();
+
+  // 4. outputs of the G heads are contiguous: o[b, hk*G .. hk*G+G-1, :]
+  T* ob = o + (b * Hv + (int64_t)hk * G) * D;
+  for (int e = threadIdx.x; e < rows; e += kThreads) ob[e] = from_f<T>(os[e]);
+}
+
+template <typename T, int D>
+cudaError_t launch_typed(const void* x, const void* w, void* cs, const float* g, const float* beta,
+                         float* state, void* o, int32_t B, int32_t Hk, int32_t Hv, float scale,
+                         cudaStream_t st) {
+  const int G = Hv / Hk;
+  const size_t smem = sizeof(float) * (size_t)((2 + G) * D + G * D);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(decode_step_kernel<T, D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  dim3 grid((unsigned)((int64_t)B * Hk));
+  decode_step_kernel<T, D><<<grid, kThreads, smem, st>>>(
+      (const T*)x, (const T*)w, (T*)cs, g, beta, state, (T*)o, Hk, Hv, scale);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_d(const void* x, const void* w, void* cs, const float* g, const float* beta,
+                     float* state, void* o, int32_t B, int32_t Hk, int32_t Hv, int32_t d,
+                     float scale, cudaStream_t st) {
+  switch (d) {
+    case 16: return launch_typed<T, 16>(x, w, cs, g, beta, state, o, B, Hk, Hv, scale, st);
+    case 32: return launch_typed<T, 32>(x, w, cs, g, beta, state, o, B, Hk, Hv, scale, st);
+    case 64: return launch_typed<T, 64>(x, w, cs, g, beta, state, o, B, Hk, Hv, scale, st);
+    default: return launch_typed<T, 128>(x, w, cs, g, beta, state, o, B, Hk, Hv, scale, st);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_decode_step(int dtype, const void* x, const void* conv_w, void* conv_state,
+                               const float* g, const float* beta, float* state, void* o,
+                               int32_t B, int32_t Hk, int32_t Hv, int32_t d, float scale,
+                               cudaStream_t stream) {
+  if (B == 0) return cudaSuccess;
+  if (dtype == kF32)
+    return launch_d<float>(x, conv_w, conv_state, g, beta, state, o, B, Hk, Hv, d, scale, stream);
+  return launch_d<bf16>(x, conv_w, conv_state, g, beta, state, o, B, Hk, Hv, d, scale, stream);
+}
+
+}  // namespace gdn

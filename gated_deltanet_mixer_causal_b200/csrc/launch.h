@@ -1,0 +1,32 @@
+// launch.h -- internal launchers behind the C ABI (gdn_api.cu). Each enqueues its kernels
+// on `stream` and returns cudaGetLastError(); arguments are validated by the caller.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace gdn {
+
+constexpr int kF32 = 0;   // GDN_F32
+constexpr int kBF16 = 1;  // GDN_BF16
+
+cudaError_t launch_conv1d_silu(int dtype, const void* x, void* y, const void* w,
+                               const int32_t* cu, int32_t n_seq, int64_t T, int32_t Cc,
+                               const void* conv_state_in, void* conv_state_out,
+                               cudaStream_t stream);
+
+cudaError_t launch_decode_step(int dtype, const void* x, const void* conv_w, void* conv_state,
+                               const float* g, const float* beta, float* state, void* o,
+                               int32_t B, int32_t Hk, int32_t Hv, int32_t d, float scale,
+                               cudaStream_t stream);
+
+// Token-by-token fp32 recurrence (SIMT): the fp32-activation prefill path.
+cudaError_t launch_prefill_recurrent(int dtype, const void* q, const void* k, const void* v,
+                                     const float* g, const float* beta, void* o, int64_t T,
+                                     int32_t Hk, int32_t Hv, int32_t d, int64_t qk_stride,
+                                     int64_t v_stride, const int32_t* cu, int32_t n_seq,
+                                     const float* init, float* final_state, float scale,
+                                     int32_t l2norm, cudaStream_t stream);
+
+}  // namespace gdn

@@ -1,0 +1,170 @@
+/*
+ * gdn.h -- C ABI of libgdn.so, the B200 (sm_100a) Gated DeltaNet token mixer.
+ *
+ * The mixer (from "Inside Qwen3.5: a hybrid linear + full attention LLM",
+ * romaanj.github.io/study/models/hybrid-attention, sections 2, 4, 5 and the config
+ * footnote; the ungated rule is in "Hybrid Mamba-Transformer MoE", sotaaz.com,
+ * section "Gated DeltaNet"):
+ *
+ *   y      = SiLU(depthwise causal conv, width 4, of x)           over q|k|v channels
+ *   q, k  <- q / sqrt(|q|^2 + 1e-6), k / sqrt(|k|^2 + 1e-6)      per token and key head
+ *   S_t    = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,  alpha_t = exp(g_t)
+ *   o_t    = scale * S_t q_t
+ *
+ * One recurrent state S (dv x dk, fp32, row index = value dimension) exists per sequence
+ * and value head. Value head h reads key head h / (Hv / Hk).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Pointers: device pointers unless stated; 16-byte aligned; tensors row-major and dense
+ *   unless a stride argument says otherwise. The caller owns every buffer, including the
+ *   workspace; the library allocates no device memory and keeps no state between calls.
+ * Streams: every call is asynchronous on `stream` (NULL = the legacy default stream) and
+ *   returns once its kernels are enqueued. Inputs must stay valid until they complete.
+ * Errors: arguments are validated before anything is launched; an invalid call returns a
+ *   status and launches nothing. Nothing is printed and no exception crosses the ABI.
+ *   gdn_last_error() gives a short reason for the calling thread's last failure.
+ *   A launch failure returns GDN_ERR_CUDA (and leaves the outputs undefined).
+ * Channel order of the conv input/output and of the decode input x:
+ *   [ q: Hk*dk | k: Hk*dk | v: Hv*dv ]  (Cc = 2*Hk*dk + Hv*dv).
+ * Supported shapes: dk = dv in {16, 32, 64, 128}; Hv a multiple of Hk; conv width 4.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t (the same handle type); NULL is the legacy default stream. */
+typedef struct CUstream_st* gdn_stream_t;
+
+typedef enum {
+  GDN_OK = 0,
+  GDN_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, aliasing, bad cu_seqlens */
+  GDN_ERR_UNSUPPORTED = 2,   /* valid but not built: head size, dtype, Hv % Hk != 0 */
+  GDN_ERR_WORKSPACE = 3,     /* workspace too small (see the *_workspace_size query) */
+  GDN_ERR_CUDA = 4,          /* a CUDA launch or runtime call failed */
+  GDN_ERR_TIMEOUT = 5        /* reserved: a bounded device-side wait gave up */
+} gdn_status_t;
+
+typedef enum {
+  GDN_F32 = 0,               /* fp32 activations (the state is always fp32) */
+  GDN_BF16 = 1               /* bf16 activations, fp32 math and state */
+} gdn_dtype_t;
+
+/* Static string naming a status code. Never NULL. */
+const char* gdn_status_string(gdn_status_t status);
+
+/* Reason for the calling thread's most recent non-OK status ("" if none). The pointer is
+ * valid until that thread's next call into the library. */
+const char* gdn_last_error(void);
+
+/* Library version, "major.minor.patch". */
+const char* gdn_version(void);
+
+/*
+ * gdn_conv1d_silu -- width-4 depthwise causal conv followed by SiLU (prefill).
+ *
+ * Defined by the Qwen3.5 page, section 5 (the short kernel-4 causal convolution that
+ * gives the recurrence local mixing) and its config footnote (conv kernel 4); SiLU
+ * z / (1 + e^-z) follows the conv on every channel.
+ *
+ *   y[t, c] = SiLU( sum_{j=0..3} w[c, j] * x[t - 3 + j, c] )
+ *
+ * x, y            [T, Cc], dtype dt. y must not overlap x.
+ * w               [Cc, 4], dtype dt; w[c, 3] multiplies the current token (PyTorch
+ *                 cross-correlation order), no bias.
+ * cu_seqlens      device int32 [n_seq + 1], cu[0] = 0, cu[n_seq] = T, non-decreasing;
+ *                 every sequence restarts its window. NULL means one sequence of length T
+ *                 (n_seq is then ignored and taken as 1).
+ * conv_state_in   [n_seq, 3, Cc] dtype dt, the three inputs preceding each sequence
+ *                 (oldest first), or NULL for zeros.
+ * conv_state_out  [n_seq, 3, Cc] dtype dt, receives the last three inputs of each
+ *                 sequence (reaching into conv_state_in for sequences shorter than 3),
+ *                 or NULL. Must not overlap conv_state_in.
+ * Returns GDN_OK, GDN_ERR_INVALID_ARG (T < 0, Cc <= 0 or Cc % 8 != 0, bad pointers),
+ * GDN_ERR_UNSUPPORTED (dtype), GDN_ERR_CUDA. T = 0 is valid and launches only what
+ * conv_state_out needs.
+ */
+gdn_status_t gdn_conv1d_silu(const void* x, void* y, gdn_dtype_t dt, const void* w,
+                             const int32_t* cu_seqlens, int32_t n_seq, int64_t T, int32_t Cc,
+                             const void* conv_state_in, void* conv_state_out,
+                             gdn_stream_t stream);
+
+/*
+ * gdn_chunk_prefill_workspace_size -- bytes of device workspace gdn_chunk_prefill needs
+ * for these sizes (0 is a valid answer). Returns SIZE_MAX for unsupported shapes.
+ */
+size_t gdn_chunk_prefill_workspace_size(int64_t T, int32_t n_seq, int32_t Hk, int32_t Hv,
+                                        int32_t dk, int32_t dv, gdn_dtype_t dt);
+
+/*
+ * gdn_chunk_prefill -- the gated delta rule over packed sequences (prefill).
+ *
+ * Defined by the Qwen3.5 page, section 5: S <- alpha S + beta (v - S k) k^T read as
+ * decay then delta write (equivalently S_t = alpha_t S_{t-1}(I - beta_t k_t k_t^T) +
+ * beta_t v_t k_t^T), the L2 norm on q and k, alpha and beta per token and per head;
+ * section 2 for the read-out o = S q. The kernels evaluate it chunk by chunk (the
+ * WY/UT form of the same recurrence); results equal the token-by-token recurrence up to
+ * rounding.
+ *
+ * q, k        token t, key head j at q + t*qk_stride + j*dk (elements), dtype dt.
+ * v           token t, value head h at v + t*v_stride + h*dv, dtype dt.
+ *             qk_stride = 0 means Hk*dk, v_stride = 0 means Hv*dv (dense). Strides let
+ *             q/k/v be views into gdn_conv1d_silu's output (stride Cc, no copy).
+ * g           [T, Hv] fp32 log-decay (alpha = exp(g), g <= 0 expected, not checked).
+ * beta        [T, Hv] fp32 write strength.
+ * o           [T, Hv, dv] dtype dt, written. Must not overlap any input.
+ * cu_seqlens  device int32 [n_seq + 1] as for gdn_conv1d_silu, or NULL (one sequence).
+ * initial_state  fp32 [n_seq, Hv, dv, dk] or NULL (zeros).
+ * final_state    fp32 [n_seq, Hv, dv, dk] or NULL (not written). May equal
+ *                initial_state (updated in place); must not partially overlap it.
+ * scale       multiplies o (1.0 for the plain o = S q).
+ * qk_l2norm   1: normalise q and k as above; 0: use them as given.
+ * workspace   device memory of at least gdn_chunk_prefill_workspace_size(...) bytes,
+ *             256-byte aligned, or NULL when that size is 0. Contents on entry are
+ *             ignored; the caller must not use it concurrently with the call.
+ * Returns GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_WORKSPACE, GDN_ERR_CUDA.
+ */
+gdn_status_t gdn_chunk_prefill(const void* q, const void* k, const void* v,
+                               const float* g, const float* beta, void* o,
+                               gdn_dtype_t dt, int64_t T, int32_t Hk, int32_t Hv,
+                               int32_t dk, int32_t dv, int64_t qk_stride, int64_t v_stride,
+                               const int32_t* cu_seqlens, int32_t n_seq,
+                               const float* initial_state, float* final_state,
+                               float scale, int32_t qk_l2norm,
+                               void* workspace, size_t workspace_bytes, gdn_stream_t stream);
+
+/*
+ * gdn_decode_step -- one token for each of B sequences, state updated in place.
+ *
+ * Defined by the Qwen3.5 page, section 8 (decode becomes a state-update workload:
+ * fixed-size fp32 state read, modified and written every token) with the update of
+ * section 5 and the conv of the config footnote. Per sequence b:
+ *   z_c = w[c,0] cs[b,0,c] + w[c,1] cs[b,1,c] + w[c,2] cs[b,2,c] + w[c,3] x[b,c]; y = SiLU(z)
+ *   cs[b] <- [cs[b,1], cs[b,2], x[b]]             (taps shift by one, in place)
+ *   q, k, v from y (channel order above), q and k L2-normalised
+ *   S[b,h] <- alpha S[b,h] (I - beta k k^T) + beta v k^T;  o[b,h] = scale * S[b,h] q
+ *
+ * x           [B, Cc] dtype dt, this step's pre-conv q|k|v.
+ * conv_w      [Cc, 4] dtype dt.
+ * conv_state  [B, 3, Cc] dtype dt, read and updated in place.
+ * g, beta     [B, Hv] fp32.
+ * state       [B, Hv, dv, dk] fp32, read and updated in place.
+ * o           [B, Hv, dv] dtype dt.
+ * Returns GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA. B = 0 is a no-op.
+ */
+gdn_status_t gdn_decode_step(const void* x, const void* conv_w, void* conv_state,
+                             const float* g, const float* beta, float* state, void* o,
+                             gdn_dtype_t dt, int32_t B, int32_t Hk, int32_t Hv,
+                             int32_t dk, int32_t dv, float scale, gdn_stream_t stream);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* GDN_H_ */

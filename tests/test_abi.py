@@ -1,0 +1,127 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every
+function include/gdn.h declares, and rejects invalid arguments before launching.
+
+Invalid calls return before any CUDA call, so fake device addresses are safe here.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_deltanet_mixer_causal_b200 as gdn
+from gated_deltanet_mixer_causal_b200 import _lib
+from gated_deltanet_mixer_causal_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+FAKE = 0x7f0000000000        # 16-byte aligned, never dereferenced (validation fails first)
+
+
+@pytest.fixture(scope="module")
+def L():
+    build()
+    return _lib.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w\*\s]+?\b(gdn_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ["gdn_conv1d_silu", "gdn_chunk_prefill", "gdn_chunk_prefill_workspace_size",
+              "gdn_decode_step", "gdn_status_string", "gdn_last_error", "gdn_version"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), f"{name} declared in gdn.h but not exported"
+        assert name in _lib.SIGNATURES, f"{name} has no Python binding"
+
+
+def test_status_strings(L):
+    for code, name in enumerate(["GDN_OK", "GDN_ERR_INVALID_ARG", "GDN_ERR_UNSUPPORTED",
+                                 "GDN_ERR_WORKSPACE", "GDN_ERR_CUDA", "GDN_ERR_TIMEOUT"]):
+        assert L.gdn_status_string(code).decode() == name
+    assert L.gdn_version().decode().count(".") == 2
+
+
+def _conv(L, **kw):
+    a = dict(x=FAKE, y=FAKE + (1 << 30), dt=1, w=FAKE + (2 << 30), cu=None, n=1, T=64, Cc=64,
+             sin=None, sout=None)
+    a.update(kw)
+    return L.gdn_conv1d_silu(a["x"], a["y"], a["dt"], a["w"], a["cu"], a["n"], a["T"], a["Cc"],
+                             a["sin"], a["sout"], None)
+
+
+def test_conv_validation(L):
+    assert _conv(L, T=-1) == _lib.GDN_ERR_INVALID_ARG
+    assert _conv(L, Cc=12) == _lib.GDN_ERR_INVALID_ARG
+    assert _conv(L, dt=7) == _lib.GDN_ERR_UNSUPPORTED
+    assert _conv(L, x=None) == _lib.GDN_ERR_INVALID_ARG
+    assert _conv(L, y=FAKE + 8) == _lib.GDN_ERR_INVALID_ARG             # misaligned
+    assert _conv(L, y=FAKE + 64) == _lib.GDN_ERR_INVALID_ARG            # overlaps x
+    assert "overlaps" in L.gdn_last_error().decode()
+    assert _conv(L, sin=FAKE + (3 << 30), sout=FAKE + (3 << 30) + 16) == _lib.GDN_ERR_INVALID_ARG
+    assert _conv(L, cu=FAKE + (4 << 30), n=0) == _lib.GDN_ERR_INVALID_ARG
+
+
+def _prefill(L, **kw):
+    a = dict(q=FAKE, k=FAKE + (1 << 30), v=FAKE + (2 << 30), g=FAKE + (3 << 30),
+             b=FAKE + (4 << 30), o=FAKE + (5 << 30), dt=1, T=100, Hk=2, Hv=4, dk=64, dv=64,
+             qks=0, vs=0, cu=None, n=1, init=None, fin=None, ws=None, wsb=0)
+    a.update(kw)
+    return L.gdn_chunk_prefill(a["q"], a["k"], a["v"], a["g"], a["b"], a["o"], a["dt"], a["T"],
+                               a["Hk"], a["Hv"], a["dk"], a["dv"], a["qks"], a["vs"], a["cu"],
+                               a["n"], a["init"], a["fin"], 1.0, 1, a["ws"], a["wsb"], None)
+
+
+def test_prefill_validation(L):
+    assert _prefill(L, dk=48, dv=48) == _lib.GDN_ERR_UNSUPPORTED
+    assert _prefill(L, dk=64, dv=128) == _lib.GDN_ERR_UNSUPPORTED
+    assert _prefill(L, Hv=3) == _lib.GDN_ERR_UNSUPPORTED
+    assert _prefill(L, Hk=0) == _lib.GDN_ERR_INVALID_ARG
+    assert _prefill(L, T=-5) == _lib.GDN_ERR_INVALID_ARG
+    assert _prefill(L, qks=100) == _lib.GDN_ERR_INVALID_ARG           # shorter than a row
+    assert _prefill(L, qks=132) == _lib.GDN_ERR_INVALID_ARG           # not a multiple of 8
+    assert _prefill(L, g=None) == _lib.GDN_ERR_INVALID_ARG
+    assert _prefill(L, o=FAKE + 4) == _lib.GDN_ERR_INVALID_ARG        # misaligned
+    assert _prefill(L, o=FAKE + (2 << 30) + 512) == _lib.GDN_ERR_INVALID_ARG   # o overlaps v
+    st = FAKE + (6 << 30)
+    assert _prefill(L, init=st, fin=st + 4096) == _lib.GDN_ERR_INVALID_ARG    # partial overlap
+    need = L.gdn_chunk_prefill_workspace_size(100, 1, 2, 4, 64, 64, 1)
+    if need > 0:
+        assert _prefill(L, wsb=need - 1, ws=FAKE + (7 << 30)) == _lib.GDN_ERR_WORKSPACE
+    assert L.gdn_chunk_prefill_workspace_size(100, 1, 2, 3, 64, 64, 1) == ctypes.c_size_t(-1).value
+
+
+def _decode(L, **kw):
+    a = dict(x=FAKE, w=FAKE + (1 << 30), cs=FAKE + (2 << 30), g=FAKE + (3 << 30),
+             b=FAKE + (4 << 30), st=FAKE + (5 << 30), o=FAKE + (6 << 30), dt=1, B=8, Hk=2, Hv=4,
+             dk=32, dv=32)
+    a.update(kw)
+    return L.gdn_decode_step(a["x"], a["w"], a["cs"], a["g"], a["b"], a["st"], a["o"], a["dt"],
+                             a["B"], a["Hk"], a["Hv"], a["dk"], a["dv"], 1.0, None)
+
+
+def test_decode_validation(L):
+    assert _decode(L, B=-1) == _lib.GDN_ERR_INVALID_ARG
+    assert _decode(L, B=0) == _lib.GDN_OK                       # no-op, nothing launched
+    assert _decode(L, dk=24, dv=24) == _lib.GDN_ERR_UNSUPPORTED
+    assert _decode(L, Hv=5) == _lib.GDN_ERR_UNSUPPORTED
+    assert _decode(L, st=None) == _lib.GDN_ERR_INVALID_ARG
+    assert _decode(L, o=FAKE + (5 << 30) + 128) == _lib.GDN_ERR_INVALID_ARG   # o inside state
+    assert _decode(L, cs=FAKE + 16) == _lib.GDN_ERR_INVALID_ARG               # conv_state over x
+
+
+def test_python_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(8, 64, dtype=torch.bfloat16)
+    w = torch.zeros(64, 4, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        gdn.gdn_conv1d_silu(x, w)

@@ -1,0 +1,289 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the same
+seeded inputs.
+
+Small cases are compared element by element and span several chunks and a ragged tail;
+the full-size workloads run in the benchmark's launch configuration and are compared on
+sampled heads/sequences that the oracle computes on its own.
+"""
+import numpy as np
+import pytest
+import torch
+
+import gated_deltanet_mixer_causal_b200 as gdn
+from gated_deltanet_mixer_causal_b200 import workloads as W
+import oracle
+from parity import (BF16_TOL, FP32_TOL, frob_rel, max_rel, np64, oracle_layer_heads, worst_head_o,
+                    worst_head_state)
+
+pytestmark = pytest.mark.gpu
+
+_CACHE = {}
+
+
+def cached(name, fn):
+    """Large seeded workloads are generated once per session."""
+    if name not in _CACHE:
+        _CACHE[name] = fn()
+    return _CACHE[name]
+
+
+def to_dev(t, dev):
+    return None if t is None else t.to(dev)
+
+
+def run_layer(p, dev, conv_state_in=None, want_conv_state=False):
+    sh = p.shape
+    x = p.x.to(dev)
+    cu = to_dev(p.cu_seqlens, dev)
+    init = to_dev(p.initial_state, dev)
+    fin = torch.empty((p.n_seq, sh.Hv, sh.dv, sh.dk), dtype=torch.float32, device=dev)
+    cs_out = (torch.empty((p.n_seq, 3, sh.conv_channels), dtype=x.dtype, device=dev)
+              if want_conv_state else None)
+    o = gdn.prefill_layer(x, p.conv_w.to(dev), p.g.to(dev), p.beta.to(dev), sh.Hk, sh.Hv, sh.dk,
+                          cu, init, to_dev(conv_state_in, dev), fin, cs_out)
+    torch.cuda.synchronize()
+    return o, fin, cs_out
+
+
+# ------------------------------------------------------------------ fp32 tiny gate
+
+def test_tiny_recurrence_fp32(cuda_device):
+    r = W.tiny_recurrence()
+    o_ref, f_ref = oracle.recurrence(r.q.numpy(), r.k.numpy(), r.v.numpy(), r.g.numpy(),
+                                     r.beta.numpy())
+    fin = torch.empty((1, 2, 16, 16), device=cuda_device)
+    o = gdn.gdn_chunk_prefill(r.q.to(cuda_device), r.k.to(cuda_device), r.v.to(cuda_device),
+                              r.g.to(cuda_device), r.beta.to(cuda_device), final_state=fin)
+    assert max_rel(np64(o), o_ref) <= FP32_TOL
+    assert max_rel(np64(fin), f_ref) <= FP32_TOL
+
+
+def test_tiny_layer_fp32(cuda_device):
+    p = W.tiny_layer()
+    sh = p.shape
+    o_ref, f_ref, cs_ref = oracle.layer_prefill(p.x.numpy(), p.conv_w.numpy(), p.g.numpy(),
+                                                p.beta.numpy(), sh.Hk, sh.Hv, sh.dk, sh.dv)
+    o, fin, cs = run_layer(p, cuda_device, want_conv_state=True)
+    assert max_rel(np64(o), o_ref) <= FP32_TOL
+    assert max_rel(np64(fin), f_ref) <= FP32_TOL
+    np.testing.assert_array_equal(np64(cs), cs_ref)
+
+
+# ----------------------------------------------------------------------------- conv
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_conv_varlen_edges(cuda_device, dtype):
+    """Empty, 1-, 2-, 3-token sequences, run boundaries (31/32/33) and a ragged tail,
+    with carried taps in and out."""
+    rng = np.random.default_rng(21)
+    lengths = [0, 1, 2, 3, 31, 32, 33, 0, 100, 5]
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    T, Cc = int(cu[-1]), 96
+    x = torch.from_numpy(rng.standard_normal((T, Cc), dtype=np.float32)).to(dtype)
+    w = torch.from_numpy(rng.standard_normal((Cc, 4), dtype=np.float32) * 0.5).to(dtype)
+    s_in = torch.from_numpy(rng.standard_normal((len(lengths), 3, Cc), dtype=np.float32)).to(dtype)
+    y_ref, s_ref = oracle.conv1d_silu(np64(x), np64(w), cu, np64(s_in), return_state=True)
+    s_out = torch.empty_like(s_in, device=cuda_device)
+    y = gdn.gdn_conv1d_silu(x.to(cuda_device), w.to(cuda_device),
+                            torch.from_numpy(cu).to(cuda_device), s_in.to(cuda_device), s_out)
+    torch.cuda.synchronize()
+    rtol = 2.0 ** -8 if dtype == torch.bfloat16 else 1e-5
+    np.testing.assert_allclose(np64(y), y_ref, rtol=rtol, atol=1e-6)
+    np.testing.assert_array_equal(np64(s_out), s_ref)
+
+
+def test_conv_full_27b_rows(cuda_device):
+    """The 27B-shaped conv at T=65536 in the benchmark's configuration; the oracle checks
+    sampled token rows (each row needs only its three predecessors)."""
+    p = cached('27b', W.qwen35_27b_prefill)
+    y = gdn.gdn_conv1d_silu(p.x.to(cuda_device), p.conv_w.to(cuda_device))
+    torch.cuda.synchronize()
+    for t in [0, 1, 2, 3, 4095, 32768, 65535]:
+        lo = max(0, t - 3)
+        y_ref = oracle.conv1d_silu(p.x[lo:t + 1].float().numpy(), p.conv_w.float().numpy())
+        # rows before t are reconstructed from a window starting at lo, so only row t is exact
+        if lo == 0:
+            ref = y_ref[t]
+        else:
+            ref = y_ref[-1]
+        np.testing.assert_allclose(np64(y[t]), ref, rtol=2.0 ** -8, atol=1e-6)
+
+
+# --------------------------------------------------------------------- bf16 prefill
+
+def test_prefill_bf16_ragged_9b_shape(cuda_device):
+    """9B-shaped heads, T = 300 (several chunks plus a ragged tail), every head compared."""
+    p = W.make_prefill(W.QWEN35_9B, 300, seed=31, g_low=-0.5)
+    sh = p.shape
+    o_ref, f_ref, _ = oracle.layer_prefill(p.x.float().numpy(), p.conv_w.float().numpy(),
+                                           p.g.numpy(), p.beta.numpy(), sh.Hk, sh.Hv, sh.dk, sh.dv)
+    o, fin, _ = run_layer(p, cuda_device)
+    assert worst_head_o(np64(o), o_ref, None) <= BF16_TOL
+    assert worst_head_state(np64(fin), f_ref) <= BF16_TOL
+
+
+def test_prefill_bf16_varlen_with_state(cuda_device):
+    """27B-shaped heads, packed sequences of 1, 64, 65, 130, 7 and 0 tokens, nonzero
+    initial states and carried conv taps; every sequence and head compared."""
+    lengths = [1, 64, 65, 130, 7, 0]
+    p = W.make_prefill(W.QWEN35_27B, 0, seed=32, g_low=-0.3, init_std=0.02, lengths=lengths)
+    sh = p.shape
+    rng = np.random.default_rng(33)
+    cs_in = torch.from_numpy(rng.standard_normal((len(lengths), 3, sh.conv_channels),
+                                                 dtype=np.float32)).to(torch.bfloat16)
+    cu = p.cu_seqlens.numpy()
+    o_ref, f_ref, cs_ref = oracle.layer_prefill(p.x.float().numpy(), p.conv_w.float().numpy(),
+                                                p.g.numpy(), p.beta.numpy(), sh.Hk, sh.Hv,
+                                                sh.dk, sh.dv, cu, p.initial_state.numpy(),
+                                                cs_in.float().numpy())
+    o, fin, cs = run_layer(p, cuda_device, conv_state_in=cs_in, want_conv_state=True)
+    assert worst_head_o(np64(o), o_ref, cu) <= BF16_TOL
+    assert worst_head_state(np64(fin), f_ref) <= BF16_TOL
+    np.testing.assert_array_equal(np64(fin)[5], p.initial_state.numpy()[5])   # empty sequence
+    np.testing.assert_array_equal(np64(cs), cs_ref)
+
+
+def test_prefill_final_state_in_place(cuda_device):
+    p = W.make_prefill(W.QWEN35_9B, 70, seed=34, init_std=0.02)
+    sh = p.shape
+    o_ref, f_ref, _ = oracle.layer_prefill(p.x.float().numpy(), p.conv_w.float().numpy(),
+                                           p.g.numpy(), p.beta.numpy(), sh.Hk, sh.Hv, sh.dk, sh.dv,
+                                           None, p.initial_state.numpy())
+    st = p.initial_state.to(cuda_device).clone()
+    o = gdn.prefill_layer(p.x.to(cuda_device), p.conv_w.to(cuda_device), p.g.to(cuda_device),
+                          p.beta.to(cuda_device), sh.Hk, sh.Hv, sh.dk, initial_state=st,
+                          final_state=st)
+    torch.cuda.synchronize()
+    assert worst_head_o(np64(o), o_ref, None) <= BF16_TOL
+    assert worst_head_state(np64(st), f_ref) <= BF16_TOL
+
+
+def test_prefill_empty_batch_passes_state(cuda_device):
+    sh = W.QWEN35_9B
+    init = torch.randn(1, sh.Hv, sh.dv, sh.dk, device=cuda_device)
+    fin = torch.empty_like(init)
+    e = torch.empty((0, sh.Hk, sh.dk), dtype=torch.bfloat16, device=cuda_device)
+    ev = torch.empty((0, sh.Hv, sh.dv), dtype=torch.bfloat16, device=cuda_device)
+    eg = torch.empty((0, sh.Hv), dtype=torch.float32, device=cuda_device)
+    gdn.gdn_chunk_prefill(e, e, ev, eg, eg, initial_state=init, final_state=fin)
+    torch.cuda.synchronize()
+    assert torch.equal(fin, init)
+
+
+def test_prefill_9b_full(cuda_device):
+    """Qwen3.5-9B-shaped layer, T = 8192, every head against the oracle."""
+    p = W.qwen35_9b_prefill()
+    sh = p.shape
+    o, fin, _ = run_layer(p, cuda_device)
+    o_ref, f_ref, _ = oracle.layer_prefill(p.x.float().numpy(), p.conv_w.float().numpy(),
+                                           p.g.numpy(), p.beta.numpy(), sh.Hk, sh.Hv, sh.dk, sh.dv)
+    assert worst_head_o(np64(o), o_ref, None) <= BF16_TOL
+    assert worst_head_state(np64(fin), f_ref) <= BF16_TOL
+
+
+def test_prefill_27b_64k_sampled_heads(cuda_device):
+    """Qwen3.5-27B-shaped layer at T = 65536 (the benchmark workload); value heads 0, 25
+    and 47 (key heads 0, 8, 15) against the oracle over the whole sequence."""
+    p = cached('27b', W.qwen35_27b_prefill)
+    o, fin, _ = run_layer(p, cuda_device)
+    heads = [0, 25, 47]
+    ref = oracle_layer_heads(p, heads)
+    o_np, f_np = np64(o), np64(fin)
+    for h in heads:
+        o_r, f_r = ref[(0, h)]
+        assert frob_rel(o_np[:, h], o_r) <= BF16_TOL, h
+        assert frob_rel(f_np[0, h], f_r) <= BF16_TOL, h
+
+
+def test_prefill_27b_varlen_sampled(cuda_device):
+    """32 packed sequences (log-uniform lengths, nonzero initial states): the shortest
+    sequence on every head and the longest on two heads."""
+    p = W.qwen35_27b_varlen()
+    o, fin, _ = run_layer(p, cuda_device)
+    cu = p.cu_seqlens.numpy()
+    lens = np.diff(cu)
+    short, long_ = int(np.argmin(lens)), int(np.argmax(lens))
+    o_np, f_np = np64(o), np64(fin)
+    checks = [(short, list(range(p.shape.Hv))), (long_, [7, 40])]
+    for n, heads in checks:
+        ref = oracle_layer_heads(p, heads, seqs=[n])
+        a, b = int(cu[n]), int(cu[n + 1])
+        for h in heads:
+            o_r, f_r = ref[(n, h)]
+            assert frob_rel(o_np[a:b, h], o_r) <= BF16_TOL, (n, h)
+            assert frob_rel(f_np[n, h], f_r) <= BF16_TOL, (n, h)
+
+
+# --------------------------------------------------------------------------- decode
+
+def test_decode_fp32_small(cuda_device):
+    d = W.make_decode(W.LayerShape(2, 4, 32, 32), B=3, steps=5, seed=41, dtype=torch.float32)
+    sh = d.shape
+    cs = d.conv_state.to(cuda_device).clone()
+    st = d.state.to(cuda_device).clone()
+    cs_r, st_r = d.conv_state.numpy().astype(np.float64), d.state.numpy().astype(np.float64)
+    w = d.conv_w.to(cuda_device)
+    for t in range(5):
+        o = gdn.gdn_decode_step(d.xs[t].to(cuda_device), w, cs, d.gs[t].to(cuda_device),
+                                d.betas[t].to(cuda_device), st, sh.Hk)
+        o_r, st_r, cs_r = oracle.decode_step(d.xs[t].numpy(), d.conv_w.numpy(), cs_r,
+                                             d.gs[t].numpy(), d.betas[t].numpy(), st_r, sh.Hk,
+                                             sh.Hv, sh.dk, sh.dv)
+        torch.cuda.synchronize()
+        assert max_rel(np64(o), o_r) <= FP32_TOL
+        assert max_rel(np64(st), st_r) <= FP32_TOL
+        np.testing.assert_array_equal(np64(cs), cs_r)
+
+
+def test_decode_27b_batch256_100_steps(cuda_device):
+    """The 27B decode workload (B = 256, 100 steps, states updated in place); sequences
+    0, 131 and 255 against the oracle after every 10th step."""
+    d = W.qwen35_27b_decode()
+    sh = d.shape
+    sample = [0, 131, 255]
+    cs = d.conv_state.to(cuda_device).clone()
+    st = d.state.to(cuda_device).clone()
+    w = d.conv_w.to(cuda_device)
+    cs_r = d.conv_state.float().numpy()[sample].astype(np.float64)
+    st_r = d.state.numpy()[sample].astype(np.float64)
+    for t in range(100):
+        o = gdn.gdn_decode_step(d.xs[t].to(cuda_device), w, cs, d.gs[t].to(cuda_device),
+                                d.betas[t].to(cuda_device), st, sh.Hk)
+        o_r, st_r, cs_r = oracle.decode_step(d.xs[t].float().numpy()[sample],
+                                             d.conv_w.float().numpy(), cs_r,
+                                             d.gs[t].numpy()[sample], d.betas[t].numpy()[sample],
+                                             st_r, sh.Hk, sh.Hv, sh.dk, sh.dv)
+        if (t + 1) % 10 == 0:
+            torch.cuda.synchronize()
+            o_g = np64(o)[sample]
+            st_g = np64(st[sample])
+            for j in range(len(sample)):
+                for h in range(sh.Hv):
+                    assert frob_rel(o_g[j, h], o_r[j, h]) <= BF16_TOL, (t, j, h)
+                    assert frob_rel(st_g[j, h], st_r[j, h]) <= BF16_TOL, (t, j, h)
+            np.testing.assert_array_equal(np64(cs[sample]), cs_r)
+
+
+def test_decode_matches_prefill_on_gpu(cuda_device):
+    """Eight decode steps equal a prefill of the same eight tokens from the same states
+    (both on the GPU; bf16 tolerance)."""
+    sh = W.LayerShape(2, 6, 64, 64)
+    d = W.make_decode(sh, B=2, steps=8, seed=42)
+    cs = d.conv_state.to(cuda_device).clone()
+    st = d.state.to(cuda_device).clone()
+    w = d.conv_w.to(cuda_device)
+    outs = []
+    for t in range(8):
+        outs.append(gdn.gdn_decode_step(d.xs[t].to(cuda_device), w, cs, d.gs[t].to(cuda_device),
+                                        d.betas[t].to(cuda_device), st, sh.Hk))
+    x = torch.stack(d.xs, 1).reshape(16, -1).to(cuda_device)
+    g = torch.stack(d.gs, 1).reshape(16, -1).to(cuda_device)
+    b = torch.stack(d.betas, 1).reshape(16, -1).to(cuda_device)
+    cu = torch.tensor([0, 8, 16], dtype=torch.int32, device=cuda_device)
+    fin = torch.empty_like(st)
+    o_p = gdn.prefill_layer(x, w, g, b, sh.Hk, sh.Hv, sh.dk, cu, d.state.to(cuda_device),
+                            d.conv_state.to(cuda_device), fin)
+    torch.cuda.synchronize()
+    o_d = torch.stack(outs, 1).reshape(16, sh.Hv, sh.dv)
+    assert worst_head_o(np64(o_d), np64(o_p), [0, 8, 16]) <= BF16_TOL
+    assert worst_head_state(np64(st), np64(fin)) <= BF16_TOL
