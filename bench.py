@@ -378,8 +378,9 @@ def main():
 
 
 def gdn_prefill_launches() -> int:
-    """Kernels one gdn_chunk_prefill call enqueues on the benchmark's path."""
-    return 1
+    """Kernels one gdn_chunk_prefill call enqueues on the benchmark's path (bf16, d = 128):
+    the chunk plan, the intra-chunk kernel and the chain kernel."""
+    return 3
 
 
 # DRAM traffic per launch from an ncu capture of the same kernel (bytes), or None when

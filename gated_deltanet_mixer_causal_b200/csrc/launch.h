@@ -29,4 +29,13 @@ cudaError_t launch_prefill_recurrent(int dtype, const void* q, const void* k, co
                                      const float* init, float* final_state, float scale,
                                      int32_t l2norm, cudaStream_t stream);
 
+// Chunked WY/UT prefill on tcgen05 (bf16 activations, dk = dv = 128). Needs
+// prefill_chunk_tc_workspace(...) bytes of workspace.
+size_t prefill_chunk_tc_workspace(int64_t T, int32_t n_seq, int32_t Hv);
+cudaError_t launch_prefill_chunk_tc(const void* q, const void* k, const void* v, const float* g,
+                                    const float* beta, void* o, int64_t T, int32_t Hk, int32_t Hv,
+                                    int64_t qk_stride, int64_t v_stride, const int32_t* cu,
+                                    int32_t n_seq, const float* init, float* fin, float scale,
+                                    void* workspace, cudaStream_t stream);
+
 }  // namespace gdn

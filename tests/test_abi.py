@@ -98,6 +98,14 @@ def test_prefill_validation(L):
     if need > 0:
         assert _prefill(L, wsb=need - 1, ws=FAKE + (7 << 30)) == _lib.GDN_ERR_WORKSPACE
     assert L.gdn_chunk_prefill_workspace_size(100, 1, 2, 3, 64, 64, 1) == ctypes.c_size_t(-1).value
+    # the bf16 tensor-core path (d = 128) needs workspace; short workspace is refused
+    need = L.gdn_chunk_prefill_workspace_size(100, 1, 2, 4, 128, 128, 1)
+    assert need > 0
+    assert L.gdn_chunk_prefill_workspace_size(100, 1, 2, 4, 128, 128, 0) == 0   # fp32: none
+    ws = FAKE + (7 << 30)
+    assert _prefill(L, dk=128, dv=128, ws=ws, wsb=need - 1) == _lib.GDN_ERR_WORKSPACE
+    assert _prefill(L, dk=128, dv=128, ws=None, wsb=need) == _lib.GDN_ERR_WORKSPACE
+    assert _prefill(L, dk=128, dv=128, ws=ws + 16, wsb=need) == _lib.GDN_ERR_INVALID_ARG  # not 256-aligned
 
 
 def _decode(L, **kw):
