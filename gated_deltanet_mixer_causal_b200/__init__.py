@@ -14,11 +14,12 @@ from typing import Optional
 
 import torch
 
-from ._lib import (GDNError, LIB_PATH, gdn_chunk_prefill, gdn_chunk_prefill_workspace_size,
-                   gdn_conv1d_silu, gdn_decode_step, lib)
+from ._lib import (GDNError, LIB_PATH, gdn_chunk_prefill, gdn_chunk_prefill_noalloc,
+                   gdn_chunk_prefill_workspace_size, gdn_conv1d_silu, gdn_decode_step, lib)
 
 __all__ = ["GDNError", "LIB_PATH", "lib", "gdn_conv1d_silu", "gdn_chunk_prefill",
-           "gdn_chunk_prefill_workspace_size", "gdn_decode_step", "prefill_layer", "qkv_views"]
+           "gdn_chunk_prefill_workspace_size", "gdn_chunk_prefill_noalloc", "gdn_decode_step",
+           "prefill_layer", "qkv_views"]
 
 
 def qkv_views(y: torch.Tensor, Hk: int, Hv: int, d: int):

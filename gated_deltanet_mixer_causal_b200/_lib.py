@@ -33,6 +33,9 @@ SIGNATURES = {
                                           _P, _SZ, _P]),
     "gdn_decode_step": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _I32, _I32,
                                         _I32, _I32, _I32, _F32, _P]),
+    "gdn_chunk_prefill_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int, _I64, _I32,
+                                                  _I32, _I32, _I32, _I64, _I64, _P, _I32, _P, _P,
+                                                  _F32, _I32, _P]),
 }
 
 _lib = None
@@ -174,6 +177,37 @@ def gdn_chunk_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torc
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(o), _dtype_code(q), T, Hk, Hv, dk, dv,
         qs, vs, _ptr(cu_seqlens), n_seq, _ptr(initial_state), _ptr(final_state), float(scale),
         int(bool(qk_l2norm)), _ptr(workspace), ws_bytes, _stream(dev)), "gdn_chunk_prefill")
+    return o
+
+
+def gdn_chunk_prefill_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                              g: torch.Tensor, beta: torch.Tensor,
+                              cu_seqlens: Optional[torch.Tensor] = None,
+                              initial_state: Optional[torch.Tensor] = None,
+                              final_state: Optional[torch.Tensor] = None, scale: float = 1.0,
+                              qk_l2norm: bool = True, o: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """gdn_chunk_prefill with the library's static scratch instead of a workspace, for
+    callers that cannot allocate device memory (see include/gdn.h for the size limit and
+    the rule that overlapping calls race). Pass ``o`` to keep this call allocation-free
+    on the Python side as well."""
+    T, Hk, dk = q.shape
+    _, Hv, dv = v.shape
+    dev = q.device
+    n_seq = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    qs = _row_view(q, "q"); ks = _row_view(k, "k"); _row_view(v, "v")
+    if k.shape != q.shape or ks != qs:
+        raise ValueError("k must match q in shape and token stride")
+    _need(g, "g", (T, Hv), torch.float32, dev)
+    _need(beta, "beta", (T, Hv), torch.float32, dev)
+    _need(initial_state, "initial_state", (n_seq, Hv, dv, dk), torch.float32, dev)
+    _need(final_state, "final_state", (n_seq, Hv, dv, dk), torch.float32, dev)
+    if o is None:
+        o = torch.empty((T, Hv, dv), dtype=q.dtype, device=dev)
+    _need(o, "o", (T, Hv, dv), q.dtype, dev)
+    _check(lib().gdn_chunk_prefill_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(o), _dtype_code(q), T, Hk, Hv, dk, dv,
+        qs, v.stride(0), _ptr(cu_seqlens), n_seq, _ptr(initial_state), _ptr(final_state),
+        float(scale), int(bool(qk_l2norm)), _stream(dev)), "gdn_chunk_prefill_noalloc")
     return o
 
 

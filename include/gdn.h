@@ -140,6 +140,39 @@ gdn_status_t gdn_chunk_prefill(const void* q, const void* k, const void* v,
                                void* workspace, size_t workspace_bytes, gdn_stream_t stream);
 
 /*
+ * gdn_chunk_prefill_noalloc -- gdn_chunk_prefill for callers that cannot allocate.
+ *
+ * The pages have no counterpart to this call; it is a convenience of this library.
+ * Some callers cannot allocate device memory: a plugin inside a host application that
+ * owns all GPU memory through its own pool and gives plugins no allocation hook, or a
+ * latency-critical loop where cudaMalloc (and the synchronisation it may imply) is not
+ * acceptable. This variant takes the same arguments as gdn_chunk_prefill minus the
+ * workspace, and uses a scratch array that the library reserves statically on every GPU
+ * that loads it (64 MiB, held until the process exits). It allocates nothing and calls
+ * no allocating routine.
+ *
+ * Limit: the call is refused with GDN_ERR_WORKSPACE, launching nothing, when
+ * gdn_chunk_prefill_workspace_size(...) for these sizes exceeds 64 MiB (with 48 value
+ * heads of 128 that is about 3,300 tokens per call; use gdn_chunk_prefill with a caller
+ * workspace beyond that). Shapes that need no workspace run exactly as gdn_chunk_prefill.
+ * Set-up: the first call on each device looks up the scratch array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call before any
+ * stream capture. The array is shared by every call: the kernels rewrite everything they
+ * read from it, so no clearing is needed, but calls whose execution overlaps on the GPU
+ * (different streams, or different host threads on one device) race on it -- order them
+ * on one stream or synchronise between them.
+ * Returns the same codes as gdn_chunk_prefill.
+ */
+gdn_status_t gdn_chunk_prefill_noalloc(const void* q, const void* k, const void* v,
+                                       const float* g, const float* beta, void* o,
+                                       gdn_dtype_t dt, int64_t T, int32_t Hk, int32_t Hv,
+                                       int32_t dk, int32_t dv, int64_t qk_stride,
+                                       int64_t v_stride, const int32_t* cu_seqlens,
+                                       int32_t n_seq, const float* initial_state,
+                                       float* final_state, float scale, int32_t qk_l2norm,
+                                       gdn_stream_t stream);
+
+/*
  * gdn_decode_step -- one token for each of B sequences, state updated in place.
  *
  * Defined by the Qwen3.5 page, section 8 (decode becomes a state-update workload:
