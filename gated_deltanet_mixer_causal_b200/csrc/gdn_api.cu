@@ -48,9 +48,11 @@ bool valid_dtype(gdn_dtype_t dt) { return dt == GDN_F32 || dt == GDN_BF16; }
 
 bool supported_head_dim(int32_t d) { return d == 16 || d == 32 || d == 64 || d == 128; }
 
-// bf16 activations with 128-wide heads run the chunked tensor-core prefill; fp32
-// activations and smaller heads run the token-by-token fp32 kernel.
-bool use_tensor_core_prefill(gdn_dtype_t dt, int32_t d) { return dt == GDN_BF16 && d == 128; }
+// bf16 activations with 128-wide heads (and at most 8 value heads per key head) run the
+// chunked tensor-core prefill; everything else runs the token-by-token fp32 kernel.
+bool use_tensor_core_prefill(gdn_dtype_t dt, int32_t d, int32_t Hk, int32_t Hv) {
+  return dt == GDN_BF16 && d == 128 && Hv / Hk <= gdn::kPrefillTcMaxG;
+}
 
 }  // namespace
 
@@ -107,7 +109,7 @@ size_t gdn_chunk_prefill_workspace_size(int64_t T, int32_t n_seq, int32_t Hk, in
       !supported_head_dim(dk))
     return SIZE_MAX;
   if (n_seq < 1) n_seq = 1;
-  return use_tensor_core_prefill(dt, dk) ? gdn::prefill_chunk_tc_workspace(T, n_seq, Hv) : 0;
+  return use_tensor_core_prefill(dt, dk, Hk, Hv) ? gdn::prefill_chunk_tc_workspace(T, n_seq, Hv) : 0;
 }
 
 gdn_status_t gdn_chunk_prefill(const void* q, const void* k, const void* v, const float* g,
@@ -151,7 +153,7 @@ gdn_status_t gdn_chunk_prefill(const void* q, const void* k, const void* v, cons
   if (workspace_bytes < need || (need > 0 && workspace == nullptr))
     return fail(GDN_ERR_WORKSPACE, "chunk_prefill: workspace %zu bytes < %zu needed", workspace_bytes, need);
   if (T == 0 && final_state == nullptr) return ok();
-  if (use_tensor_core_prefill(dt, dk)) {
+  if (use_tensor_core_prefill(dt, dk, Hk, Hv)) {
     if (!aligned16(workspace) || ((uintptr_t)workspace & 255u) != 0)
       return fail(GDN_ERR_INVALID_ARG, "chunk_prefill: workspace must be 256-byte aligned");
     return cuda_status(gdn::launch_prefill_chunk_tc(q, k, v, g, beta, o, T, Hk, Hv, qk_stride, v_stride,

@@ -29,8 +29,10 @@ cudaError_t launch_prefill_recurrent(int dtype, const void* q, const void* k, co
                                      const float* init, float* final_state, float scale,
                                      int32_t l2norm, cudaStream_t stream);
 
-// Chunked WY/UT prefill on tcgen05 (bf16 activations, dk = dv = 128). Needs
+// Chunked WY/UT prefill on tcgen05 (bf16 activations, dk = dv = 128, at most
+// kPrefillTcMaxG value heads per key head). Needs
 // prefill_chunk_tc_workspace(...) bytes of workspace.
+constexpr int kPrefillTcMaxG = 8;
 size_t prefill_chunk_tc_workspace(int64_t T, int32_t n_seq, int32_t Hv);
 cudaError_t launch_prefill_chunk_tc(const void* q, const void* k, const void* v, const float* g,
                                     const float* beta, void* o, int64_t T, int32_t Hk, int32_t Hv,

@@ -11,19 +11,23 @@
 //
 // Three kernels:
 //  1. plan  : chunk offsets of every packed sequence (chunks never straddle sequences).
-//  2. intra : one CTA per (chunk, key head): TMA loads q, k; tcgen05 computes K K^T and
-//             Q K^T in TMEM; per value head the decay-masked A and M o QK^T, the unit lower
-//             triangular inverse Tm (fp32, 16x16 diagonal blocks by warps, then block
-//             products), and writes P = Tm diag(beta), Pk = Tm diag(beta e^G / |k|) and
-//             Mqk = M o QK^T / (|q||k|) (bf16) plus row scales to the workspace.
-//  3. chain : one CTA per (sequence, value head, 64-wide slice of dv): walks the chunks in
-//             order with the fp32 state slice in registers (its bf16 copy in shared memory
-//             feeds the MMAs), five tcgen05 GEMMs per chunk:
-//               W = Pk K,  U = P V - W S0^T,  O1 = Q S0^T,  O2 = Mqk U,  dS^T = K^T U'
-//             and writes o = scale (e^{G_r}/|q_r| O1 + O2). Inputs for chunk c+1 stream in
-//             by TMA while chunk c computes.
+//  2. intra : one CTA per (chunk, key head), everything that does not depend on the state:
+//             [K; Q] K^T on tcgen05 (M = 128); per value head the decay-masked A and
+//             Mqk = M o QK^T / (|q||k|), the unit lower triangular inverse Tm (fp32), then
+//             [P; Pk] V and [P; Pk] K on tcgen05 with P = Tm diag(beta),
+//             Pk = Tm diag(beta e^G / |k|), giving U~ = P V and W = Pk K. Writes -W, U~,
+//             Mqk (bf16) and the row scales to the workspace.
+//  3. chain : one CTA per (sequence, value head, 64-wide slice of dv) walks the chunks in
+//             order with the fp32 state slice in registers and its bf16 copy in shared
+//             memory; per chunk only the state-dependent GEMMs remain:
+//               [-W; Q] S0^T  (U = U~ - W S0^T in rows 0..63, Q S0^T in rows 64..127)
+//               dS^T = K^T U',   O2 = Mqk U
+//             The two GEMMs on the serial path are split along K over two issuing threads
+//             (tcgen05.mma costs a fixed issue time per instruction, so two issuers halve
+//             the path); a third thread issues O2 and the TMA loads.
 // Operands are staged in shared memory in the 128-byte-swizzled layouts TMA writes; K-major
-// and MN-major descriptors read the same q/k/v tiles. Every wait is bounded.
+// and MN-major descriptors read the same tiles, and stacking two 64-row tiles 8 KB apart
+// makes one M = 128 operand. Every wait is bounded.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -49,8 +53,15 @@ constexpr int kErrIntraTma = 11, kErrIntraMma = 12, kErrChainTma = 21, kErrChain
 // ------------------------------------------------------------------ workspace layout
 
 struct Ws {
-  size_t err, prefix, mats, vecs, last, total;
+  size_t err, prefix, wu, mq, vecs, total;
 };
+
+// Per (chunk, value head): wu = [-W (64 x 128) ; U~ (64 x 128)] bf16 rows of 128 elements,
+// mq = Mqk (64 x 64) bf16, vecs = row scales: [0, 64) e^{G_r}/|q_r|, [64, 128)
+// e^{G_L - G_r}/|k_r|, [128] e^{G_L}; 132 floats = 528 bytes (a multiple of 16).
+constexpr int kWuBytes = 2 * C * D * 2;
+constexpr int kVecFloats = 132;
+constexpr int kVecBytes = kVecFloats * 4;
 
 __host__ __device__ inline int64_t max_slots(int64_t T, int32_t n_seq) { return (T + C - 1) / C + n_seq; }
 
@@ -61,10 +72,10 @@ __host__ __device__ inline Ws ws_layout(int64_t T, int32_t n_seq, int32_t Hv) {
   const size_t slots = (size_t)max_slots(T, n_seq);
   w.err = 0;
   w.prefix = 256;
-  w.mats = align256(w.prefix + (size_t)(n_seq + 1) * 4);
-  w.vecs = align256(w.mats + slots * Hv * 3 * kMatBytes);
-  w.last = align256(w.vecs + slots * Hv * 2 * C * 4);
-  w.total = align256(w.last + slots * Hv * 4);
+  w.wu = align256(w.prefix + (size_t)(n_seq + 1) * 4);
+  w.mq = align256(w.wu + slots * Hv * kWuBytes);
+  w.vecs = align256(w.mq + slots * Hv * kMatBytes);
+  w.total = align256(w.vecs + slots * Hv * kVecBytes);
   return w;
 }
 
@@ -126,39 +137,67 @@ __device__ __forceinline__ int32_t slot_to_seq(const int32_t* prefix, int32_t n_
 
 // ------------------------------------------------------------------ MMA descriptors
 
-// K-major operand: [rows][128-byte swizzled row] atoms of 64 columns, atoms atom_bytes
-// apart; kk-th K step of 16 elements.
-__device__ __forceinline__ uint64_t desc_k(uint32_t base, int kk, uint32_t atom_bytes) {
-  return smem_desc(base + (uint32_t)(kk >> 2) * atom_bytes + (uint32_t)(kk & 3) * 32u, 16u, 1024u);
-}
-// MN-major operand: rows are the K index (128 bytes = 64 MN elements each), MN atoms
-// atom_bytes apart; kk-th K step = 16 rows.
-__device__ __forceinline__ uint64_t desc_mn(uint32_t base, int kk, uint32_t atom_bytes) {
-  return smem_desc(base + (uint32_t)kk * 2048u, atom_bytes, 1024u);
-}
-
-// Row r (0..63) of an M = 64 accumulator lives in TMEM lane 32 * (r / 16) + r % 16.
+// TMEM address of lane 32 * quadrant (a warp reads the 32 lanes of its quadrant, warp % 4).
 __device__ __forceinline__ uint32_t tmem_quadrant(uint32_t tmem, int warp) {
   return tmem + ((uint32_t)(warp * 32) << 16);
 }
 
 // ------------------------------------------------------------------------ intra
 
+// Warp-level tf32 MMA (m16n8k8) for the 16x16 block products of the triangular inverse.
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// c (a 16x16 block as two m16n8 fragments) += X[xr.., xc..] * Y[yr.., yc..], fp32 matrices with
+// row pitch px / py. X is read transposed (X(i, k) = Xs[k][i]) when x_t is set.
+template <bool x_t>
+__device__ __forceinline__ void block_mma16(float (&c)[2][4], const float* Xs, int px, int xr, int xc,
+                                            const float* Ys, int py, int yr, int yc, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int ks = 0; ks < 2; ++ks) {
+    const int k0 = 8 * ks + t;
+    auto X = [&](int i, int k) { return x_t ? Xs[(xc + k) * px + xr + i] : Xs[(xr + i) * px + xc + k]; };
+    const uint32_t a[4] = {to_tf32(X(g, k0)), to_tf32(X(g + 8, k0)), to_tf32(X(g, k0 + 4)), to_tf32(X(g + 8, k0 + 4))};
+#pragma unroll
+    for (int nh = 0; nh < 2; ++nh) {
+      const uint32_t bb[2] = {to_tf32(Ys[(yr + k0) * py + yc + 8 * nh + g]),
+                              to_tf32(Ys[(yr + k0 + 4) * py + yc + 8 * nh + g])};
+      mma_tf32_16x8x8(c[nh], a, bb);
+    }
+  }
+}
+
 // shared memory of the intra kernel (offsets from a 1024-aligned base)
-constexpr int kIQ = 0;                          // q tile: 2 atoms x 8 KB
-constexpr int kIK = 16384;                      // k tile: 2 atoms x 8 KB
-constexpr int kIA = 32768;                      // A   fp32 [64][65]
-constexpr int kIT = kIA + 64 * 65 * 4;          // Tm  fp32 [64][65]
-constexpr int kITmp = kIT + 64 * 65 * 4;        // block-product scratch fp32 [3][16][17]
-constexpr int kIVec = kITmp + 3 * 16 * 17 * 4;  // rq, rk, G, beta  [4][64] fp32
-constexpr int kIBar = kIVec + 4 * 64 * 4;       // 2 mbarriers + tmem address
+constexpr int kMaxG = kPrefillTcMaxG;           // value heads per key head on this path
+constexpr int kIKQ = 0;                         // [K0 | Q0 | K1 | Q1]: [K; Q] is one 128-row operand
+constexpr int kIV = 32768;                      // V tile of one value head: 2 atoms
+constexpr int kIPP = 49152;                     // [P | Pk] bf16, K-major
+constexpr int kLd = 72;                         // fp32 row pitch of A^T and Tm (= 8 mod 32:
+                                                // conflict-free tf32 fragment loads)
+constexpr int kIA = 65536;                      // A^T fp32 [64][kLd] (A^T[i][r] = A[r][i])
+constexpr int kIT = kIA + 64 * kLd * 4;         // Tm  fp32 [64][kLd]
+constexpr int kITmp = kIT + 64 * kLd * 4;       // per-warp block scratch fp32 [4][16][kLd16]
+constexpr int kLd16 = 24;
+constexpr int kIVec = kITmp + 4 * 16 * kLd16 * 4;   // rq, rk, G, colP, colPk [5][64]
+constexpr int kIGB = kIVec + 5 * 64 * 4;        // g, beta of every value head [2][kMaxG][64]
+constexpr int kIBar = kIGB + 2 * kMaxG * 64 * 4;    // 2 mbarriers + tmem address
 constexpr int kIntraSmem = kIBar + 64 + 1024;   // + alignment slack
+constexpr uint32_t kTKQ = 0, kTUW = 128;        // TMEM columns: [KK^T; QK^T], [P;Pk] V or K
 
 __global__ void __launch_bounds__(128)
 chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
-                   const float* __restrict__ g, const float* __restrict__ beta,
-                   const int32_t* __restrict__ cu, int32_t n_seq, int64_t T, int32_t Hk, int32_t Hv,
-                   uint8_t* __restrict__ ws) {
+                   const __grid_constant__ CUtensorMap map_v, const float* __restrict__ g,
+                   const float* __restrict__ beta, const int32_t* __restrict__ cu, int32_t n_seq,
+                   int64_t T, int32_t Hk, int32_t Hv, uint8_t* __restrict__ ws) {
   const Ws L = ws_layout(T, n_seq, Hv);
   int* err = reinterpret_cast<int*>(ws + L.err);
   const int32_t* prefix = reinterpret_cast<const int32_t*>(ws + L.prefix);
@@ -174,13 +213,16 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float(*A)[65] = reinterpret_cast<float(*)[65]>(sm + kIA);
-  float(*Tm)[65] = reinterpret_cast<float(*)[65]>(sm + kIT);
-  float(*tmp)[16][17] = reinterpret_cast<float(*)[16][17]>(sm + kITmp);
+  float* At = reinterpret_cast<float*>(sm + kIA);
+  float* Tm = reinterpret_cast<float*>(sm + kIT);
+  float* scratch = reinterpret_cast<float*>(sm + kITmp) + warp * 16 * kLd16;
   float* rq = reinterpret_cast<float*>(sm + kIVec);
   float* rk = rq + 64;
   float* sG = rq + 128;
-  float* sb = rq + 192;
+  float* colP = rq + 192;
+  float* colPk = rq + 256;
+  float* gAll = reinterpret_cast<float*>(sm + kIGB);
+  float* bAll = gAll + kMaxG * 64;
   uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + kIBar);
   uint64_t* bar_mma = bar_tma + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_tma + 2);
@@ -190,29 +232,40 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     mbar_init(bar_mma, 1);
     fence_mbar_init();
   }
-  if (warp == 0) { tmem_alloc(tmem_slot, 128); tmem_relinquish(); }
+  if (warp == 0) { tmem_alloc(tmem_slot, 256); tmem_relinquish(); }
+  // g, beta of all G value heads for the chunk (rows past the sequence end: 0)
+  for (int e = tid; e < G * 64; e += 128) {
+    const int j = e >> 6, r = e & 63;
+    const bool v = r < len;
+    gAll[e] = v ? g[(t0 + r) * Hv + hk * G + j] : 0.f;
+    bAll[e] = v ? beta[(t0 + r) * Hv + hk * G + j] : 0.f;
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const uint32_t tq = tmem_quadrant(tmem, warp);   // lanes 32 w .. 32 w + 31: rows of M = 128 results
+  uint32_t ph_tma = 0u, ph_mma = 0u;
 
   if (tid == 0) {
-    mbar_arrive_expect_tx(bar_tma, 4 * 8192);
+    mbar_arrive_expect_tx(bar_tma, 32768 + 16384);
     for (int hh = 0; hh < 2; ++hh) {
-      tma_load_2d(sm + kIQ + hh * 8192, &map_q, hk * D + hh * 64, (int32_t)t0, bar_tma);
-      tma_load_2d(sm + kIK + hh * 8192, &map_k, hk * D + hh * 64, (int32_t)t0, bar_tma);
+      tma_load_2d(sm + kIKQ + hh * 16384, &map_k, hk * D + hh * 64, (int32_t)t0, bar_tma);
+      tma_load_2d(sm + kIKQ + hh * 16384 + 8192, &map_q, hk * D + hh * 64, (int32_t)t0, bar_tma);
+      tma_load_2d(sm + kIV + hh * 8192, &map_v, (hk * G) * D + hh * 64, (int32_t)t0, bar_tma);
     }
   }
-  bool ok = mbar_wait(bar_tma, 0, err, kErrIntraTma);
+  bool ok = mbar_wait(bar_tma, ph_tma, err, kErrIntraTma);
+  ph_tma ^= 1u;
   if (__syncthreads_or(!ok)) goto teardown;
 
   {  // inverse L2 norms of the chunk's q and k rows (0 for rows past the sequence end)
     const int r = tid & 63;
-    const uint8_t* tile = sm + (tid < 64 ? kIQ : kIK);
+    const uint8_t* tile = sm + kIKQ + (tid < 64 ? 8192 : 0);
     float ss = 0.f;
     for (int hh = 0; hh < 2; ++hh)
       for (int c8 = 0; c8 < 8; ++c8) {
-        const uint4 u = *reinterpret_cast<const uint4*>(tile + hh * 8192 + sw128_off(r, c8 * 8));
+        const uint4 u = *reinterpret_cast<const uint4*>(tile + hh * 16384 + sw128_off(r, c8 * 8));
         const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -224,28 +277,25 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     (tid < 64 ? rq : rk)[r] = inv;
   }
 
-  if (tid == 0) {   // K K^T -> TMEM cols [0, 64), Q K^T -> cols [64, 128); M = N = 64, K = 128
+  if (tid == 0) {   // [K; Q] K^T -> rows 0..63: K K^T, rows 64..127: Q K^T  (M = 128, N = 64, K = 128)
     tc_fence_after();
-    const uint32_t q0 = smem_u32(sm + kIQ), k0 = smem_u32(sm + kIK);
-    const uint32_t id = idesc_bf16(64, 64, 0, 0);
-    for (int kk = 0; kk < 8; ++kk) mma_bf16(tmem, desc_k(k0, kk, 8192), desc_k(k0, kk, 8192), id, kk > 0);
-    for (int kk = 0; kk < 8; ++kk) mma_bf16(tmem + 64, desc_k(q0, kk, 8192), desc_k(k0, kk, 8192), id, kk > 0);
+    const uint64_t kq = smem_desc(smem_u32(sm + kIKQ), 16u, 1024u);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const uint64_t off = (uint64_t)((kk >> 2) * (16384 >> 4) + (kk & 3) * 2);
+      mma_bf16(tmem + kTKQ, kq + off, kq + off, idesc_bf16(128, 64, 0, 0), kk > 0);
+    }
     mma_commit(bar_mma);
   }
-  ok = mbar_wait(bar_mma, 0, err, kErrIntraMma);
+  ok = mbar_wait(bar_mma, ph_mma, err, kErrIntraMma);
+  ph_mma ^= 1u;
   if (__syncthreads_or(!ok)) goto teardown;
   tc_fence_after();
 
   for (int j = 0; j < G; ++j) {
     const int h = hk * G + j;
-    if (tid < 64) {
-      const bool v = tid < len;
-      sG[tid] = v ? g[(t0 + tid) * Hv + h] : 0.f;
-      sb[tid] = v ? beta[(t0 + tid) * Hv + h] : 0.f;
-    }
-    __syncthreads();
     if (warp == 0) {   // inclusive cumulative log-decay over the chunk (2 values per lane)
-      float a0 = sG[2 * lane], a1 = sG[2 * lane + 1];
+      const float a0 = gAll[j * 64 + 2 * lane], a1 = gAll[j * 64 + 2 * lane + 1];
       float s = a0 + a1;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -257,28 +307,36 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
       sG[2 * lane + 1] = excl + a0 + a1;
     }
     __syncthreads();
+    const float* sb = bAll + j * 64;
+    if (tid < 64) {   // column factors of P = Tm diag(beta) and Pk = Tm diag(beta e^G / |k|)
+      colP[tid] = sb[tid];
+      colPk[tid] = sb[tid] * __expf(sG[tid]) * rk[tid];
+    }
 
-    // rows of A (from K K^T) and of Mqk (from Q K^T): lane l < 16 of warp w owns row 16w+l
+    // thread t < 64: row t of A (stored transposed) from K K^T; t >= 64: row t-64 of Mqk
     {
-      const int r = warp * 16 + lane;
-      const bool own = lane < 16;
-      const float Gr = own ? sG[r] : 0.f, br = own ? sb[r] : 0.f;
-      const float rkr = own ? rk[r] : 0.f, rqr = own ? rq[r] : 0.f;
-      uint8_t* mq = ws + L.mats + ((size_t)(slot * Hv + h) * 3 + 2) * kMatBytes;
+      const int r = tid & 63;
+      const float Gr = sG[r];
+      uint8_t* mq = ws + L.mq + (size_t)(slot * Hv + h) * kMatBytes;
       for (int cb = 0; cb < 2; ++cb) {
-        float kkv[32], qkv[32];
-        tmem_ld32(tmem_quadrant(tmem, warp) + cb * 32, kkv);
-        tmem_ld32(tmem_quadrant(tmem, warp) + 64 + cb * 32, qkv);
-        if (own) {
-          float mrow[32];
+        float v[32];
+        tmem_ld32(tq + kTKQ + cb * 32, v);
+        if (tid < 64) {
+          const float f = sb[r] * rk[r];
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const int i = cb * 32 + e;
-            const float dec = (i <= r) ? expf(Gr - sG[i]) : 0.f;
-            A[r][i] = (i < r) ? br * dec * rkr * rk[i] * kkv[e] : 0.f;
-            mrow[e] = dec * rqr * rk[i] * qkv[e];
+            At[i * kLd + r] = (i < r) ? f * __expf(Gr - sG[i]) * rk[i] * v[e] : 0.f;
           }
-          VecIO<bf16, 32>::store(reinterpret_cast<bf16*>(mq) + r * C + cb * 32, mrow);
+        } else {
+          const float f = rq[r];
+          float m[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int i = cb * 32 + e;
+            m[e] = (i <= r) ? f * __expf(Gr - sG[i]) * rk[i] * v[e] : 0.f;
+          }
+          VecIO<bf16, 32>::store(reinterpret_cast<bf16*>(mq) + r * C + cb * 32, m);
         }
       }
     }
@@ -293,94 +351,161 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
       for (int r = 0; r < 16; ++r) {
         float s = (r == jc) ? 1.f : 0.f;
 #pragma unroll
-        for (int i = 0; i < r; ++i) s = fmaf(-A[b0 + r][b0 + i], x[i], s);
+        for (int i = 0; i < r; ++i) s = fmaf(-At[(b0 + i) * kLd + b0 + r], x[i], s);
         x[r] = s;
       }
       if (lane < 16) {
 #pragma unroll
-        for (int r = 0; r < 16; ++r) Tm[b0 + r][b0 + jc] = x[r];
+        for (int r = 0; r < 16; ++r) Tm[(b0 + r) * kLd + b0 + jc] = x[r];
       }
-      // blocks above the diagonal are zero
-      for (int e = lane; e < 16 * 64; e += 32) {
+      for (int e = lane; e < 16 * 64; e += 32) {   // blocks above the diagonal are zero
         const int r = e >> 6, c = e & 63;
-        if (c >= b0 + 16) Tm[b0 + r][c] = 0.f;
+        if (c >= b0 + 16) Tm[(b0 + r) * kLd + c] = 0.f;
       }
     }
     __syncthreads();
-    // off-diagonal blocks: Tm_ba = -Tm_bb sum_{c=a}^{b-1} A_bc Tm_ca, by block distance
+    // off-diagonal blocks by block distance, one warp per block: Tm_ba = -Tm_bb sum_c A_bc Tm_ca
     for (int dist = 1; dist < 4; ++dist) {
-      const int npair = 4 - dist;
-      for (int e = tid; e < npair * 256; e += 128) {
-        const int p = e >> 8, r = (e >> 4) & 15, col = e & 15;
-        const int bb = p + dist, aa = p;
-        float s = 0.f;
+      if (warp < 4 - dist) {
+        const int aa = warp, bb = warp + dist;
+        float c[2][4] = {};
         for (int cblk = aa; cblk < bb; ++cblk)
+          block_mma16<true>(c, At, kLd, 16 * bb, 16 * cblk, Tm, kLd, 16 * cblk, 16 * aa, lane);
+        const int gq = lane >> 2, tq4 = lane & 3;
 #pragma unroll
-          for (int k = 0; k < 16; ++k) s = fmaf(A[16 * bb + r][16 * cblk + k], Tm[16 * cblk + k][16 * aa + col], s);
-        tmp[p][r][col] = s;
-      }
-      __syncthreads();
-      for (int e = tid; e < npair * 256; e += 128) {
-        const int p = e >> 8, r = (e >> 4) & 15, col = e & 15;
-        const int bb = p + dist, aa = p;
-        float s = 0.f;
+        for (int nh = 0; nh < 2; ++nh) {
+          scratch[gq * kLd16 + 8 * nh + 2 * tq4] = c[nh][0];
+          scratch[gq * kLd16 + 8 * nh + 2 * tq4 + 1] = c[nh][1];
+          scratch[(gq + 8) * kLd16 + 8 * nh + 2 * tq4] = c[nh][2];
+          scratch[(gq + 8) * kLd16 + 8 * nh + 2 * tq4 + 1] = c[nh][3];
+        }
+        __syncwarp();
+        float d[2][4] = {};
+        block_mma16<false>(d, Tm, kLd, 16 * bb, 16 * bb, scratch, kLd16, 0, 0, lane);
 #pragma unroll
-        for (int k = 0; k < 16; ++k) s = fmaf(Tm[16 * bb + r][16 * bb + k], tmp[p][k][col], s);
-        Tm[16 * bb + r][16 * aa + col] = -s;
+        for (int nh = 0; nh < 2; ++nh) {
+          float* row0 = Tm + (16 * bb + gq) * kLd + 16 * aa + 8 * nh + 2 * tq4;
+          float* row8 = row0 + 8 * kLd;
+          row0[0] = -d[nh][0]; row0[1] = -d[nh][1];
+          row8[0] = -d[nh][2]; row8[1] = -d[nh][3];
+        }
       }
       __syncthreads();
     }
 
-    // P = Tm diag(beta), Pk = Tm diag(beta e^G |k|^-1), row scales
+    // [P | Pk] as bf16 K-major operands: thread = one column of one matrix; row scales out
     {
-      uint8_t* base = ws + L.mats + (size_t)(slot * Hv + h) * 3 * kMatBytes;
-      for (int e = tid; e < 64 * 8; e += 128) {     // (row, 8-column group)
-        const int r = e >> 3, c0 = (e & 7) * 8;
-        float pv[8], pk[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const int i = c0 + q;
-          const float t = Tm[r][i] * sb[i];
-          pv[q] = t;
-          pk[q] = t * expf(sG[i]) * rk[i];
-        }
-        VecIO<bf16, 8>::store(reinterpret_cast<bf16*>(base) + r * C + c0, pv);
-        VecIO<bf16, 8>::store(reinterpret_cast<bf16*>(base + kMatBytes) + r * C + c0, pk);
-      }
-      float* vec = reinterpret_cast<float*>(ws + L.vecs) + (size_t)(slot * Hv + h) * 2 * C;
+      const int i = tid & 63, m = tid >> 6;
+      const float f = m == 0 ? colP[i] : colPk[i];
+      uint8_t* tile = sm + kIPP + m * 8192;
+#pragma unroll 8
+      for (int r = 0; r < 64; ++r)
+        *reinterpret_cast<bf16*>(tile + sw128_off(r, i)) = __float2bfloat16_rn(Tm[r * kLd + i] * f);
+      float* vec = reinterpret_cast<float*>(ws + L.vecs) + (size_t)(slot * Hv + h) * kVecFloats;
       const float Gl = sG[C - 1];
-      if (tid < 64) vec[tid] = expf(sG[tid]) * rq[tid];
-      else vec[tid] = expf(Gl - sG[tid - 64]) * rk[tid - 64];
-      if (tid == 0) reinterpret_cast<float*>(ws + L.last)[slot * Hv + h] = expf(Gl);
+      if (tid < 64) vec[tid] = __expf(sG[tid]) * rq[tid];
+      else vec[tid] = __expf(Gl - sG[tid - 64]) * rk[tid - 64];
+      if (tid < kVecFloats - 128) vec[128 + tid] = tid == 0 ? __expf(Gl) : 0.f;
     }
+    fence_async_smem();
+    tc_fence_before();
     __syncthreads();
+
+    uint8_t* wu = ws + L.wu + (size_t)(slot * Hv + h) * kWuBytes;
+    const uint64_t dpp = smem_desc(smem_u32(sm + kIPP), 16u, 1024u);
+    if (tid == 0) {   // [P; Pk] V: rows 0..63 = U~ (M = 128, N = 128, K = 64)
+      tc_fence_after();
+      const uint64_t dv = smem_desc(smem_u32(sm + kIV), 8192u, 1024u);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16(tmem + kTUW, dpp + 2 * kk, dv + 128 * kk, idesc_bf16(128, 128, 0, 1), kk > 0);
+      mma_commit(bar_mma);
+    }
+    ok = mbar_wait(bar_mma, ph_mma, err, kErrIntraMma);
+    ph_mma ^= 1u;
+    if (__syncthreads_or(!ok)) goto teardown;
+    tc_fence_after();
+    if (tid == 0 && j + 1 < G) {   // the V tile is free: next value head's V
+      mbar_arrive_expect_tx(bar_tma, 16384);
+      for (int hh = 0; hh < 2; ++hh)
+        tma_load_2d(sm + kIV + hh * 8192, &map_v, (h + 1) * D + hh * 64, (int32_t)t0, bar_tma);
+    }
+    if (warp < 2) {   // U~ row tid -> bf16
+      for (int cb = 0; cb < 4; ++cb) {
+        float v[32];
+        tmem_ld32(tq + kTUW + cb * 32, v);
+        VecIO<bf16, 32>::store(reinterpret_cast<bf16*>(wu) + (C + tid) * D + cb * 32, v);
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {   // [P; Pk] K: rows 64..127 = W (N = 128, K read MN-major across its atoms)
+      tc_fence_after();
+      const uint64_t dk = smem_desc(smem_u32(sm + kIKQ), 16384u, 1024u);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16(tmem + kTUW, dpp + 2 * kk, dk + 128 * kk, idesc_bf16(128, 128, 0, 1), kk > 0);
+      mma_commit(bar_mma);
+    }
+    ok = mbar_wait(bar_mma, ph_mma, err, kErrIntraMma);
+    ph_mma ^= 1u;
+    if (__syncthreads_or(!ok)) goto teardown;
+    tc_fence_after();
+    if (warp >= 2) {   // -W row (tid - 64) -> bf16
+      for (int cb = 0; cb < 4; ++cb) {
+        float v[32];
+        tmem_ld32(tq + kTUW + cb * 32, v);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = -v[e];
+        VecIO<bf16, 32>::store(reinterpret_cast<bf16*>(wu) + (tid - 64) * D + cb * 32, v);
+      }
+    }
+    if (j + 1 < G) {
+      ok = mbar_wait(bar_tma, ph_tma, err, kErrIntraTma);
+      ph_tma ^= 1u;
+    }
+    tc_fence_before();
+    if (__syncthreads_or(!ok)) goto teardown;
   }
 
 teardown:
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, 128);
+  if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
 // ------------------------------------------------------------------------ chain
 
-// shared memory of the chain kernel (offsets from a 1024-aligned base)
-constexpr int kStage = 65536;                 // one chunk's TMA inputs
-constexpr int kSK = 0, kSQ = 16384, kSV = 32768, kSP = 40960, kSPk = 49152, kSM = 57344;
-constexpr int kCW = 2 * kStage;               // -W as bf16, K-major [64][128]: 16 KB
-constexpr int kCS = kCW + 16384;              // S0^T bf16, MN-major [128][64]: 16 KB
+// shared memory of the chain kernel (offsets from a 1024-aligned base). Per stage:
+//   WQ : [-W atom0 | Q atom0 | -W atom1 | Q atom1]: [-W; Q] is one K-major 128-row operand
+//   K  : 2 atoms;  U~ (this slice) then Mqk: [U~; Mqk] is a 128-row operand whose top half
+//        only lands in rows nobody reads
+constexpr int kSWQ = 0, kSK = 32768, kSU = 49152, kSM = 57344;
+constexpr int kSVec = 65536;                  // the chunk's row scales (kVecBytes)
+constexpr int kStage = 66560;                 // one chunk (1024-aligned)
+constexpr int kStageTx = 32768 + 16384 + 8192 + 8192 + kVecBytes;   // bytes its loads deliver
+constexpr int kCS = 2 * kStage;               // S0^T bf16, MN-major [128][64]: 16 KB
 constexpr int kCU = kCS + 16384;              // U   bf16 [64][64]: 8 KB
 constexpr int kCU2 = kCU + 8192;              // U'  bf16 [64][64]: 8 KB
-constexpr int kCVec = kCU2 + 8192;            // o_scale, u_scale fp32 [2][64]
-constexpr int kCBar = kCVec + 512;            // 3 mbarriers + tmem address
-constexpr int kChainSmem = kCBar + 64 + 1024;
+constexpr int kCBar = kCU2 + 8192;            // mbarriers + tmem address
+constexpr int kChainSmem = kCBar + 128 + 1024;
+constexpr int kChainThreads = 256;
 
-// TMEM columns
-constexpr uint32_t kTW = 0, kTU = 128, kTO1 = 192, kTO2 = 256, kTdS = 320;
+// TMEM columns (M = 128 accumulators, lane = row). A = [-W; Q] S0^T is accumulated in two
+// K halves (lo: dk 0..63, hi: dk 64..127) by two issuers, each double-buffered; dS^T in two
+// K halves (tokens 0..31, 32..63); O2 = [U~; Mqk] U.
+constexpr uint32_t kTAlo = 0, kTAhi = 128, kTdSlo = 256, kTdShi = 320, kTO2 = 384;
 
-__global__ void __launch_bounds__(128, 1)
+// Wait by every thread, then agree: false if any thread's wait gave up.
+__device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t& phase, int* err, int code) {
+  const bool ok = mbar_wait(bar, phase, err, code);
+  phase ^= 1u;
+  return !__syncthreads_or(!ok);
+}
+
+__global__ void __launch_bounds__(kChainThreads, 1)
 chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
-                   const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_ws,
+                   const __grid_constant__ CUtensorMap map_wu, const __grid_constant__ CUtensorMap map_mq,
                    const int32_t* __restrict__ cu, int32_t n_seq, int64_t T, int32_t Hk, int32_t Hv,
                    const uint8_t* __restrict__ ws_ro, int* err_word, const float* init, float* fin,
                    bf16* __restrict__ o, float scale) {
@@ -391,220 +516,226 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
   const int32_t n = blockIdx.x / (NT * Hv);
   const int hk = h / (Hv / Hk);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int quad = warp & 3, half = warp >> 2;     // TMEM lanes 32 quad.., column half
+  const int lrow = quad * 32 + lane;               // this thread's accumulator row (lane)
   int64_t bos, eos;
   seq_bounds(cu, n, T, bos, eos);
   const int nc = (int)((eos - bos + C - 1) / C);
   const int32_t slot0 = prefix[n];
+  const bool issuer0 = tid == 0, issuer1 = tid == 128, issuer2 = tid == 32;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* s_os = reinterpret_cast<float*>(sm + kCVec);
-  float* s_us = s_os + 64;
   uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + kCBar);   // [2]
-  uint64_t* bar_mma = bar_tma + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_tma + 3);
+  uint64_t* bar_A0 = bar_tma + 2;
+  uint64_t* bar_A1 = bar_tma + 3;
+  uint64_t* bar_B0 = bar_tma + 4;
+  uint64_t* bar_B1 = bar_tma + 5;
+  uint64_t* bar_O = bar_tma + 6;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_tma + 7);
 
   if (tid == 0) {
-    mbar_init(&bar_tma[0], 1);
-    mbar_init(&bar_tma[1], 1);
-    mbar_init(bar_mma, 1);
+    for (int i = 0; i < 7; ++i) mbar_init(&bar_tma[i], 1);
     fence_mbar_init();
-    if (nc > 0) {
-      tma_prefetch_desc(&map_q); tma_prefetch_desc(&map_k);
-      tma_prefetch_desc(&map_v); tma_prefetch_desc(&map_ws);
-    }
+  }
+  if (issuer2 && nc > 0) {
+    tma_prefetch_desc(&map_q); tma_prefetch_desc(&map_k);
+    tma_prefetch_desc(&map_wu); tma_prefetch_desc(&map_mq);
   }
   if (warp == 0) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
 
-  // state slice: thread t holds column t of S for rows tile*DT .. +DT (i.e. row t of S^T)
-  float s[DT];
-  const int64_t sbase = ((int64_t)n * Hv + h) * D * D + (int64_t)tile * DT * D;
+  // state slice: thread (lrow, half) holds S[tile*64 + half*32 + j][lrow], j < 32
+  constexpr int SJ = DT / 2;
+  float s[SJ];
+  const int64_t sbase = ((int64_t)n * Hv + h) * D * D + (int64_t)(tile * DT + half * SJ) * D + lrow;
 #pragma unroll
-  for (int j = 0; j < DT; ++j) s[j] = init ? init[sbase + (int64_t)j * D + tid] : 0.f;
-  {
-    uint8_t* st = sm + kCS;
+  for (int j = 0; j < SJ; ++j) s[j] = init ? init[sbase + (int64_t)j * D] : 0.f;
+  auto store_state_bf16 = [&]() {
 #pragma unroll
-    for (int c8 = 0; c8 < DT / 8; ++c8) {
+    for (int c8 = 0; c8 < SJ / 8; ++c8) {
       float v8[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) v8[q] = s[c8 * 8 + q];
-      VecIO<bf16, 8>::store(reinterpret_cast<bf16*>(st + sw128_off(tid, c8 * 8)), v8);
+      VecIO<bf16, 8>::store(reinterpret_cast<bf16*>(sm + kCS + sw128_off(lrow, half * SJ + c8 * 8)), v8);
     }
-  }
+  };
+  store_state_bf16();
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const uint32_t tq = tmem_quadrant(tmem, quad);
 
   auto issue_loads = [&](int c, int b) {
     const int64_t t0 = bos + (int64_t)c * C;
     const int32_t slot = slot0 + c;
     uint8_t* stg = sm + b * kStage;
-    mbar_arrive_expect_tx(&bar_tma[b], kStage);
+    const int32_t wrow = (int32_t)(((int64_t)slot * Hv + h) * 2 * C);
+    mbar_arrive_expect_tx(&bar_tma[b], kStageTx);
     for (int hh = 0; hh < 2; ++hh) {
+      tma_load_2d(stg + kSWQ + hh * 16384, &map_wu, hh * 64, wrow, &bar_tma[b]);
+      tma_load_2d(stg + kSWQ + hh * 16384 + 8192, &map_q, hk * D + hh * 64, (int32_t)t0, &bar_tma[b]);
       tma_load_2d(stg + kSK + hh * 8192, &map_k, hk * D + hh * 64, (int32_t)t0, &bar_tma[b]);
-      tma_load_2d(stg + kSQ + hh * 8192, &map_q, hk * D + hh * 64, (int32_t)t0, &bar_tma[b]);
     }
-    tma_load_2d(stg + kSV, &map_v, h * D + tile * DT, (int32_t)t0, &bar_tma[b]);
-    const int32_t row = (int32_t)(((int64_t)slot * Hv + h) * 3 * C);
-    tma_load_2d(stg + kSP, &map_ws, 0, row, &bar_tma[b]);
-    tma_load_2d(stg + kSPk, &map_ws, 0, row + C, &bar_tma[b]);
-    tma_load_2d(stg + kSM, &map_ws, 0, row + 2 * C, &bar_tma[b]);
+    tma_load_2d(stg + kSU, &map_wu, tile * DT, wrow + C, &bar_tma[b]);
+    tma_load_2d(stg + kSM, &map_mq, 0, (int32_t)(((int64_t)slot * Hv + h) * C), &bar_tma[b]);
+    bulk_load(stg + kSVec, ws_ro + L.vecs + ((size_t)slot * Hv + h) * kVecBytes, kVecBytes, &bar_tma[b]);
   };
 
-  if (tid == 0 && nc > 0) issue_loads(0, 0);
-  uint32_t ph_tma[2] = {0u, 0u}, ph_mma = 0u;
-  bool ok = true;
-  const float* vecs = reinterpret_cast<const float*>(ws_ro + L.vecs);
-  const float* lastv = reinterpret_cast<const float*>(ws_ro + L.last);
+  // descriptors: stage 1's are stage 0's plus kStage in the start-address field
+  const uint32_t st0 = smem_u32(sm);
+  const uint64_t dWQ0 = smem_desc(st0 + kSWQ, 16u, 1024u), dK0 = smem_desc(st0 + kSK, 8192u, 1024u);
+  const uint64_t dUM0 = smem_desc(st0 + kSU, 16u, 1024u);
+  auto soff = [](int b) { return (uint64_t)(b * (kStage >> 4)); };
+  const uint64_t dS = smem_desc(smem_u32(sm + kCS), 8192u, 1024u);
+  const uint64_t dU = smem_desc(smem_u32(sm + kCU), 8192u, 1024u);
+  const uint64_t dU2 = smem_desc(smem_u32(sm + kCU2), 8192u, 1024u);
+  constexpr uint32_t kIA = idesc_bf16(128, DT, 0, 1);     // K-major A, MN-major B
+  constexpr uint32_t kIB = idesc_bf16(128, DT, 1, 1);     // MN-major A and B
 
-  for (int c = 0; c < nc; ++c) {
-    const int b = c & 1;
+  // rA half: [-W; Q] S0^T over dk [64 part, 64 part + 64) -> A_part[ab]
+  auto issue_rA = [&](int b, int ab, int part) {
+    const uint64_t a = dWQ0 + soff(b) + (uint64_t)(part * (16384 >> 4));
+    const uint32_t ta = tmem + (part ? kTAhi : kTAlo) + 64 * ab;
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+      mma_bf16(ta, a + 2 * kk, dS + 128 * (4 * part + kk), kIA, kk > 0);
+    mma_commit(part ? bar_A1 : bar_A0);
+  };
+  // rB half: dS^T = K^T U' over tokens [32 part, 32 part + 32)
+  auto issue_rB = [&](int b, int part) {
+    const uint64_t k = dK0 + soff(b);
+    const uint32_t ts = tmem + (part ? kTdShi : kTdSlo);
+#pragma unroll
+    for (int kk = 0; kk < 2; ++kk)
+      mma_bf16(ts, k + 128 * (2 * part + kk), dU2 + 128 * (2 * part + kk), kIB, kk > 0);
+    mma_commit(part ? bar_B1 : bar_B0);
+  };
+  auto issue_rO = [&](int b) {   // rows 64..127 of [U~; Mqk] U
+    const uint64_t a = dUM0 + soff(b);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) mma_bf16(tmem + kTO2, a + 2 * kk, dU + 128 * kk, kIA, kk > 0);
+    mma_commit(bar_O);
+  };
+
+  uint32_t ph_tma[2] = {0u, 0u}, phA0 = 0u, phA1 = 0u, phB0 = 0u, phB1 = 0u, phO = 0u;
+  bool ok = true;
+
+  if (nc > 0) {   // prologue: loads for chunks 0 and 1, rA(0)
+    if (issuer2) {
+      issue_loads(0, 0);
+      if (nc > 1) issue_loads(1, 1);
+    }
+    ok = wait_all(&bar_tma[0], ph_tma[0], err_word, kErrChainTma);
+    if (ok && (issuer0 || issuer1)) { tc_fence_after(); issue_rA(0, 0, issuer1 ? 1 : 0); }
+  }
+
+  for (int c = 0; ok && c < nc; ++c) {
+    const int b = c & 1;                 // stage and A buffer of chunk c
     const int64_t t0 = bos + (int64_t)c * C;
     const int len = (int)(eos - t0 < C ? eos - t0 : C);
-    const int32_t slot = slot0 + c;
-    if (tid == 0 && c + 1 < nc) issue_loads(c + 1, b ^ 1);
+    const float* vec = reinterpret_cast<const float*>(sm + b * kStage + kSVec);
+    const bool more = c + 1 < nc;
+
+    // U = U~ + (-W S0^T) rows 0..63 (quadrants 0, 1), U and U' to bf16
     {
-      const float* v = vecs + (size_t)(slot * Hv + h) * 2 * C;
-      if (tid < 64) s_os[tid] = v[tid]; else s_us[tid - 64] = v[tid];
+      const bool okA = mbar_wait(bar_A0, phA0, err_word, kErrChainMma) &&
+                       mbar_wait(bar_A1, phA1, err_word, kErrChainMma);
+      phA0 ^= 1u; phA1 ^= 1u;
+      if (__syncthreads_or(!okA)) { ok = false; break; }
     }
-    const float decay_last = lastv[slot * Hv + h];
-    ok = mbar_wait(&bar_tma[b], ph_tma[b], err_word, kErrChainTma);
-    ph_tma[b] ^= 1u;
-    if (__syncthreads_or(!ok)) break;
-
-    uint8_t* stg = sm + b * kStage;
-    const uint32_t aK = smem_u32(stg + kSK), aQ = smem_u32(stg + kSQ), aV = smem_u32(stg + kSV);
-    const uint32_t aP = smem_u32(stg + kSP), aPk = smem_u32(stg + kSPk), aM = smem_u32(stg + kSM);
-    const uint32_t aW = smem_u32(sm + kCW), aS = smem_u32(sm + kCS);
-    const uint32_t aU = smem_u32(sm + kCU), aU2 = smem_u32(sm + kCU2);
-
-    // round 1: W = Pk K (64 x 128), U = P V (64 x 64)
-    if (tid == 0) {
-      tc_fence_after();
-      for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + kTW, desc_k(aPk, kk, 0), desc_mn(aK, kk, 8192), idesc_bf16(64, 128, 0, 1), kk > 0);
-      for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + kTU, desc_k(aP, kk, 0), desc_mn(aV, kk, 8192), idesc_bf16(64, DT, 0, 1), kk > 0);
-      mma_commit(bar_mma);
-    }
-    ok = mbar_wait(bar_mma, ph_mma, err_word, kErrChainMma);
-    ph_mma ^= 1u;
-    if (__syncthreads_or(!ok)) break;
     tc_fence_after();
-    {  // W -> bf16, K-major [64 rows][128]
-      const int r = warp * 16 + lane;
-      for (int cb = 0; cb < 4; ++cb) {
-        float v[32];
-        tmem_ld32(tmem_quadrant(tmem, warp) + kTW + cb * 32, v);
-        if (lane < 16) {
-          uint8_t* atom = sm + kCW + (cb >> 1) * 8192;
+    float os = 0.f;
+    if (quad < 2) {
+      const int r = lrow;
+      const float us = vec[64 + r];
+      float a0[32], a1[32];
+      tmem_ld32(tq + kTAlo + 64 * b + half * 32, a0);
+      tmem_ld32(tq + kTAhi + 64 * b + half * 32, a1);
+      const uint8_t* ut = sm + b * kStage + kSU;
 #pragma unroll
-          for (int c8 = 0; c8 < 4; ++c8) {
-            float v8[8];
+      for (int c8 = 0; c8 < 4; ++c8) {
+        float v8[8], w8[8];
+        VecIO<bf16, 8>::load(reinterpret_cast<const bf16*>(ut + sw128_off(r, half * 32 + c8 * 8)), v8);
 #pragma unroll
-            for (int q = 0; q < 8; ++q) v8[q] = v[c8 * 8 + q];
-            VecIO<bf16, 8>::store(reinterpret_cast<bf16*>(atom + sw128_off(r, (cb & 1) * 32 + c8 * 8)), v8);
-          }
-        }
+        for (int q = 0; q < 8; ++q) { v8[q] += a0[c8 * 8 + q] + a1[c8 * 8 + q]; w8[q] = us * v8[q]; }
+        const uint32_t off = sw128_off(r, half * 32 + c8 * 8);
+        VecIO<bf16, 8>::store(reinterpret_cast<bf16*>(sm + kCU + off), v8);
+        VecIO<bf16, 8>::store(reinterpret_cast<bf16*>(sm + kCU2 + off), w8);
       }
+    } else {
+      os = vec[lrow - 64];   // the output row scale, before the stage is reused
     }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
+    if (issuer0 || issuer1) { tc_fence_after(); issue_rB(b, issuer1 ? 1 : 0); }
 
-    // round 2: U += (-W) S0^T, O1 = Q S0^T   (K = 128)
-    if (tid == 0) {
-      tc_fence_after();
-      for (int kk = 0; kk < 8; ++kk)
-        mma_bf16(tmem + kTU, desc_k(aW, kk, 8192), desc_mn(aS, kk, 0), idesc_bf16(64, DT, 0, 1, 1), true);
-      for (int kk = 0; kk < 8; ++kk)
-        mma_bf16(tmem + kTO1, desc_k(aQ, kk, 8192), desc_mn(aS, kk, 0), idesc_bf16(64, DT, 0, 1), kk > 0);
-      mma_commit(bar_mma);
+    // state update: S^T <- e^{G_L} S^T + dS^T (both K halves)
+    {
+      const bool okB = mbar_wait(bar_B0, phB0, err_word, kErrChainMma) &&
+                       mbar_wait(bar_B1, phB1, err_word, kErrChainMma);
+      phB0 ^= 1u; phB1 ^= 1u;
+      if (__syncthreads_or(!okB)) { ok = false; break; }
     }
-    ok = mbar_wait(bar_mma, ph_mma, err_word, kErrChainMma);
-    ph_mma ^= 1u;
-    if (__syncthreads_or(!ok)) break;
     tc_fence_after();
-    {  // U and U' = diag(e^{G_L - G} / |k|) U as bf16 [64 tokens][64]
-      const int r = warp * 16 + lane;
-      const float us = lane < 16 ? s_us[r] : 0.f;
-      for (int cb = 0; cb < DT / 32; ++cb) {
-        float v[32];
-        tmem_ld32(tmem_quadrant(tmem, warp) + kTU + cb * 32, v);
-        if (lane < 16) {
+    {
+      const float decay_last = vec[128];
+      float d0[32], d1[32];
+      tmem_ld32(tq + kTdSlo + half * 32, d0);
+      tmem_ld32(tq + kTdShi + half * 32, d1);
 #pragma unroll
-          for (int c8 = 0; c8 < 4; ++c8) {
-            float v8[8], w8[8];
+      for (int e = 0; e < SJ; ++e) s[e] = fmaf(decay_last, s[e], d0[e] + d1[e]);
+      store_state_bf16();
+    }
+    if (more) {   // chunk c+1's inputs must have landed before its rA
+      const bool okT = mbar_wait(&bar_tma[b ^ 1], ph_tma[b ^ 1], err_word, kErrChainTma);
+      ph_tma[b ^ 1] ^= 1u;
+      fence_async_smem();
+      tc_fence_before();
+      if (__syncthreads_or(!okT)) { ok = false; break; }
+    } else {
+      fence_async_smem();
+      tc_fence_before();
+      __syncthreads();
+    }
+    if (more && (issuer0 || issuer1)) { tc_fence_after(); issue_rA(b ^ 1, b ^ 1, issuer1 ? 1 : 0); }
+    if (issuer2) { tc_fence_after(); issue_rO(b); }
+
+    // chunk c's output while rA(c+1) runs: o_r = scale (e^{G_r}/|q_r| O1_r + O2_r)
+    {
+      const bool okO = mbar_wait(bar_O, phO, err_word, kErrChainMma);
+      phO ^= 1u;
+      if (__syncthreads_or(!okO)) { ok = false; break; }
+    }
+    tc_fence_after();
+    if (issuer2 && c + 2 < nc) issue_loads(c + 2, b);
+    if (quad >= 2) {
+      const int r = lrow - 64;
+      float a0[32], a1[32], o2[32];
+      tmem_ld32(tq + kTAlo + 64 * b + half * 32, a0);
+      tmem_ld32(tq + kTAhi + 64 * b + half * 32, a1);
+      tmem_ld32(tq + kTO2 + half * 32, o2);
+      if (r < len) {
+        bf16* dst = o + ((t0 + r) * Hv + h) * (int64_t)D + tile * DT + half * 32;
 #pragma unroll
-            for (int q = 0; q < 8; ++q) { v8[q] = v[c8 * 8 + q]; w8[q] = us * v8[q]; }
-            const uint32_t off = sw128_off(r, cb * 32 + c8 * 8);
-            VecIO<bf16, 8>::store(reinterpret_cast<bf16*>(sm + kCU + off), v8);
-            VecIO<bf16, 8>::store(reinterpret_cast<bf16*>(sm + kCU2 + off), w8);
+        for (int c8 = 0; c8 < 4; ++c8) {
+          float v8[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int e = c8 * 8 + q;
+            v8[q] = scale * fmaf(os, a0[e] + a1[e], o2[e]);
           }
+          VecIO<bf16, 8>::store(dst + c8 * 8, v8);
         }
       }
     }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-
-    // round 3: O2 = Mqk U (K = 64), dS^T = K^T U' (M = 128, K = 64)
-    if (tid == 0) {
-      tc_fence_after();
-      for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + kTO2, desc_k(aM, kk, 0), desc_mn(aU, kk, 0), idesc_bf16(64, DT, 0, 1), kk > 0);
-      for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + kTdS, desc_mn(aK, kk, 8192), desc_mn(aU2, kk, 0), idesc_bf16(128, DT, 1, 1), kk > 0);
-      mma_commit(bar_mma);
-    }
-    ok = mbar_wait(bar_mma, ph_mma, err_word, kErrChainMma);
-    ph_mma ^= 1u;
-    if (__syncthreads_or(!ok)) break;
-    tc_fence_after();
-    {  // state: S^T row tid <- e^{G_L} S^T + dS^T; refresh the bf16 copy
-      for (int cb = 0; cb < DT / 32; ++cb) {
-        float v[32];
-        tmem_ld32(tmem_quadrant(tmem, warp) + kTdS + cb * 32, v);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) s[cb * 32 + e] = fmaf(decay_last, s[cb * 32 + e], v[e]);
-      }
-#pragma unroll
-      for (int c8 = 0; c8 < DT / 8; ++c8) {
-        float v8[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) v8[q] = s[c8 * 8 + q];
-        VecIO<bf16, 8>::store(reinterpret_cast<bf16*>(sm + kCS + sw128_off(tid, c8 * 8)), v8);
-      }
-    }
-    {  // outputs: o_r = scale (e^{G_r}/|q_r| O1_r + O2_r)
-      const int r = warp * 16 + lane;
-      const float os = lane < 16 ? s_os[r] : 0.f;
-      for (int cb = 0; cb < DT / 32; ++cb) {
-        float v1[32], v2[32];
-        tmem_ld32(tmem_quadrant(tmem, warp) + kTO1 + cb * 32, v1);
-        tmem_ld32(tmem_quadrant(tmem, warp) + kTO2 + cb * 32, v2);
-        if (lane < 16 && r < len) {
-          bf16* dst = o + ((t0 + r) * Hv + h) * (int64_t)D + tile * DT + cb * 32;
-#pragma unroll
-          for (int c8 = 0; c8 < 4; ++c8) {
-            float v8[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) v8[q] = scale * fmaf(os, v1[c8 * 8 + q], v2[c8 * 8 + q]);
-            VecIO<bf16, 8>::store(dst + c8 * 8, v8);
-          }
-        }
-      }
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
   }
 
   if (ok && fin != nullptr) {
 #pragma unroll
-    for (int j = 0; j < DT; ++j) fin[sbase + (int64_t)j * D + tid] = s[j];
+    for (int j = 0; j < SJ; ++j) fin[sbase + (int64_t)j * D] = s[j];
   }
   tc_fence_before();
   __syncthreads();
@@ -670,22 +801,23 @@ cudaError_t launch_prefill_chunk_tc(const void* q, const void* k, const void* v,
   const int64_t slots = max_slots(T, n_seq);
   // with no tokens every sequence is empty: the chain kernel only copies the states and
   // never touches the maps, which are left zeroed
-  CUtensorMap mq{}, mk{}, mv{}, mw{};
+  CUtensorMap mq{}, mk{}, mv{}, mwu{}, mmq{};
   if (T > 0 && (!make_map(&mq, q, (uint64_t)Hk * D, (uint64_t)T, (uint64_t)qk_stride) ||
                 !make_map(&mk, k, (uint64_t)Hk * D, (uint64_t)T, (uint64_t)qk_stride) ||
                 !make_map(&mv, v, (uint64_t)Hv * D, (uint64_t)T, (uint64_t)v_stride) ||
-                !make_map(&mw, ws + L.mats, 64, (uint64_t)slots * Hv * 3 * C, 64)))
+                !make_map(&mwu, ws + L.wu, D, (uint64_t)slots * Hv * 2 * C, D) ||
+                !make_map(&mmq, ws + L.mq, C, (uint64_t)slots * Hv * C, C)))
     return cudaErrorInvalidValue;
   chunk_plan_kernel<<<1, 1024, 0, stream>>>(cu, n_seq, T, reinterpret_cast<int32_t*>(ws + L.prefix),
                                             reinterpret_cast<int*>(ws + L.err));
   if (T > 0) {
     dim3 gi((unsigned)slots, (unsigned)Hk);
-    chunk_intra_kernel<<<gi, 128, kIntraSmem, stream>>>(mq, mk, g, beta, cu, n_seq, T, Hk, Hv, ws);
+    chunk_intra_kernel<<<gi, 128, kIntraSmem, stream>>>(mq, mk, mv, g, beta, cu, n_seq, T, Hk, Hv, ws);
   }
   dim3 gc((unsigned)((int64_t)n_seq * Hv * NT));
-  chunk_chain_kernel<<<gc, 128, kChainSmem, stream>>>(mq, mk, mv, mw, cu, n_seq, T, Hk, Hv, ws,
-                                                      reinterpret_cast<int*>(ws + L.err), init, fin,
-                                                      static_cast<bf16*>(o), scale);
+  chunk_chain_kernel<<<gc, kChainThreads, kChainSmem, stream>>>(mq, mk, mwu, mmq, cu, n_seq, T, Hk, Hv, ws,
+                                                              reinterpret_cast<int*>(ws + L.err), init, fin,
+                                                              static_cast<bf16*>(o), scale);
   return cudaGetLastError();
 }
 
