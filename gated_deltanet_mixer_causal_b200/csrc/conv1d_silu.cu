@@ -3,20 +3,24 @@
 // y[t, c] = SiLU(sum_j w[c, j] x[t - 3 + j, c]), restarting at every sequence start from
 // the carried taps or zeros (Qwen3.5 page, section 5 and config footnote: conv kernel 4).
 //
-// HBM-bound: each thread owns 8 channels (one 16-byte bf16 vector) and a run of
-// kRunTokens tokens, sliding a 3-token window in registers, so every input is read once
-// (plus a 3-token halo per run, which hits L2) and every output written once. A warp
-// covers 32 consecutive vectors of one token row: 512 contiguous bytes per access.
+// HBM-bound: every input is read once and every output written once. A CTA owns a tile of
+// kTileTokens tokens x kTileVecs * 8 channels: it copies the tile plus a 3-token halo into
+// shared memory with 16-byte cp.async (zero-filled outside [0, T)), so many bytes are in
+// flight per SM without holding them in registers; then each thread slides a 3-token
+// window over 16 consecutive tokens of 8 channels and writes 16-byte vectors, consecutive
+// threads covering consecutive channels (1 KB contiguous per token row for bf16).
 #include "common.cuh"
 #include "launch.h"
 
 namespace gdn {
 namespace {
 
-constexpr int kVec = 8;          // channels per thread
-constexpr int kThreads = 128;    // threads per CTA (128 vectors = 1024 channels)
-constexpr int kRunTokens = 32;   // tokens per thread
-constexpr int kPrefetch = 4;     // tokens loaded ahead of use
+constexpr int kVec = 8;            // channels per thread
+constexpr int kTileTokens = 64;
+constexpr int kTileVecs = 64;      // 8-channel vectors per tile (512 channels)
+constexpr int kThreads = 256;
+constexpr int kTokPerThread = kTileTokens * kTileVecs / kThreads;   // 16
+constexpr int kRows = kTileTokens + 3;
 
 // Index of the sequence holding token t: the n with cu[n] <= t < cu[n+1] (clamped).
 __device__ __forceinline__ int32_t find_seq(const int32_t* cu, int32_t n_seq, int64_t t) {
@@ -39,18 +43,45 @@ __device__ __forceinline__ void load_tap(const T* state_in, int32_t n, int32_t j
   }
 }
 
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool valid) {
+  const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(s), "l"(gmem), "r"(valid ? 16 : 0)
+               : "memory");
+}
+
 template <typename T>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 3)
 conv1d_silu_kernel(const T* __restrict__ x, T* __restrict__ y, const T* __restrict__ w,
                    const int32_t* __restrict__ cu, int32_t n_seq, int64_t T_tok, int32_t Cc,
                    const T* __restrict__ state_in, T* __restrict__ state_out) {
-  const int32_t n_vec = Cc / kVec;
-  const int32_t cv = blockIdx.y * kThreads + threadIdx.x;
-  if (cv >= n_vec) return;
-  const int32_t c0 = cv * kVec;
-  const int64_t t0 = (int64_t)blockIdx.x * kRunTokens;
-  int64_t t1 = t0 + kRunTokens;
-  if (t1 > T_tok) t1 = T_tok;
+  constexpr int kRowElems = kTileVecs * kVec;
+  constexpr int kChunksPerRow = kRowElems * (int)sizeof(T) / 16;
+  constexpr int kElemsPerChunk = 16 / (int)sizeof(T);
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  T* tile = reinterpret_cast<T*>(smem_raw);   // [kRows][kRowElems], row 0 = token t0 - 3
+
+  const int64_t t0 = (int64_t)blockIdx.x * kTileTokens;
+  const int32_t cbase = blockIdx.y * kRowElems;
+  const int tid = threadIdx.x;
+
+  for (int idx = tid; idx < kRows * kChunksPerRow; idx += kThreads) {
+    const int row = idx / kChunksPerRow, ch = idx % kChunksPerRow;
+    const int64_t t = t0 - 3 + row;
+    const int32_t c = cbase + ch * kElemsPerChunk;
+    const bool valid = t >= 0 && t < T_tok && c < Cc;
+    const T* src = valid ? x + t * Cc + c : x;
+    cp_async16(tile + row * kRowElems + ch * kElemsPerChunk, src, valid);
+  }
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+  __syncthreads();
+
+  const int cv = tid % kTileVecs, tg = tid / kTileVecs;
+  const int32_t c0 = cbase + cv * kVec;
+  if (c0 >= Cc) return;
+  const int64_t ta = t0 + (int64_t)tg * kTokPerThread;
+  if (ta >= T_tok) return;
+  int64_t tb = ta + kTokPerThread;
+  if (tb > T_tok) tb = T_tok;
 
   float wt[4][kVec];
   {
@@ -62,53 +93,46 @@ conv1d_silu_kernel(const T* __restrict__ x, T* __restrict__ y, const T* __restri
       for (int j = 0; j < 4; ++j) wt[j][i] = wr[i * 4 + j];
   }
 
-  int32_t n = (cu == nullptr) ? 0 : find_seq(cu, n_seq, t0);
+  int32_t n = (cu == nullptr) ? 0 : find_seq(cu, n_seq, ta);
   int64_t bos, eos;
   seq_bounds(cu, n, T_tok, bos, eos);
+  auto row_of = [&](int64_t t) { return tile + (int)(t - t0 + 3) * kRowElems + cv * kVec; };
 
   // window[0] = x[t-3], window[1] = x[t-2], window[2] = x[t-1]
   float win[3][kVec];
 #pragma unroll
   for (int j = 0; j < 3; ++j) {
-    const int64_t s = t0 - 3 + j;
-    if (s >= bos) VecIO<T, kVec>::load(x + s * Cc + c0, win[j]);
+    const int64_t s = ta - 3 + j;
+    if (s >= bos) VecIO<T, kVec>::load(row_of(s), win[j]);
     else load_tap(state_in, n, (int32_t)(3 + (s - bos)), Cc, c0, win[j]);
   }
 
-  for (int64_t tb = t0; tb < t1; tb += kPrefetch) {
-    float xin[kPrefetch][kVec];
+  for (int64_t t = ta; t < tb; ++t) {
+    if (t >= eos) {                       // entered the next non-empty sequence
+      while (n + 1 < n_seq && (int64_t)cu[n + 1] <= t) ++n;
+      seq_bounds(cu, n, T_tok, bos, eos);
 #pragma unroll
-    for (int p = 0; p < kPrefetch; ++p)
-      if (tb + p < t1) VecIO<T, kVec>::load(x + (tb + p) * Cc + c0, xin[p]);
+      for (int j = 0; j < 3; ++j) load_tap(state_in, n, j, Cc, c0, win[j]);
+    }
+    float xin[kVec], out[kVec];
+    VecIO<T, kVec>::load(row_of(t), xin);
 #pragma unroll
-    for (int p = 0; p < kPrefetch; ++p) {
-      const int64_t t = tb + p;
-      if (t >= t1) break;
-      if (t >= eos) {                       // entered the next non-empty sequence
-        while (n + 1 < n_seq && (int64_t)cu[n + 1] <= t) ++n;
-        seq_bounds(cu, n, T_tok, bos, eos);
+    for (int i = 0; i < kVec; ++i) {
+      float z = wt[0][i] * win[0][i];
+      z = fmaf(wt[1][i], win[1][i], z);
+      z = fmaf(wt[2][i], win[2][i], z);
+      z = fmaf(wt[3][i], xin[i], z);
+      out[i] = silu(z);
+    }
+    VecIO<T, kVec>::store(y + t * Cc + c0, out);
 #pragma unroll
-        for (int j = 0; j < 3; ++j) load_tap(state_in, n, j, Cc, c0, win[j]);
-      }
-      float out[kVec];
+    for (int i = 0; i < kVec; ++i) {
+      win[0][i] = win[1][i]; win[1][i] = win[2][i]; win[2][i] = xin[i];
+    }
+    if (state_out != nullptr && t == eos - 1) {
 #pragma unroll
-      for (int i = 0; i < kVec; ++i) {
-        float z = wt[0][i] * win[0][i];
-        z = fmaf(wt[1][i], win[1][i], z);
-        z = fmaf(wt[2][i], win[2][i], z);
-        z = fmaf(wt[3][i], xin[p][i], z);
-        out[i] = silu(z);
-      }
-      VecIO<T, kVec>::store(y + t * Cc + c0, out);
-#pragma unroll
-      for (int i = 0; i < kVec; ++i) {
-        win[0][i] = win[1][i]; win[1][i] = win[2][i]; win[2][i] = xin[p][i];
-      }
-      if (state_out != nullptr && t == eos - 1) {
-#pragma unroll
-        for (int j = 0; j < 3; ++j)
-          VecIO<T, kVec>::store(state_out + ((int64_t)n * 3 + j) * Cc + c0, win[j]);
-      }
+      for (int j = 0; j < 3; ++j)
+        VecIO<T, kVec>::store(state_out + ((int64_t)n * 3 + j) * Cc + c0, win[j]);
     }
   }
 }
@@ -133,10 +157,20 @@ template <typename T>
 cudaError_t launch_typed(const void* x, void* y, const void* w, const int32_t* cu, int32_t n_seq,
                          int64_t T_tok, int32_t Cc, const void* sin, void* sout, cudaStream_t st) {
   if (T_tok > 0) {
-    // x: token runs (consecutive CTAs share halo rows in L2), y: channel blocks
-    dim3 grid((unsigned)((T_tok + kRunTokens - 1) / kRunTokens),
-              (unsigned)((Cc / kVec + kThreads - 1) / kThreads));
-    conv1d_silu_kernel<T><<<grid, kThreads, 0, st>>>(
+    const int smem = kRows * kTileVecs * kVec * (int)sizeof(T);
+    static uint64_t attrs_set = 0;   // devices with the shared-memory attribute set
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (smem > 48 * 1024 && (dev >= 64 || !(attrs_set >> dev & 1))) {
+      e = cudaFuncSetAttribute(conv1d_silu_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return e;
+      if (dev < 64) attrs_set |= 1ull << dev;
+    }
+    // x: token tiles (consecutive CTAs share halo rows in L2), y: channel tiles
+    dim3 grid((unsigned)((T_tok + kTileTokens - 1) / kTileTokens),
+              (unsigned)((Cc + kTileVecs * kVec - 1) / (kTileVecs * kVec)));
+    conv1d_silu_kernel<T><<<grid, kThreads, smem, st>>>(
         (const T*)x, (T*)y, (const T*)w, cu, n_seq, T_tok, Cc, (const T*)sin, (T*)sout);
   }
   if (sout != nullptr) {

@@ -195,7 +195,8 @@ constexpr uint32_t kTKQ = 0, kTUW = 128;        // TMEM columns: [KK^T; QK^T], [
 
 __global__ void __launch_bounds__(128)
 chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
-                   const __grid_constant__ CUtensorMap map_v, const float* __restrict__ g,
+                   const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_wu,
+                   const float* __restrict__ g,
                    const float* __restrict__ beta, const int32_t* __restrict__ cu, int32_t n_seq,
                    int64_t T, int32_t Hk, int32_t Hv, uint8_t* __restrict__ ws) {
   const Ws L = ws_layout(T, n_seq, Hv);
@@ -313,30 +314,39 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
       colPk[tid] = sb[tid] * __expf(sG[tid]) * rk[tid];
     }
 
-    // thread t < 64: row t of A (stored transposed) from K K^T; t >= 64: row t-64 of Mqk
+    // thread t < 64: row t of A (stored transposed) from K K^T; t >= 64: row t-64 of Mqk.
+    // Column factors are read into registers first so that the loop is load-free.
     {
       const int r = tid & 63;
       const float Gr = sG[r];
       uint8_t* mq = ws + L.mq + (size_t)(slot * Hv + h) * kMatBytes;
+      const float f = tid < 64 ? sb[r] * rk[r] : rq[r];
+      uint32_t raw[2][32];
+      tmem_ld32_async(tq + kTKQ, raw[0]);
+      tmem_ld32_async(tq + kTKQ + 32, raw[1]);
+      tmem_wait_ld(raw[0], raw[1]);
+#pragma unroll
       for (int cb = 0; cb < 2; ++cb) {
-        float v[32];
-        tmem_ld32(tq + kTKQ + cb * 32, v);
+        float v[32], gi[32], ki[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          gi[e] = sG[cb * 32 + e]; ki[e] = rk[cb * 32 + e]; v[e] = __uint_as_float(raw[cb][e]);
+        }
         if (tid < 64) {
-          const float f = sb[r] * rk[r];
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const int i = cb * 32 + e;
-            At[i * kLd + r] = (i < r) ? f * __expf(Gr - sG[i]) * rk[i] * v[e] : 0.f;
+            v[e] = (i < r) ? f * __expf(Gr - gi[e]) * ki[e] * v[e] : 0.f;
           }
+#pragma unroll
+          for (int e = 0; e < 32; ++e) At[(cb * 32 + e) * kLd + r] = v[e];
         } else {
-          const float f = rq[r];
-          float m[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const int i = cb * 32 + e;
-            m[e] = (i <= r) ? f * __expf(Gr - sG[i]) * rk[i] * v[e] : 0.f;
+            v[e] = (i <= r) ? f * __expf(Gr - gi[e]) * ki[e] * v[e] : 0.f;
           }
-          VecIO<bf16, 32>::store(reinterpret_cast<bf16*>(mq) + r * C + cb * 32, m);
+          VecIO<bf16, 32>::store(reinterpret_cast<bf16*>(mq) + r * C + cb * 32, v);
         }
       }
     }
@@ -398,9 +408,14 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
       const int i = tid & 63, m = tid >> 6;
       const float f = m == 0 ? colP[i] : colPk[i];
       uint8_t* tile = sm + kIPP + m * 8192;
-#pragma unroll 8
-      for (int r = 0; r < 64; ++r)
-        *reinterpret_cast<bf16*>(tile + sw128_off(r, i)) = __float2bfloat16_rn(Tm[r * kLd + i] * f);
+      for (int r0 = 0; r0 < 64; r0 += 16) {
+        float tv[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) tv[r] = Tm[(r0 + r) * kLd + i];
+#pragma unroll
+        for (int r = 0; r < 16; ++r)
+          *reinterpret_cast<bf16*>(tile + sw128_off(r0 + r, i)) = __float2bfloat16_rn(tv[r] * f);
+      }
       float* vec = reinterpret_cast<float*>(ws + L.vecs) + (size_t)(slot * Hv + h) * kVecFloats;
       const float Gl = sG[C - 1];
       if (tid < 64) vec[tid] = __expf(sG[tid]) * rq[tid];
@@ -411,7 +426,6 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     tc_fence_before();
     __syncthreads();
 
-    uint8_t* wu = ws + L.wu + (size_t)(slot * Hv + h) * kWuBytes;
     const uint64_t dpp = smem_desc(smem_u32(sm + kIPP), 16u, 1024u);
     if (tid == 0) {   // [P; Pk] V: rows 0..63 = U~ (M = 128, N = 128, K = 64)
       tc_fence_after();
@@ -430,15 +444,38 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
       for (int hh = 0; hh < 2; ++hh)
         tma_load_2d(sm + kIV + hh * 8192, &map_v, (h + 1) * D + hh * 64, (int32_t)t0, bar_tma);
     }
-    if (warp < 2) {   // U~ row tid -> bf16
-      for (int cb = 0; cb < 4; ++cb) {
-        float v[32];
-        tmem_ld32(tq + kTUW + cb * 32, v);
-        VecIO<bf16, 32>::store(reinterpret_cast<bf16*>(wu) + (C + tid) * D + cb * 32, v);
+    // U~ (rows 0..63 of the result) -> bf16 tile [64][128] in the free A^T region -> TMA store
+    uint8_t* stage_u = sm + kIA;   // 2 swizzled atoms of [64][64]
+    if (warp < 2) {
+#pragma unroll
+      for (int cp = 0; cp < 4; cp += 2) {
+        uint32_t raw[2][32];
+        tmem_ld32_async(tq + kTUW + cp * 32, raw[0]);
+        tmem_ld32_async(tq + kTUW + cp * 32 + 32, raw[1]);
+        tmem_wait_ld(raw[0], raw[1]);
+#pragma unroll
+        for (int hb = 0; hb < 2; ++hb) {
+          const int cb = cp + hb;
+          uint8_t* atom = stage_u + (cb >> 1) * 8192;
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8) {
+            float v8[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) v8[q] = __uint_as_float(raw[hb][c8 * 8 + q]);
+            VecIO<bf16, 8>::store(reinterpret_cast<bf16*>(atom + sw128_off(tid, (cb & 1) * 32 + c8 * 8)), v8);
+          }
+        }
       }
     }
+    fence_async_smem();
     tc_fence_before();
     __syncthreads();
+    const int32_t wrow = (int32_t)(((int64_t)slot * Hv + h) * 2 * C);
+    if (tid == 0) {
+      tma_store_2d(&map_wu, 0, wrow + C, stage_u);
+      tma_store_2d(&map_wu, 64, wrow + C, stage_u + 8192);
+      tma_store_commit();
+    }
     if (tid == 0) {   // [P; Pk] K: rows 64..127 = W (N = 128, K read MN-major across its atoms)
       tc_fence_after();
       const uint64_t dk = smem_desc(smem_u32(sm + kIKQ), 16384u, 1024u);
@@ -451,14 +488,36 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     ph_mma ^= 1u;
     if (__syncthreads_or(!ok)) goto teardown;
     tc_fence_after();
-    if (warp >= 2) {   // -W row (tid - 64) -> bf16
-      for (int cb = 0; cb < 4; ++cb) {
-        float v[32];
-        tmem_ld32(tq + kTUW + cb * 32, v);
+    uint8_t* stage_w = sm + kIT;   // -W (rows 64..127 of the result) staged in the free Tm region
+    if (warp >= 2) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = -v[e];
-        VecIO<bf16, 32>::store(reinterpret_cast<bf16*>(wu) + (tid - 64) * D + cb * 32, v);
+      for (int cp = 0; cp < 4; cp += 2) {
+        uint32_t raw[2][32];
+        tmem_ld32_async(tq + kTUW + cp * 32, raw[0]);
+        tmem_ld32_async(tq + kTUW + cp * 32 + 32, raw[1]);
+        tmem_wait_ld(raw[0], raw[1]);
+#pragma unroll
+        for (int hb = 0; hb < 2; ++hb) {
+          const int cb = cp + hb;
+          uint8_t* atom = stage_w + (cb >> 1) * 8192;
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8) {
+            float v8[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) v8[q] = -__uint_as_float(raw[hb][c8 * 8 + q]);
+            VecIO<bf16, 8>::store(reinterpret_cast<bf16*>(atom + sw128_off(tid - 64, (cb & 1) * 32 + c8 * 8)), v8);
+          }
+        }
       }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {   // both staged tiles must be read out before the next head reuses them
+      tma_store_2d(&map_wu, 0, wrow, stage_w);
+      tma_store_2d(&map_wu, 64, wrow, stage_w + 8192);
+      tma_store_commit();
+      tma_store_wait_read();
     }
     if (j + 1 < G) {
       ok = mbar_wait(bar_tma, ph_tma, err, kErrIntraTma);
@@ -469,6 +528,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
   }
 
 teardown:
+  if (tid == 0) tma_store_wait_all();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 256);
@@ -489,20 +549,23 @@ constexpr int kCU = kCS + 16384;              // U   bf16 [64][64]: 8 KB
 constexpr int kCU2 = kCU + 8192;              // U'  bf16 [64][64]: 8 KB
 constexpr int kCBar = kCU2 + 8192;            // mbarriers + tmem address
 constexpr int kChainSmem = kCBar + 128 + 1024;
-constexpr int kChainThreads = 256;
+// warps 0..7 compute, 8 and 9 issue MMAs, 10 issues the TMA loads
+constexpr int kComputeWarps = 8;
+constexpr int kChainThreads = (kComputeWarps + 3) * 32;
 
 // TMEM columns (M = 128 accumulators, lane = row). A = [-W; Q] S0^T is accumulated in two
-// K halves (lo: dk 0..63, hi: dk 64..127) by two issuers, each double-buffered; dS^T in two
-// K halves (tokens 0..31, 32..63); O2 = [U~; Mqk] U.
+// K halves (lo: dk 0..63, hi: dk 64..127) by the two issuers, each double-buffered; dS^T in
+// two K halves (tokens 0..31, 32..63); O2 = [U~; Mqk] U.
 constexpr uint32_t kTAlo = 0, kTAhi = 128, kTdSlo = 256, kTdShi = 320, kTO2 = 384;
 
-// Wait by every thread, then agree: false if any thread's wait gave up.
-__device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t& phase, int* err, int code) {
-  const bool ok = mbar_wait(bar, phase, err, code);
-  phase ^= 1u;
-  return !__syncthreads_or(!ok);
-}
-
+// One chain CTA: sequence n, value head h, dv rows [tile*64, tile*64 + 64). Per chunk c:
+//   issuers : rA(c) = [-W; Q] S0^T (after "S ready"), rB(c) = K^T U', rO(c) = [U~; Mqk] U
+//             (after "U ready")
+//   compute : U = U~ + rows 0..63 of rA -> U, U' (warps of quadrants 0, 1)      -> "U ready"
+//             S^T <- e^{G_L} S^T + dS^T, bf16 copy (all 8 warps)               -> "S ready"
+//             o = scale (e^{G_r}/|q_r| rows 64..127 of rA + O2) (quadrants 2, 3) -> "stage free"
+//   producer: chunk c+2's loads into stage c % 2 once it is free.
+// The serial path is rA -> U -> rB -> S -> rA(c+1); no thread on it issues anything else.
 __global__ void __launch_bounds__(kChainThreads, 1)
 chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                    const __grid_constant__ CUtensorMap map_wu, const __grid_constant__ CUtensorMap map_mq,
@@ -516,227 +579,250 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
   const int32_t n = blockIdx.x / (NT * Hv);
   const int hk = h / (Hv / Hk);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int quad = warp & 3, half = warp >> 2;     // TMEM lanes 32 quad.., column half
-  const int lrow = quad * 32 + lane;               // this thread's accumulator row (lane)
   int64_t bos, eos;
   seq_bounds(cu, n, T, bos, eos);
   const int nc = (int)((eos - bos + C - 1) / C);
   const int32_t slot0 = prefix[n];
-  const bool issuer0 = tid == 0, issuer1 = tid == 128, issuer2 = tid == 32;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + kCBar);   // [2]
-  uint64_t* bar_A0 = bar_tma + 2;
-  uint64_t* bar_A1 = bar_tma + 3;
-  uint64_t* bar_B0 = bar_tma + 4;
-  uint64_t* bar_B1 = bar_tma + 5;
-  uint64_t* bar_O = bar_tma + 6;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_tma + 7);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kCBar);
+  uint64_t* bar_tma = bars;        // [2] stage landed
+  uint64_t* bar_free = bars + 2;   // [2] stage no longer read (8 compute warps)
+  uint64_t* bar_A0 = bars + 4;
+  uint64_t* bar_A1 = bars + 5;
+  uint64_t* bar_B0 = bars + 6;
+  uint64_t* bar_B1 = bars + 7;
+  uint64_t* bar_O = bars + 8;
+  uint64_t* bar_U = bars + 9;      // U, U' written (8 compute warps)
+  uint64_t* bar_S = bars + 10;     // state bf16 written (8 compute warps)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
 
   if (tid == 0) {
-    for (int i = 0; i < 7; ++i) mbar_init(&bar_tma[i], 1);
+    for (int i = 0; i < 2; ++i) { mbar_init(&bar_tma[i], 1); mbar_init(&bar_free[i], kComputeWarps); }
+    for (int i = 4; i < 9; ++i) mbar_init(&bars[i], 1);
+    mbar_init(bar_U, kComputeWarps);
+    mbar_init(bar_S, kComputeWarps);
     fence_mbar_init();
   }
-  if (issuer2 && nc > 0) {
-    tma_prefetch_desc(&map_q); tma_prefetch_desc(&map_k);
-    tma_prefetch_desc(&map_wu); tma_prefetch_desc(&map_mq);
-  }
   if (warp == 0) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
-
-  // state slice: thread (lrow, half) holds S[tile*64 + half*32 + j][lrow], j < 32
-  constexpr int SJ = DT / 2;
-  float s[SJ];
-  const int64_t sbase = ((int64_t)n * Hv + h) * D * D + (int64_t)(tile * DT + half * SJ) * D + lrow;
-#pragma unroll
-  for (int j = 0; j < SJ; ++j) s[j] = init ? init[sbase + (int64_t)j * D] : 0.f;
-  auto store_state_bf16 = [&]() {
-#pragma unroll
-    for (int c8 = 0; c8 < SJ / 8; ++c8) {
-      float v8[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) v8[q] = s[c8 * 8 + q];
-      VecIO<bf16, 8>::store(reinterpret_cast<bf16*>(sm + kCS + sw128_off(lrow, half * SJ + c8 * 8)), v8);
-    }
-  };
-  store_state_bf16();
-  fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tq = tmem_quadrant(tmem, quad);
-
-  auto issue_loads = [&](int c, int b) {
-    const int64_t t0 = bos + (int64_t)c * C;
-    const int32_t slot = slot0 + c;
-    uint8_t* stg = sm + b * kStage;
-    const int32_t wrow = (int32_t)(((int64_t)slot * Hv + h) * 2 * C);
-    mbar_arrive_expect_tx(&bar_tma[b], kStageTx);
-    for (int hh = 0; hh < 2; ++hh) {
-      tma_load_2d(stg + kSWQ + hh * 16384, &map_wu, hh * 64, wrow, &bar_tma[b]);
-      tma_load_2d(stg + kSWQ + hh * 16384 + 8192, &map_q, hk * D + hh * 64, (int32_t)t0, &bar_tma[b]);
-      tma_load_2d(stg + kSK + hh * 8192, &map_k, hk * D + hh * 64, (int32_t)t0, &bar_tma[b]);
-    }
-    tma_load_2d(stg + kSU, &map_wu, tile * DT, wrow + C, &bar_tma[b]);
-    tma_load_2d(stg + kSM, &map_mq, 0, (int32_t)(((int64_t)slot * Hv + h) * C), &bar_tma[b]);
-    bulk_load(stg + kSVec, ws_ro + L.vecs + ((size_t)slot * Hv + h) * kVecBytes, kVecBytes, &bar_tma[b]);
-  };
-
-  // descriptors: stage 1's are stage 0's plus kStage in the start-address field
-  const uint32_t st0 = smem_u32(sm);
-  const uint64_t dWQ0 = smem_desc(st0 + kSWQ, 16u, 1024u), dK0 = smem_desc(st0 + kSK, 8192u, 1024u);
-  const uint64_t dUM0 = smem_desc(st0 + kSU, 16u, 1024u);
-  auto soff = [](int b) { return (uint64_t)(b * (kStage >> 4)); };
-  const uint64_t dS = smem_desc(smem_u32(sm + kCS), 8192u, 1024u);
-  const uint64_t dU = smem_desc(smem_u32(sm + kCU), 8192u, 1024u);
-  const uint64_t dU2 = smem_desc(smem_u32(sm + kCU2), 8192u, 1024u);
-  constexpr uint32_t kIA = idesc_bf16(128, DT, 0, 1);     // K-major A, MN-major B
-  constexpr uint32_t kIB = idesc_bf16(128, DT, 1, 1);     // MN-major A and B
-
-  // rA half: [-W; Q] S0^T over dk [64 part, 64 part + 64) -> A_part[ab]
-  auto issue_rA = [&](int b, int ab, int part) {
-    const uint64_t a = dWQ0 + soff(b) + (uint64_t)(part * (16384 >> 4));
-    const uint32_t ta = tmem + (part ? kTAhi : kTAlo) + 64 * ab;
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-      mma_bf16(ta, a + 2 * kk, dS + 128 * (4 * part + kk), kIA, kk > 0);
-    mma_commit(part ? bar_A1 : bar_A0);
-  };
-  // rB half: dS^T = K^T U' over tokens [32 part, 32 part + 32)
-  auto issue_rB = [&](int b, int part) {
-    const uint64_t k = dK0 + soff(b);
-    const uint32_t ts = tmem + (part ? kTdShi : kTdSlo);
-#pragma unroll
-    for (int kk = 0; kk < 2; ++kk)
-      mma_bf16(ts, k + 128 * (2 * part + kk), dU2 + 128 * (2 * part + kk), kIB, kk > 0);
-    mma_commit(part ? bar_B1 : bar_B0);
-  };
-  auto issue_rO = [&](int b) {   // rows 64..127 of [U~; Mqk] U
-    const uint64_t a = dUM0 + soff(b);
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) mma_bf16(tmem + kTO2, a + 2 * kk, dU + 128 * kk, kIA, kk > 0);
-    mma_commit(bar_O);
-  };
-
-  uint32_t ph_tma[2] = {0u, 0u}, phA0 = 0u, phA1 = 0u, phB0 = 0u, phB1 = 0u, phO = 0u;
   bool ok = true;
 
-  if (nc > 0) {   // prologue: loads for chunks 0 and 1, rA(0)
-    if (issuer2) {
+  if (warp >= kComputeWarps) {
+    // ---------------------------------------------------------------- issuers / producer
+    if (lane != 0 || nc == 0) goto done;
+    const uint32_t st0 = smem_u32(sm);
+    auto soff = [](int b) { return (uint64_t)(b * (kStage >> 4)); };
+    const uint64_t dS = smem_desc(smem_u32(sm + kCS), 8192u, 1024u);
+    const uint64_t dU = smem_desc(smem_u32(sm + kCU), 8192u, 1024u);
+    const uint64_t dU2 = smem_desc(smem_u32(sm + kCU2), 8192u, 1024u);
+    constexpr uint32_t kIA = idesc_bf16(128, DT, 0, 1);     // K-major A, MN-major B
+    constexpr uint32_t kIB = idesc_bf16(128, DT, 1, 1);     // MN-major A and B
+    if (warp == kComputeWarps + 2) {   // TMA producer
+      if (nc > 0) tma_prefetch_desc(&map_q);
+      auto issue_loads = [&](int c, int b) {
+        const int64_t t0 = bos + (int64_t)c * C;
+        const int32_t slot = slot0 + c;
+        uint8_t* stg = sm + b * kStage;
+        const int32_t wrow = (int32_t)(((int64_t)slot * Hv + h) * 2 * C);
+        mbar_arrive_expect_tx(&bar_tma[b], kStageTx);
+        for (int hh = 0; hh < 2; ++hh) {
+          tma_load_2d(stg + kSWQ + hh * 16384, &map_wu, hh * 64, wrow, &bar_tma[b]);
+          tma_load_2d(stg + kSWQ + hh * 16384 + 8192, &map_q, hk * D + hh * 64, (int32_t)t0, &bar_tma[b]);
+          tma_load_2d(stg + kSK + hh * 8192, &map_k, hk * D + hh * 64, (int32_t)t0, &bar_tma[b]);
+        }
+        tma_load_2d(stg + kSU, &map_wu, tile * DT, wrow + C, &bar_tma[b]);
+        tma_load_2d(stg + kSM, &map_mq, 0, (int32_t)(((int64_t)slot * Hv + h) * C), &bar_tma[b]);
+        bulk_load(stg + kSVec, ws_ro + L.vecs + ((size_t)slot * Hv + h) * kVecBytes, kVecBytes, &bar_tma[b]);
+      };
       issue_loads(0, 0);
       if (nc > 1) issue_loads(1, 1);
+      for (int c = 0; c + 2 < nc; ++c) {
+        if (!mbar_wait(&bar_free[c & 1], (uint32_t)(c >> 1) & 1u, err_word, kErrChainTma)) break;
+        issue_loads(c + 2, c & 1);
+      }
+      goto done;
     }
-    ok = wait_all(&bar_tma[0], ph_tma[0], err_word, kErrChainTma);
-    if (ok && (issuer0 || issuer1)) { tc_fence_after(); issue_rA(0, 0, issuer1 ? 1 : 0); }
+    const int part = warp - kComputeWarps;   // 0: lo halves and O2, 1: hi halves
+    const uint64_t dWQ = smem_desc(st0 + kSWQ, 16u, 1024u) + (uint64_t)(part * (16384 >> 4));
+    const uint64_t dK = smem_desc(st0 + kSK, 8192u, 1024u);
+    const uint64_t dUM = smem_desc(st0 + kSU, 16u, 1024u);
+    auto issue_rA = [&](int b) {
+      const uint32_t ta = tmem + (part ? kTAhi : kTAlo) + 64 * b;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16(ta, dWQ + soff(b) + 2 * kk, dS + 128 * (4 * part + kk), kIA, kk > 0);
+      mma_commit(part ? bar_A1 : bar_A0);
+    };
+    uint32_t phT[2] = {0u, 0u};
+    // rA(0): chunk 0 landed and the initial state is in shared memory
+    if (!mbar_wait(&bar_tma[0], phT[0], err_word, kErrChainTma) ||
+        !mbar_wait(bar_S, 0u, err_word, kErrChainMma)) goto done;
+    phT[0] ^= 1u;
+    tc_fence_after();
+    issue_rA(0);
+    for (int c = 0; c < nc; ++c) {
+      const int b = c & 1;
+      if (!mbar_wait(bar_U, (uint32_t)c & 1u, err_word, kErrChainMma)) break;
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < 2; ++kk)   // dS^T = K^T U' over tokens [32 part, 32 part + 32)
+        mma_bf16(tmem + (part ? kTdShi : kTdSlo), dK + soff(b) + 128 * (2 * part + kk),
+                 dU2 + 128 * (2 * part + kk), kIB, kk > 0);
+      mma_commit(part ? bar_B1 : bar_B0);
+      if (part == 0) {   // rows 64..127 of [U~; Mqk] U
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) mma_bf16(tmem + kTO2, dUM + soff(b) + 2 * kk, dU + 128 * kk, kIA, kk > 0);
+        mma_commit(bar_O);
+      }
+      if (c + 1 < nc) {
+        if (!mbar_wait(&bar_tma[b ^ 1], phT[b ^ 1], err_word, kErrChainTma) ||
+            !mbar_wait(bar_S, (uint32_t)(c + 1) & 1u, err_word, kErrChainMma)) break;
+        phT[b ^ 1] ^= 1u;
+        tc_fence_after();
+        issue_rA(b ^ 1);
+      }
+    }
+    goto done;
   }
 
-  for (int c = 0; ok && c < nc; ++c) {
-    const int b = c & 1;                 // stage and A buffer of chunk c
-    const int64_t t0 = bos + (int64_t)c * C;
-    const int len = (int)(eos - t0 < C ? eos - t0 : C);
-    const float* vec = reinterpret_cast<const float*>(sm + b * kStage + kSVec);
-    const bool more = c + 1 < nc;
+  {
+    // ------------------------------------------------------------------- compute warps
+    const int quad = warp & 3, half = warp >> 2;     // TMEM lanes 32 quad.., column half
+    const int lrow = quad * 32 + lane;               // this thread's accumulator row (lane)
+    const uint32_t tq = tmem_quadrant(tmem, quad);
 
-    // U = U~ + (-W S0^T) rows 0..63 (quadrants 0, 1), U and U' to bf16
-    {
-      const bool okA = mbar_wait(bar_A0, phA0, err_word, kErrChainMma) &&
-                       mbar_wait(bar_A1, phA1, err_word, kErrChainMma);
-      phA0 ^= 1u; phA1 ^= 1u;
-      if (__syncthreads_or(!okA)) { ok = false; break; }
-    }
-    tc_fence_after();
-    float os = 0.f;
-    if (quad < 2) {
-      const int r = lrow;
-      const float us = vec[64 + r];
-      float a0[32], a1[32];
-      tmem_ld32(tq + kTAlo + 64 * b + half * 32, a0);
-      tmem_ld32(tq + kTAhi + 64 * b + half * 32, a1);
-      const uint8_t* ut = sm + b * kStage + kSU;
+    // state slice: thread (lrow, half) holds S[tile*64 + half*32 + j][lrow], j < 32
+    constexpr int SJ = DT / 2;
+    float s[SJ];
+    const int64_t sbase = ((int64_t)n * Hv + h) * D * D + (int64_t)(tile * DT + half * SJ) * D + lrow;
 #pragma unroll
-      for (int c8 = 0; c8 < 4; ++c8) {
-        float v8[8], w8[8];
-        VecIO<bf16, 8>::load(reinterpret_cast<const bf16*>(ut + sw128_off(r, half * 32 + c8 * 8)), v8);
+    for (int j = 0; j < SJ; ++j) s[j] = init ? init[sbase + (int64_t)j * D] : 0.f;
+    auto store_state_bf16 = [&]() {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) { v8[q] += a0[c8 * 8 + q] + a1[c8 * 8 + q]; w8[q] = us * v8[q]; }
-        const uint32_t off = sw128_off(r, half * 32 + c8 * 8);
-        VecIO<bf16, 8>::store(reinterpret_cast<bf16*>(sm + kCU + off), v8);
-        VecIO<bf16, 8>::store(reinterpret_cast<bf16*>(sm + kCU2 + off), w8);
+      for (int c8 = 0; c8 < SJ / 8; ++c8) {
+        float v8[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v8[q] = s[c8 * 8 + q];
+        VecIO<bf16, 8>::store(reinterpret_cast<bf16*>(sm + kCS + sw128_off(lrow, half * SJ + c8 * 8)), v8);
       }
-    } else {
-      os = vec[lrow - 64];   // the output row scale, before the stage is reused
-    }
+    };
+    auto warp_arrive = [&](uint64_t* bar) {   // one arrival per warp after all its lanes
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar);
+    };
+    store_state_bf16();
     fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (issuer0 || issuer1) { tc_fence_after(); issue_rB(b, issuer1 ? 1 : 0); }
+    warp_arrive(bar_S);
 
-    // state update: S^T <- e^{G_L} S^T + dS^T (both K halves)
-    {
-      const bool okB = mbar_wait(bar_B0, phB0, err_word, kErrChainMma) &&
-                       mbar_wait(bar_B1, phB1, err_word, kErrChainMma);
-      phB0 ^= 1u; phB1 ^= 1u;
-      if (__syncthreads_or(!okB)) { ok = false; break; }
-    }
-    tc_fence_after();
-    {
-      const float decay_last = vec[128];
-      float d0[32], d1[32];
-      tmem_ld32(tq + kTdSlo + half * 32, d0);
-      tmem_ld32(tq + kTdShi + half * 32, d1);
-#pragma unroll
-      for (int e = 0; e < SJ; ++e) s[e] = fmaf(decay_last, s[e], d0[e] + d1[e]);
-      store_state_bf16();
-    }
-    if (more) {   // chunk c+1's inputs must have landed before its rA
-      const bool okT = mbar_wait(&bar_tma[b ^ 1], ph_tma[b ^ 1], err_word, kErrChainTma);
-      ph_tma[b ^ 1] ^= 1u;
-      fence_async_smem();
-      tc_fence_before();
-      if (__syncthreads_or(!okT)) { ok = false; break; }
-    } else {
-      fence_async_smem();
-      tc_fence_before();
-      __syncthreads();
-    }
-    if (more && (issuer0 || issuer1)) { tc_fence_after(); issue_rA(b ^ 1, b ^ 1, issuer1 ? 1 : 0); }
-    if (issuer2) { tc_fence_after(); issue_rO(b); }
+    uint32_t phA = 0u, phB = 0u;
+    for (int c = 0; c < nc; ++c) {
+      const int b = c & 1;
+      const int64_t t0 = bos + (int64_t)c * C;
+      const int len = (int)(eos - t0 < C ? eos - t0 : C);
+      const float* vec = reinterpret_cast<const float*>(sm + b * kStage + kSVec);
 
-    // chunk c's output while rA(c+1) runs: o_r = scale (e^{G_r}/|q_r| O1_r + O2_r)
-    {
-      const bool okO = mbar_wait(bar_O, phO, err_word, kErrChainMma);
-      phO ^= 1u;
-      if (__syncthreads_or(!okO)) { ok = false; break; }
-    }
-    tc_fence_after();
-    if (issuer2 && c + 2 < nc) issue_loads(c + 2, b);
-    if (quad >= 2) {
-      const int r = lrow - 64;
-      float a0[32], a1[32], o2[32];
-      tmem_ld32(tq + kTAlo + 64 * b + half * 32, a0);
-      tmem_ld32(tq + kTAhi + 64 * b + half * 32, a1);
-      tmem_ld32(tq + kTO2 + half * 32, o2);
-      if (r < len) {
-        bf16* dst = o + ((t0 + r) * Hv + h) * (int64_t)D + tile * DT + half * 32;
+      // U = U~ + (-W S0^T): rows 0..63 (quadrants 0, 1) -> U and U' in bf16
+      if (!(ok = mbar_wait(bar_A0, phA, err_word, kErrChainMma) && mbar_wait(bar_A1, phA, err_word, kErrChainMma))) break;
+      phA ^= 1u;
+      tc_fence_after();
+      float os = 0.f;
+      if (quad < 2) {
+        // the previous chunk's O2 has finished reading U before it is overwritten
+        if (c > 0 && !(ok = mbar_wait(bar_O, (uint32_t)(c - 1) & 1u, err_word, kErrChainMma))) break;
+        const int r = lrow;
+        const float us = vec[64 + r];
+        uint32_t a0[32], a1[32];
+        tmem_ld32_async(tq + kTAlo + 64 * b + half * 32, a0);
+        tmem_ld32_async(tq + kTAhi + 64 * b + half * 32, a1);
+        const uint8_t* ut = sm + b * kStage + kSU;
+        float ub[32];
 #pragma unroll
         for (int c8 = 0; c8 < 4; ++c8) {
           float v8[8];
+          VecIO<bf16, 8>::load(reinterpret_cast<const bf16*>(ut + sw128_off(r, half * 32 + c8 * 8)), v8);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) ub[c8 * 8 + q] = v8[q];
+        }
+        tmem_wait_ld(a0, a1);
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8) {
+          float v8[8], w8[8];
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
-            const int e = c8 * 8 + q;
-            v8[q] = scale * fmaf(os, a0[e] + a1[e], o2[e]);
+            v8[q] = ub[c8 * 8 + q] + __uint_as_float(a0[c8 * 8 + q]) + __uint_as_float(a1[c8 * 8 + q]);
+            w8[q] = us * v8[q];
           }
-          VecIO<bf16, 8>::store(dst + c8 * 8, v8);
+          const uint32_t off = sw128_off(r, half * 32 + c8 * 8);
+          VecIO<bf16, 8>::store(reinterpret_cast<bf16*>(sm + kCU + off), v8);
+          VecIO<bf16, 8>::store(reinterpret_cast<bf16*>(sm + kCU2 + off), w8);
         }
+        fence_async_smem();
+      } else {
+        os = vec[lrow - 64];
       }
+      tc_fence_before();
+      warp_arrive(bar_U);
+
+      // state update: S^T <- e^{G_L} S^T + dS^T (both K halves)
+      if (!(ok = mbar_wait(bar_B0, phB, err_word, kErrChainMma) && mbar_wait(bar_B1, phB, err_word, kErrChainMma))) break;
+      phB ^= 1u;
+      tc_fence_after();
+      {
+        const float decay_last = vec[128];
+        uint32_t d0[32], d1[32];
+        tmem_ld32_async(tq + kTdSlo + half * 32, d0);
+        tmem_ld32_async(tq + kTdShi + half * 32, d1);
+        tmem_wait_ld(d0, d1);
+#pragma unroll
+        for (int e = 0; e < SJ; ++e)
+          s[e] = fmaf(decay_last, s[e], __uint_as_float(d0[e]) + __uint_as_float(d1[e]));
+        store_state_bf16();
+      }
+      fence_async_smem();
+      tc_fence_before();
+      warp_arrive(bar_S);
+
+      // chunk c's output (quadrants 2, 3): o_r = scale (e^{G_r}/|q_r| O1_r + O2_r)
+      if (quad >= 2) {
+        if (!(ok = mbar_wait(bar_O, (uint32_t)c & 1u, err_word, kErrChainMma))) break;
+        tc_fence_after();
+        const int r = lrow - 64;
+        uint32_t a0[32], a1[32];
+        tmem_ld32_async(tq + kTAlo + 64 * b + half * 32, a0);
+        tmem_ld32_async(tq + kTAhi + 64 * b + half * 32, a1);
+        tmem_wait_ld(a0, a1);
+        float o1[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o1[e] = os * (__uint_as_float(a0[e]) + __uint_as_float(a1[e]));
+        uint32_t o2[32];
+        tmem_ld32_async(tq + kTO2 + half * 32, o2);
+        tmem_wait_ld(o2);
+        if (r < len) {
+          bf16* dst = o + ((t0 + r) * Hv + h) * (int64_t)D + tile * DT + half * 32;
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8) {
+            float v8[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) v8[q] = scale * (o1[c8 * 8 + q] + __uint_as_float(o2[c8 * 8 + q]));
+            VecIO<bf16, 8>::store(dst + c8 * 8, v8);
+          }
+        }
+        tc_fence_before();
+      }
+      warp_arrive(&bar_free[b]);
+    }
+    if (ok && fin != nullptr) {
+#pragma unroll
+      for (int j = 0; j < SJ; ++j) fin[sbase + (int64_t)j * D] = s[j];
     }
   }
 
-  if (ok && fin != nullptr) {
-#pragma unroll
-    for (int j = 0; j < SJ; ++j) fin[sbase + (int64_t)j * D] = s[j];
-  }
+done:
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
@@ -812,7 +898,7 @@ cudaError_t launch_prefill_chunk_tc(const void* q, const void* k, const void* v,
                                             reinterpret_cast<int*>(ws + L.err));
   if (T > 0) {
     dim3 gi((unsigned)slots, (unsigned)Hk);
-    chunk_intra_kernel<<<gi, 128, kIntraSmem, stream>>>(mq, mk, mv, g, beta, cu, n_seq, T, Hk, Hv, ws);
+    chunk_intra_kernel<<<gi, 128, kIntraSmem, stream>>>(mq, mk, mv, mwu, g, beta, cu, n_seq, T, Hk, Hv, ws);
   }
   dim3 gc((unsigned)((int64_t)n_seq * Hv * NT));
   chunk_chain_kernel<<<gc, kChainThreads, kChainSmem, stream>>>(mq, mk, mwu, mmq, cu, n_seq, T, Hk, Hv, ws,
