@@ -187,8 +187,8 @@ constexpr int kIA = 65536;                      // A^T fp32 [64][kLd] (A^T[i][r]
 constexpr int kIT = kIA + 64 * kLd * 4;         // Tm  fp32 [64][kLd]
 constexpr int kITmp = kIT + 64 * kLd * 4;       // per-warp block scratch fp32 [4][16][kLd16]
 constexpr int kLd16 = 24;
-constexpr int kIVec = kITmp + 4 * 16 * kLd16 * 4;   // rq, rk, G, colP, colPk [5][64]
-constexpr int kIGB = kIVec + 5 * 64 * 4;        // g, beta of every value head [2][kMaxG][64]
+constexpr int kIVec = kITmp + 4 * 16 * kLd16 * 4;   // rq, rk, G, colP, colPk, colInv [6][64]
+constexpr int kIGB = kIVec + 6 * 64 * 4;        // g, beta of every value head [2][kMaxG][64]
 constexpr int kIBar = kIGB + 2 * kMaxG * 64 * 4;    // 2 mbarriers + tmem address
 constexpr int kIntraSmem = kIBar + 64 + 1024;   // + alignment slack
 constexpr uint32_t kTKQ = 0, kTUW = 128;        // TMEM columns: [KK^T; QK^T], [P;Pk] V or K
@@ -222,6 +222,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
   float* sG = rq + 128;
   float* colP = rq + 192;
   float* colPk = rq + 256;
+  float* colInv = rq + 320;
   float* gAll = reinterpret_cast<float*>(sm + kIGB);
   float* bAll = gAll + kMaxG * 64;
   uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + kIBar);
@@ -309,68 +310,94 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     }
     __syncthreads();
     const float* sb = bAll + j * 64;
-    if (tid < 64) {   // column factors of P = Tm diag(beta) and Pk = Tm diag(beta e^G / |k|)
+    if (tid < 64) {   // column factors of P = Tm diag(beta), Pk = Tm diag(beta e^G / |k|), A, Mqk
       colP[tid] = sb[tid];
       colPk[tid] = sb[tid] * __expf(sG[tid]) * rk[tid];
+      colInv[tid] = -sG[C - 1] < 60.f ? __expf(-sG[tid]) * rk[tid] : 0.f;
     }
+    __syncthreads();
 
     // thread t < 64: row t of A (stored transposed) from K K^T; t >= 64: row t-64 of Mqk.
-    // Column factors are read into registers first so that the loop is load-free.
+    // e^{G_r - G_i} = e^{G_r} e^{-G_i} with the column factors e^{-G_i}/|k_i| in shared
+    // memory; when the chunk's cumulative decay could leave the fp32 range the difference
+    // form is used instead (one exp per element).
     {
       const int r = tid & 63;
       const float Gr = sG[r];
+      const bool factored = -sG[C - 1] < 60.f;     // G is non-increasing: G_63 is the minimum
       uint8_t* mq = ws + L.mq + (size_t)(slot * Hv + h) * kMatBytes;
       const float f = tid < 64 ? sb[r] * rk[r] : rq[r];
+      const float fr = factored ? f * __expf(Gr) : f;
       uint32_t raw[2][32];
       tmem_ld32_async(tq + kTKQ, raw[0]);
       tmem_ld32_async(tq + kTKQ + 32, raw[1]);
       tmem_wait_ld(raw[0], raw[1]);
 #pragma unroll
       for (int cb = 0; cb < 2; ++cb) {
-        float v[32], gi[32], ki[32];
+        float v[32], ci[32];
+        if (factored) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ci[e] = colInv[cb * 32 + e];
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ci[e] = __expf(Gr - sG[cb * 32 + e]) * rk[cb * 32 + e];
+        }
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          gi[e] = sG[cb * 32 + e]; ki[e] = rk[cb * 32 + e]; v[e] = __uint_as_float(raw[cb][e]);
+          const int i = cb * 32 + e;
+          const bool keep = tid < 64 ? (i < r) : (i <= r);
+          v[e] = keep ? fr * ci[e] * __uint_as_float(raw[cb][e]) : 0.f;
         }
         if (tid < 64) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int i = cb * 32 + e;
-            v[e] = (i < r) ? f * __expf(Gr - gi[e]) * ki[e] * v[e] : 0.f;
-          }
-#pragma unroll
           for (int e = 0; e < 32; ++e) At[(cb * 32 + e) * kLd + r] = v[e];
         } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int i = cb * 32 + e;
-            v[e] = (i <= r) ? f * __expf(Gr - gi[e]) * ki[e] * v[e] : 0.f;
-          }
           VecIO<bf16, 32>::store(reinterpret_cast<bf16*>(mq) + r * C + cb * 32, v);
         }
       }
     }
     __syncthreads();
 
-    // Tm = (I + A)^{-1}: diagonal 16x16 blocks by forward substitution, one warp each
+    // Tm = (I + A)^{-1}. Diagonal 16x16 blocks, one warp each: with L the block of A
+    // (strictly lower, L^16 = 0), (I + L)^{-1} = (I - L)(I + L^2)(I + L^4)(I + L^8), three
+    // squarings and three products on warp-level tf32 MMAs. X lives in the Tm block, the
+    // current power of L in the warp's scratch.
     {
       const int b0 = warp * 16;
-      const int jc = lane & 15;
-      float x[16];
-#pragma unroll
-      for (int r = 0; r < 16; ++r) {
-        float s = (r == jc) ? 1.f : 0.f;
-#pragma unroll
-        for (int i = 0; i < r; ++i) s = fmaf(-At[(b0 + i) * kLd + b0 + r], x[i], s);
-        x[r] = s;
-      }
-      if (lane < 16) {
-#pragma unroll
-        for (int r = 0; r < 16; ++r) Tm[(b0 + r) * kLd + b0 + jc] = x[r];
+      const int gq = lane >> 2, tq4 = lane & 3;
+      float* X = Tm + b0 * kLd + b0;
+      for (int e = lane; e < 256; e += 32) {
+        const int i = e >> 4, k = e & 15;
+        const float l = At[(b0 + k) * kLd + b0 + i];        // L(i, k)
+        X[i * kLd + k] = (i == k ? 1.f : 0.f) - l;
+        scratch[i * kLd16 + k] = l;
       }
       for (int e = lane; e < 16 * 64; e += 32) {   // blocks above the diagonal are zero
         const int r = e >> 6, c = e & 63;
         if (c >= b0 + 16) Tm[(b0 + r) * kLd + c] = 0.f;
+      }
+      __syncwarp();
+      auto store_frag = [&](float* M, int pitch, const float (&c)[2][4], bool add) {
+#pragma unroll
+        for (int nh = 0; nh < 2; ++nh) {
+          float* r0 = M + gq * pitch + 8 * nh + 2 * tq4;
+          float* r8 = r0 + 8 * pitch;
+          if (add) { r0[0] += c[nh][0]; r0[1] += c[nh][1]; r8[0] += c[nh][2]; r8[1] += c[nh][3]; }
+          else { r0[0] = c[nh][0]; r0[1] = c[nh][1]; r8[0] = c[nh][2]; r8[1] = c[nh][3]; }
+        }
+      };
+#pragma unroll 1
+      for (int step = 0; step < 3; ++step) {
+        float p2[2][4] = {};   // P <- P P  (L^2, L^4, L^8)
+        block_mma16<false>(p2, scratch, kLd16, 0, 0, scratch, kLd16, 0, 0, lane);
+        __syncwarp();
+        store_frag(scratch, kLd16, p2, false);
+        __syncwarp();
+        float xp[2][4] = {};   // X <- X + X P
+        block_mma16<false>(xp, X, kLd, 0, 0, scratch, kLd16, 0, 0, lane);
+        __syncwarp();
+        store_frag(X, kLd, xp, true);
+        __syncwarp();
       }
     }
     __syncthreads();
