@@ -361,7 +361,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     // Tm = (I + A)^{-1}. Diagonal 16x16 blocks, one warp each: with L the block of A
     // (strictly lower, L^16 = 0), (I + L)^{-1} = (I - L)(I + L^2)(I + L^4)(I + L^8), three
     // squarings and three products on warp-level tf32 MMAs. X lives in the Tm block, the
-    // current power of L in the warp's scratch.
+    // current power of L in the warp's scratch. Blocks above the diagonal are not stored.
     {
       const int b0 = warp * 16;
       const int gq = lane >> 2, tq4 = lane & 3;
@@ -371,10 +371,6 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
         const float l = At[(b0 + k) * kLd + b0 + i];        // L(i, k)
         X[i * kLd + k] = (i == k ? 1.f : 0.f) - l;
         scratch[i * kLd16 + k] = l;
-      }
-      for (int e = lane; e < 16 * 64; e += 32) {   // blocks above the diagonal are zero
-        const int r = e >> 6, c = e & 63;
-        if (c >= b0 + 16) Tm[(b0 + r) * kLd + c] = 0.f;
       }
       __syncwarp();
       auto store_frag = [&](float* M, int pitch, const float (&c)[2][4], bool add) {
@@ -435,10 +431,13 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
       const int i = tid & 63, m = tid >> 6;
       const float f = m == 0 ? colP[i] : colPk[i];
       uint8_t* tile = sm + kIPP + m * 8192;
+      // Tm is block lower triangular; its blocks above the diagonal are never written
+      // (the staging tiles reuse that memory), so they are masked here
       for (int r0 = 0; r0 < 64; r0 += 16) {
         float tv[16];
+        const bool live = r0 >= (i & ~15);
 #pragma unroll
-        for (int r = 0; r < 16; ++r) tv[r] = Tm[(r0 + r) * kLd + i];
+        for (int r = 0; r < 16; ++r) tv[r] = live ? Tm[(r0 + r) * kLd + i] : 0.f;
 #pragma unroll
         for (int r = 0; r < 16; ++r)
           *reinterpret_cast<bf16*>(tile + sw128_off(r0 + r, i)) = __float2bfloat16_rn(tv[r] * f);

@@ -12,7 +12,11 @@
 namespace gdn {
 namespace sm100 {
 
-constexpr uint32_t kSpinLimit = 1u << 26;
+// A waiting thread is suspended in hardware until the phase completes or kSuspendNs
+// elapses, so waiting warps do not take issue slots from working ones; kSpinLimit such
+// waits bound the total at a few seconds.
+constexpr uint32_t kSuspendNs = 1000;
+constexpr uint32_t kSpinLimit = 1u << 22;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -41,9 +45,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n .reg .pred p;\n"
-      " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
       " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs) : "memory");
   return ok != 0;
 }
 
