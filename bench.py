@@ -295,16 +295,16 @@ def main():
                 "peak": tc_sust, "unit": "TFLOP/s", "frac": pre_tflops / tc_sust,
                 "peak_kind": f"bf16 dense sustained ({peak_src})",
                 "algorithmic_per_launch": prefill_flops_per_token() * T,
-                "traffic": TRAFFIC.get("prefill")}
+                "traffic": traffic("prefill", T)}
     elif dominant == "decode":
         roof = {"kernel": "gdn_decode_step", "bound": "hbm", "achieved": dec_gbs, "peak": hbm_gbs,
                 "unit": "GB/s", "frac": dec_gbs / hbm_gbs, "peak_kind": f"HBM copy ({peak_src})",
                 "algorithmic_per_launch": decode_bytes(args.decode_batch),
-                "traffic": TRAFFIC.get("decode")}
+                "traffic": traffic("decode", args.decode_batch)}
     else:
         roof = {"kernel": "gdn_conv1d_silu", "bound": "hbm", "achieved": conv_gbs, "peak": hbm_gbs,
                 "unit": "GB/s", "frac": conv_gbs / hbm_gbs, "peak_kind": f"HBM copy ({peak_src})",
-                "algorithmic_per_launch": conv_bytes(T), "traffic": TRAFFIC.get("conv")}
+                "algorithmic_per_launch": conv_bytes(T), "traffic": traffic("conv", T)}
 
     # ---- end to end: host buffers in pinned memory, copies inside the timed region
     e2e = None
@@ -383,9 +383,17 @@ def gdn_prefill_launches() -> int:
     return 3
 
 
-# DRAM traffic per launch from an ncu capture of the same kernel (bytes), or None when
-# the kernel changed since the counters were taken.
-TRAFFIC = {"prefill": None, "conv": None, "decode": None}
+# DRAM traffic (bytes, dram__bytes_read.sum + dram__bytes_write.sum) from one ncu capture
+# of each kernel on the small case (T = 8192, decode batch 64), per unit processed (token
+# for the prefill kernels and the conv, sequence for the decode step), scaled to the
+# benchmark's launch; None when the kernel changed since the capture.
+TRAFFIC_PER_UNIT = {"prefill": (374.95e6 + 404.60e6) / 8192, "conv": 288.99e6 / 8192,
+                    "decode": 354.37e6 / 64}
+
+
+def traffic(kernel: str, units: int):
+    per = TRAFFIC_PER_UNIT.get(kernel)
+    return None if per is None else per * units
 
 if __name__ == "__main__":
     main()
