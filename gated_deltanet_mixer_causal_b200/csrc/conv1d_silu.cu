@@ -8,7 +8,10 @@
 // shared memory with 16-byte cp.async (zero-filled outside [0, T)), so many bytes are in
 // flight per SM without holding them in registers; then each thread slides a 3-token
 // window over 16 consecutive tokens of 8 channels and writes 16-byte vectors, consecutive
-// threads covering consecutive channels (1 KB contiguous per token row for bf16).
+// threads covering consecutive channels (1 KB contiguous per token row for bf16). Runs
+// that lie inside one sequence with their three predecessors take a fully unrolled path
+// (no per-token boundary tests, the window in renamed registers); the general path
+// handles sequence starts, carried taps and ragged ends.
 #include "common.cuh"
 #include "launch.h"
 
@@ -50,7 +53,7 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool va
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads, 3)
+__global__ void __launch_bounds__(kThreads, 2)
 conv1d_silu_kernel(const T* __restrict__ x, T* __restrict__ y, const T* __restrict__ w,
                    const int32_t* __restrict__ cu, int32_t n_seq, int64_t T_tok, int32_t Cc,
                    const T* __restrict__ state_in, T* __restrict__ state_out) {
@@ -97,6 +100,38 @@ conv1d_silu_kernel(const T* __restrict__ x, T* __restrict__ y, const T* __restri
   int64_t bos, eos;
   seq_bounds(cu, n, T_tok, bos, eos);
   auto row_of = [&](int64_t t) { return tile + (int)(t - t0 + 3) * kRowElems + cv * kVec; };
+
+  if (ta - 3 >= bos && tb == ta + kTokPerThread && tb <= eos) {
+    // the run and its three predecessors lie in one sequence (every run of a long sequence
+    // but its first): fully unrolled, the sliding window lives in renamed registers
+    float w0[kVec], w1[kVec], w2[kVec];
+    VecIO<T, kVec>::load(row_of(ta - 3), w0);
+    VecIO<T, kVec>::load(row_of(ta - 2), w1);
+    VecIO<T, kVec>::load(row_of(ta - 1), w2);
+    T* yp = y + ta * Cc + c0;
+#pragma unroll
+    for (int k = 0; k < kTokPerThread; ++k) {
+      float xin[kVec], out[kVec];
+      VecIO<T, kVec>::load(row_of(ta + k), xin);
+#pragma unroll
+      for (int i = 0; i < kVec; ++i) {
+        float z = wt[0][i] * w0[i];
+        z = fmaf(wt[1][i], w1[i], z);
+        z = fmaf(wt[2][i], w2[i], z);
+        z = fmaf(wt[3][i], xin[i], z);
+        out[i] = silu(z);
+      }
+      VecIO<T, kVec>::store(yp + (int64_t)k * Cc, out);
+#pragma unroll
+      for (int i = 0; i < kVec; ++i) { w0[i] = w1[i]; w1[i] = w2[i]; w2[i] = xin[i]; }
+    }
+    if (state_out != nullptr && tb == eos) {   // the run ends the sequence: carry its taps
+      VecIO<T, kVec>::store(state_out + ((int64_t)n * 3 + 0) * Cc + c0, w0);
+      VecIO<T, kVec>::store(state_out + ((int64_t)n * 3 + 1) * Cc + c0, w1);
+      VecIO<T, kVec>::store(state_out + ((int64_t)n * 3 + 2) * Cc + c0, w2);
+    }
+    return;
+  }
 
   // window[0] = x[t-3], window[1] = x[t-2], window[2] = x[t-1]
   float win[3][kVec];
