@@ -179,7 +179,8 @@ __device__ __forceinline__ void block_mma16(float (&c)[2][4], const float* Xs, i
 // shared memory of the intra kernel (offsets from a 1024-aligned base)
 constexpr int kMaxG = kPrefillTcMaxG;           // value heads per key head on this path
 constexpr int kIKQ = 0;                         // [K0 | Q0 | K1 | Q1]: [K; Q] is one 128-row operand
-constexpr int kIV = 32768;                      // V tile of one value head: 2 atoms
+constexpr int kIV = 32768;                      // V tile of one value head: 2 atoms; once [K; Q] K^T
+                                                // is done the Q atoms hold a second V tile
 constexpr int kIPP = 49152;                     // [P | Pk] bf16, K-major
 constexpr int kLd = 72;                         // fp32 row pitch of A^T and Tm (= 8 mod 32:
                                                 // conflict-free tf32 fragment loads)
@@ -189,7 +190,7 @@ constexpr int kITmp = kIT + 64 * kLd * 4;       // per-warp block scratch fp32 [
 constexpr int kLd16 = 24;
 constexpr int kIVec = kITmp + 4 * 16 * kLd16 * 4;   // rq, rk, G, colP, colPk, colInv [6][64]
 constexpr int kIGB = kIVec + 6 * 64 * 4;        // g, beta of every value head [2][kMaxG][64]
-constexpr int kIBar = kIGB + 2 * kMaxG * 64 * 4;    // 2 mbarriers + tmem address
+constexpr int kIBar = kIGB + 2 * kMaxG * 64 * 4;    // 4 mbarriers + tmem address
 constexpr int kIntraSmem = kIBar + 64 + 1024;   // + alignment slack
 constexpr uint32_t kTKQ = 0, kTUW = 128;        // TMEM columns: [KK^T; QK^T], [P;Pk] V or K
 
@@ -219,19 +220,21 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
   float* scratch = reinterpret_cast<float*>(sm + kITmp) + warp * 16 * kLd16;
   float* rq = reinterpret_cast<float*>(sm + kIVec);
   float* rk = rq + 64;
-  float* sG = rq + 128;
   float* colP = rq + 192;
   float* colPk = rq + 256;
   float* colInv = rq + 320;
   float* gAll = reinterpret_cast<float*>(sm + kIGB);
   float* bAll = gAll + kMaxG * 64;
-  uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + kIBar);
+  uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + kIBar);   // K and Q landed
   uint64_t* bar_mma = bar_tma + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_tma + 2);
+  uint64_t* bar_v = bar_tma + 2;   // [2] V tile of a value head landed in buffer j % 2
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_tma + 4);
 
   if (tid == 0) {
     mbar_init(bar_tma, 1);
     mbar_init(bar_mma, 1);
+    mbar_init(&bar_v[0], 1);
+    mbar_init(&bar_v[1], 1);
     fence_mbar_init();
   }
   if (warp == 0) { tmem_alloc(tmem_slot, 256); tmem_relinquish(); }
@@ -247,18 +250,41 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tq = tmem_quadrant(tmem, warp);   // lanes 32 w .. 32 w + 31: rows of M = 128 results
-  uint32_t ph_tma = 0u, ph_mma = 0u;
+  uint32_t ph_mma = 0u;
 
+  // V tiles are double-buffered: buffer 0 at kIV, buffer 1 in the Q atoms (free once the
+  // [K; Q] K^T MMA has read them); head j + 2 loads while head j + 1 is computed
+  auto v_tile = [&](int b) { return sm + (b == 0 ? kIV : kIKQ + 8192); };
+  auto load_v = [&](int j) {   // value head hk * G + j into buffer j % 2
+    uint8_t* dst = v_tile(j & 1);
+    const uint32_t atom = (j & 1) ? 16384u : 8192u;
+    mbar_arrive_expect_tx(&bar_v[j & 1], 16384);
+    for (int hh = 0; hh < 2; ++hh)
+      tma_load_2d(dst + hh * atom, &map_v, (hk * G + j) * D + hh * 64, (int32_t)t0, &bar_v[j & 1]);
+  };
   if (tid == 0) {
-    mbar_arrive_expect_tx(bar_tma, 32768 + 16384);
+    mbar_arrive_expect_tx(bar_tma, 32768);
     for (int hh = 0; hh < 2; ++hh) {
       tma_load_2d(sm + kIKQ + hh * 16384, &map_k, hk * D + hh * 64, (int32_t)t0, bar_tma);
       tma_load_2d(sm + kIKQ + hh * 16384 + 8192, &map_q, hk * D + hh * 64, (int32_t)t0, bar_tma);
-      tma_load_2d(sm + kIV + hh * 8192, &map_v, (hk * G) * D + hh * 64, (int32_t)t0, bar_tma);
+    }
+    load_v(0);
+  }
+  if (warp < G) {   // inclusive cumulative log-decay of every value head, in place (2 values per lane)
+    for (int j = warp; j < G; j += 4) {
+      const float a0 = gAll[j * 64 + 2 * lane], a1 = gAll[j * 64 + 2 * lane + 1];
+      float s = a0 + a1;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, s, o);
+        if (lane >= o) s += y;
+      }
+      const float excl = s - (a0 + a1);
+      gAll[j * 64 + 2 * lane] = excl + a0;
+      gAll[j * 64 + 2 * lane + 1] = excl + a0 + a1;
     }
   }
-  bool ok = mbar_wait(bar_tma, ph_tma, err, kErrIntraTma);
-  ph_tma ^= 1u;
+  bool ok = mbar_wait(bar_tma, 0u, err, kErrIntraTma);
   if (__syncthreads_or(!ok)) goto teardown;
 
   {  // inverse L2 norms of the chunk's q and k rows (0 for rows past the sequence end)
@@ -293,28 +319,18 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
   ph_mma ^= 1u;
   if (__syncthreads_or(!ok)) goto teardown;
   tc_fence_after();
+  if (tid == 0 && G > 1) load_v(1);   // into the Q atoms, which the MMA has finished reading
 
   for (int j = 0; j < G; ++j) {
     const int h = hk * G + j;
-    if (warp == 0) {   // inclusive cumulative log-decay over the chunk (2 values per lane)
-      const float a0 = gAll[j * 64 + 2 * lane], a1 = gAll[j * 64 + 2 * lane + 1];
-      float s = a0 + a1;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const float y = __shfl_up_sync(0xffffffffu, s, o);
-        if (lane >= o) s += y;
-      }
-      const float excl = s - (a0 + a1);
-      sG[2 * lane] = excl + a0;
-      sG[2 * lane + 1] = excl + a0 + a1;
-    }
-    __syncthreads();
+    const float* sG = gAll + j * 64;   // cumulative log-decay of this head
     const float* sb = bAll + j * 64;
     if (tid < 64) {   // column factors of P = Tm diag(beta), Pk = Tm diag(beta e^G / |k|), A, Mqk
       colP[tid] = sb[tid];
       colPk[tid] = sb[tid] * __expf(sG[tid]) * rk[tid];
       colInv[tid] = -sG[C - 1] < 60.f ? __expf(-sG[tid]) * rk[tid] : 0.f;
     }
+    if (tid == 0) tma_store_wait_read();   // the previous head's staged tiles (A^T, Tm regions)
     __syncthreads();
 
     // thread t < 64: row t of A (stored transposed) from K K^T; t >= 64: row t-64 of Mqk.
@@ -454,22 +470,20 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
 
     const uint64_t dpp = smem_desc(smem_u32(sm + kIPP), 16u, 1024u);
     if (tid == 0) {   // [P; Pk] V: rows 0..63 = U~ (M = 128, N = 128, K = 64)
-      tc_fence_after();
-      const uint64_t dv = smem_desc(smem_u32(sm + kIV), 8192u, 1024u);
+      if (mbar_wait(&bar_v[j & 1], (uint32_t)(j >> 1) & 1u, err, kErrIntraTma)) {
+        tc_fence_after();
+        const uint64_t dv = smem_desc(smem_u32(v_tile(j & 1)), (j & 1) ? 16384u : 8192u, 1024u);
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + kTUW, dpp + 2 * kk, dv + 128 * kk, idesc_bf16(128, 128, 0, 1), kk > 0);
-      mma_commit(bar_mma);
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + kTUW, dpp + 2 * kk, dv + 128 * kk, idesc_bf16(128, 128, 0, 1), kk > 0);
+        mma_commit(bar_mma);
+      }
     }
     ok = mbar_wait(bar_mma, ph_mma, err, kErrIntraMma);
     ph_mma ^= 1u;
     if (__syncthreads_or(!ok)) goto teardown;
     tc_fence_after();
-    if (tid == 0 && j + 1 < G) {   // the V tile is free: next value head's V
-      mbar_arrive_expect_tx(bar_tma, 16384);
-      for (int hh = 0; hh < 2; ++hh)
-        tma_load_2d(sm + kIV + hh * 8192, &map_v, (h + 1) * D + hh * 64, (int32_t)t0, bar_tma);
-    }
+    if (tid == 0 && j + 2 < G) load_v(j + 2);   // this V buffer is free
     // U~ (rows 0..63 of the result) -> bf16 tile [64][128] in the free A^T region -> TMA store
     uint8_t* stage_u = sm + kIA;   // 2 swizzled atoms of [64][64]
     if (warp < 2) {
@@ -539,18 +553,12 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (tid == 0) {   // both staged tiles must be read out before the next head reuses them
+    if (tid == 0) {   // read out before the next head rewrites A^T / Tm (waited there)
       tma_store_2d(&map_wu, 0, wrow, stage_w);
       tma_store_2d(&map_wu, 64, wrow, stage_w + 8192);
       tma_store_commit();
-      tma_store_wait_read();
-    }
-    if (j + 1 < G) {
-      ok = mbar_wait(bar_tma, ph_tma, err, kErrIntraTma);
-      ph_tma ^= 1u;
     }
     tc_fence_before();
-    if (__syncthreads_or(!ok)) goto teardown;
   }
 
 teardown:
