@@ -374,42 +374,22 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     }
     __syncthreads();
 
-    // Tm = (I + A)^{-1}. Diagonal 16x16 blocks, one warp each: with L the block of A
-    // (strictly lower, L^16 = 0), (I + L)^{-1} = (I - L)(I + L^2)(I + L^4)(I + L^8), three
-    // squarings and three products on warp-level tf32 MMAs. X lives in the Tm block, the
-    // current power of L in the warp's scratch. Blocks above the diagonal are not stored.
-    {
-      const int b0 = warp * 16;
-      const int gq = lane >> 2, tq4 = lane & 3;
-      float* X = Tm + b0 * kLd + b0;
-      for (int e = lane; e < 256; e += 32) {
-        const int i = e >> 4, k = e & 15;
-        const float l = At[(b0 + k) * kLd + b0 + i];        // L(i, k)
-        X[i * kLd + k] = (i == k ? 1.f : 0.f) - l;
-        scratch[i * kLd16 + k] = l;
-      }
-      __syncwarp();
-      auto store_frag = [&](float* M, int pitch, const float (&c)[2][4], bool add) {
+    // Tm = (I + A)^{-1}. Diagonal 16x16 blocks, one warp each, by fp32 forward substitution:
+    // lane j < 16 solves column j of (I + L) X = I (L the block of A, strictly lower):
+    // x_i = delta_ij - sum_{k<i} L_ik x_k, accumulating each x_k into every later row as soon
+    // as it is known (a 15-step dependent chain; the L loads are warp broadcasts). Blocks
+    // above the diagonal are not stored.
+    if (lane < 16) {
+      const int b0 = warp * 16, j = lane;
+      float acc[16];
 #pragma unroll
-        for (int nh = 0; nh < 2; ++nh) {
-          float* r0 = M + gq * pitch + 8 * nh + 2 * tq4;
-          float* r8 = r0 + 8 * pitch;
-          if (add) { r0[0] += c[nh][0]; r0[1] += c[nh][1]; r8[0] += c[nh][2]; r8[1] += c[nh][3]; }
-          else { r0[0] = c[nh][0]; r0[1] = c[nh][1]; r8[0] = c[nh][2]; r8[1] = c[nh][3]; }
-        }
-      };
-#pragma unroll 1
-      for (int step = 0; step < 3; ++step) {
-        float p2[2][4] = {};   // P <- P P  (L^2, L^4, L^8)
-        block_mma16<false>(p2, scratch, kLd16, 0, 0, scratch, kLd16, 0, 0, lane);
-        __syncwarp();
-        store_frag(scratch, kLd16, p2, false);
-        __syncwarp();
-        float xp[2][4] = {};   // X <- X + X P
-        block_mma16<false>(xp, X, kLd, 0, 0, scratch, kLd16, 0, 0, lane);
-        __syncwarp();
-        store_frag(X, kLd, xp, true);
-        __syncwarp();
+      for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const float xk = k == j ? 1.f : (k < j ? 0.f : -acc[k]);
+        Tm[(b0 + k) * kLd + b0 + j] = xk;
+#pragma unroll
+        for (int i = k + 1; i < 16; ++i) acc[i] = fmaf(At[(b0 + k) * kLd + b0 + i], xk, acc[i]);   // L(i, k)
       }
     }
     __syncthreads();
@@ -766,8 +746,8 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
       tc_fence_after();
       float os = 0.f;
       if (quad < 2) {
-        // the previous chunk's O2 has finished reading U before it is overwritten
-        if (c > 0 && !(ok = mbar_wait(bar_O, (uint32_t)(c - 1) & 1u, err_word, kErrChainMma))) break;
+        // U is free: its last reader, O2 of chunk c - 1, was issued before rA_lo(c) by the
+        // same thread, and that thread's commit of rA_lo(c) tracks every MMA it issued before
         const int r = lrow;
         const float us = vec[64 + r];
         uint32_t a0[32], a1[32];
