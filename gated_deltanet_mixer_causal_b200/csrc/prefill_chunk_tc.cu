@@ -176,15 +176,32 @@ __device__ __forceinline__ void block_mma16(float (&c)[2][4], const float* Xs, i
   }
 }
 
+// The same for one 16x8 half (columns 8 nh .. 8 nh + 7) of the result.
+__device__ __forceinline__ void block_mma16h(float (&c)[4], const float* Xs, int px, int xr, int xc,
+                                             const float* Ys, int py, int yr, int yc, int nh, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int ks = 0; ks < 2; ++ks) {
+    const int k0 = 8 * ks + t;
+    const uint32_t a[4] = {to_tf32(Xs[(xr + g) * px + xc + k0]), to_tf32(Xs[(xr + g + 8) * px + xc + k0]),
+                           to_tf32(Xs[(xr + g) * px + xc + k0 + 4]), to_tf32(Xs[(xr + g + 8) * px + xc + k0 + 4])};
+    const uint32_t bb[2] = {to_tf32(Ys[(yr + k0) * py + yc + 8 * nh + g]),
+                            to_tf32(Ys[(yr + k0 + 4) * py + yc + 8 * nh + g])};
+    mma_tf32_16x8x8(c, a, bb);
+  }
+}
+
 // shared memory of the intra kernel (offsets from a 1024-aligned base)
 constexpr int kMaxG = kPrefillTcMaxG;           // value heads per key head on this path
 constexpr int kIKQ = 0;                         // [K0 | Q0 | K1 | Q1]: [K; Q] is one 128-row operand
 constexpr int kIV = 32768;                      // V tile of one value head: 2 atoms; once [K; Q] K^T
                                                 // is done the Q atoms hold a second V tile
 constexpr int kIPP = 49152;                     // [P | Pk] bf16, K-major
-constexpr int kLd = 72;                         // fp32 row pitch of A^T and Tm (= 8 mod 32:
-                                                // conflict-free tf32 fragment loads)
-constexpr int kIA = 65536;                      // A^T fp32 [64][kLd] (A^T[i][r] = A[r][i])
+constexpr int kLd = 72;                         // fp32 row pitch of Tm (= 8 mod 32: conflict-free
+                                                // tf32 B-fragment loads)
+constexpr int kLdA = 68;                        // fp32 row pitch of A (= 4 mod 32: conflict-free
+                                                // 16-byte row stores and tf32 A-fragment loads)
+constexpr int kIA = 65536;                      // A fp32 [64][kLdA] (region sized [64][kLd])
 constexpr int kIT = kIA + 64 * kLd * 4;         // Tm  fp32 [64][kLd]
 constexpr int kITmp = kIT + 64 * kLd * 4;       // per-warp block scratch fp32 [4][16][kLd16]
 constexpr int kLd16 = 24;
@@ -215,7 +232,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* At = reinterpret_cast<float*>(sm + kIA);
+  float* Am = reinterpret_cast<float*>(sm + kIA);
   float* Tm = reinterpret_cast<float*>(sm + kIT);
   float* scratch = reinterpret_cast<float*>(sm + kITmp) + warp * 16 * kLd16;
   float* rq = reinterpret_cast<float*>(sm + kIVec);
@@ -330,10 +347,10 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
       colPk[tid] = sb[tid] * __expf(sG[tid]) * rk[tid];
       colInv[tid] = -sG[C - 1] < 60.f ? __expf(-sG[tid]) * rk[tid] : 0.f;
     }
-    if (tid == 0) tma_store_wait_read();   // the previous head's staged tiles (A^T, Tm regions)
+    if (tid == 0) tma_store_wait_read();   // the previous head's staged tiles (A, Tm regions)
     __syncthreads();
 
-    // thread t < 64: row t of A (stored transposed) from K K^T; t >= 64: row t-64 of Mqk.
+    // thread t < 64: row t of A from K K^T; t >= 64: row t-64 of Mqk.
     // e^{G_r - G_i} = e^{G_r} e^{-G_i} with the column factors e^{-G_i}/|k_i| in shared
     // memory; when the chunk's cumulative decay could leave the fp32 range the difference
     // form is used instead (one exp per element).
@@ -353,7 +370,10 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
         float v[32], ci[32];
         if (factored) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) ci[e] = colInv[cb * 32 + e];
+          for (int e = 0; e < 32; e += 4) {
+            const float4 c4 = *reinterpret_cast<const float4*>(colInv + cb * 32 + e);
+            ci[e] = c4.x; ci[e + 1] = c4.y; ci[e + 2] = c4.z; ci[e + 3] = c4.w;
+          }
         } else {
 #pragma unroll
           for (int e = 0; e < 32; ++e) ci[e] = __expf(Gr - sG[cb * 32 + e]) * rk[cb * 32 + e];
@@ -366,7 +386,8 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
         }
         if (tid < 64) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) At[(cb * 32 + e) * kLd + r] = v[e];
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(Am + r * kLdA + cb * 32 + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
         } else {
           VecIO<bf16, 32>::store(reinterpret_cast<bf16*>(mq) + r * C + cb * 32, v);
         }
@@ -389,54 +410,86 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
         const float xk = k == j ? 1.f : (k < j ? 0.f : -acc[k]);
         Tm[(b0 + k) * kLd + b0 + j] = xk;
 #pragma unroll
-        for (int i = k + 1; i < 16; ++i) acc[i] = fmaf(At[(b0 + k) * kLd + b0 + i], xk, acc[i]);   // L(i, k)
+        for (int i = k + 1; i < 16; ++i) acc[i] = fmaf(Am[(b0 + i) * kLdA + b0 + k], xk, acc[i]);   // L(i, k)
       }
     }
     __syncthreads();
-    // off-diagonal blocks by block distance, one warp per block: Tm_ba = -Tm_bb sum_c A_bc Tm_ca
+    // off-diagonal blocks by block distance: Tm_ba = -Tm_bb sum_c A_bc Tm_ca. Distance 1:
+    // one warp per block; distances 2 and 3: two warps per block, one 8-column half each
+    // (a half of the result needs only the same half of the inner sum).
     for (int dist = 1; dist < 4; ++dist) {
-      if (warp < 4 - dist) {
-        const int aa = warp, bb = warp + dist;
-        float c[2][4] = {};
+      const int gq = lane >> 2, tq4 = lane & 3;
+      if (dist == 1) {
+        if (warp < 3) {
+          const int aa = warp, bb = warp + 1;
+          float c[2][4] = {};
+          block_mma16<false>(c, Am, kLdA, 16 * bb, 16 * aa, Tm, kLd, 16 * aa, 16 * aa, lane);
+#pragma unroll
+          for (int nh = 0; nh < 2; ++nh) {
+            scratch[gq * kLd16 + 8 * nh + 2 * tq4] = c[nh][0];
+            scratch[gq * kLd16 + 8 * nh + 2 * tq4 + 1] = c[nh][1];
+            scratch[(gq + 8) * kLd16 + 8 * nh + 2 * tq4] = c[nh][2];
+            scratch[(gq + 8) * kLd16 + 8 * nh + 2 * tq4 + 1] = c[nh][3];
+          }
+          __syncwarp();
+          float d[2][4] = {};
+          block_mma16<false>(d, Tm, kLd, 16 * bb, 16 * bb, scratch, kLd16, 0, 0, lane);
+#pragma unroll
+          for (int nh = 0; nh < 2; ++nh) {
+            float* row0 = Tm + (16 * bb + gq) * kLd + 16 * aa + 8 * nh + 2 * tq4;
+            float* row8 = row0 + 8 * kLd;
+            row0[0] = -d[nh][0]; row0[1] = -d[nh][1];
+            row8[0] = -d[nh][2]; row8[1] = -d[nh][3];
+          }
+        }
+      } else if (warp < 2 * (4 - dist)) {
+        const int aa = warp >> 1, bb = aa + dist, nh = warp & 1;
+        float c[4] = {};
         for (int cblk = aa; cblk < bb; ++cblk)
-          block_mma16<true>(c, At, kLd, 16 * bb, 16 * cblk, Tm, kLd, 16 * cblk, 16 * aa, lane);
-        const int gq = lane >> 2, tq4 = lane & 3;
-#pragma unroll
-        for (int nh = 0; nh < 2; ++nh) {
-          scratch[gq * kLd16 + 8 * nh + 2 * tq4] = c[nh][0];
-          scratch[gq * kLd16 + 8 * nh + 2 * tq4 + 1] = c[nh][1];
-          scratch[(gq + 8) * kLd16 + 8 * nh + 2 * tq4] = c[nh][2];
-          scratch[(gq + 8) * kLd16 + 8 * nh + 2 * tq4 + 1] = c[nh][3];
-        }
+          block_mma16h(c, Am, kLdA, 16 * bb, 16 * cblk, Tm, kLd, 16 * cblk, 16 * aa, nh, lane);
+        scratch[gq * kLd16 + 8 * nh + 2 * tq4] = c[0];
+        scratch[gq * kLd16 + 8 * nh + 2 * tq4 + 1] = c[1];
+        scratch[(gq + 8) * kLd16 + 8 * nh + 2 * tq4] = c[2];
+        scratch[(gq + 8) * kLd16 + 8 * nh + 2 * tq4 + 1] = c[3];
         __syncwarp();
-        float d[2][4] = {};
-        block_mma16<false>(d, Tm, kLd, 16 * bb, 16 * bb, scratch, kLd16, 0, 0, lane);
-#pragma unroll
-        for (int nh = 0; nh < 2; ++nh) {
-          float* row0 = Tm + (16 * bb + gq) * kLd + 16 * aa + 8 * nh + 2 * tq4;
-          float* row8 = row0 + 8 * kLd;
-          row0[0] = -d[nh][0]; row0[1] = -d[nh][1];
-          row8[0] = -d[nh][2]; row8[1] = -d[nh][3];
-        }
+        float d[4] = {};
+        block_mma16h(d, Tm, kLd, 16 * bb, 16 * bb, scratch, kLd16, 0, 0, nh, lane);
+        float* row0 = Tm + (16 * bb + gq) * kLd + 16 * aa + 8 * nh + 2 * tq4;
+        float* row8 = row0 + 8 * kLd;
+        row0[0] = -d[0]; row0[1] = -d[1];
+        row8[0] = -d[2]; row8[1] = -d[3];
       }
       __syncthreads();
     }
 
-    // [P | Pk] as bf16 K-major operands: thread = one column of one matrix; row scales out
+    // [P | Pk] as bf16 K-major operands: warps 0, 1 form P, warps 2, 3 Pk. A lane takes 4
+    // columns (chunk c) of a row per step, a warp 8 rows x 4 chunks: the 16-byte Tm loads
+    // (pitch 72 floats) and the 8-byte swizzled stores are free of bank conflicts. Row scales out.
     {
-      const int i = tid & 63, m = tid >> 6;
-      const float f = m == 0 ? colP[i] : colPk[i];
+      const int m = warp >> 1, wm = warp & 1, rl = lane >> 2, cl = lane & 3;
+      const float* fv = m == 0 ? colP : colPk;
+      float4 f[4];   // column factors of this lane's chunks cg * 4 + cl
+#pragma unroll
+      for (int cg = 0; cg < 4; ++cg) f[cg] = *reinterpret_cast<const float4*>(fv + 16 * cg + 4 * cl);
       uint8_t* tile = sm + kIPP + m * 8192;
-      // Tm is block lower triangular; its blocks above the diagonal are never written
-      // (the staging tiles reuse that memory), so they are masked here
-      for (int r0 = 0; r0 < 64; r0 += 16) {
-        float tv[16];
-        const bool live = r0 >= (i & ~15);
 #pragma unroll
-        for (int r = 0; r < 16; ++r) tv[r] = live ? Tm[(r0 + r) * kLd + i] : 0.f;
+      for (int rb = 0; rb < 4; ++rb) {
+        const int r = (wm * 4 + rb) * 8 + rl;
+        // Tm is block lower triangular; its blocks above the diagonal are never written
+        // (the staging tiles reuse that memory), so they are masked here
+        const int live_end = (r & ~15) + 16;
 #pragma unroll
-        for (int r = 0; r < 16; ++r)
-          *reinterpret_cast<bf16*>(tile + sw128_off(r0 + r, i)) = __float2bfloat16_rn(tv[r] * f);
+        for (int cg = 0; cg < 4; ++cg) {
+          const int c = cg * 4 + cl;
+          const float4 t = 4 * c < live_end ? *reinterpret_cast<const float4*>(Tm + r * kLd + 4 * c)
+                                            : make_float4(0.f, 0.f, 0.f, 0.f);
+          uint2 pk;
+          __nv_bfloat162 lo = __floats2bfloat162_rn(t.x * f[cg].x, t.y * f[cg].y);
+          __nv_bfloat162 hi = __floats2bfloat162_rn(t.z * f[cg].z, t.w * f[cg].w);
+          pk.x = *reinterpret_cast<uint32_t*>(&lo);
+          pk.y = *reinterpret_cast<uint32_t*>(&hi);
+          *reinterpret_cast<uint2*>(tile + sw128_off(r, 4 * c)) = pk;
+        }
       }
       float* vec = reinterpret_cast<float*>(ws + L.vecs) + (size_t)(slot * Hv + h) * kVecFloats;
       const float Gl = sG[C - 1];
@@ -464,7 +517,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     if (__syncthreads_or(!ok)) goto teardown;
     tc_fence_after();
     if (tid == 0 && j + 2 < G) load_v(j + 2);   // this V buffer is free
-    // U~ (rows 0..63 of the result) -> bf16 tile [64][128] in the free A^T region -> TMA store
+    // U~ (rows 0..63 of the result) -> bf16 tile [64][128] in the free A region -> TMA store
     uint8_t* stage_u = sm + kIA;   // 2 swizzled atoms of [64][64]
     if (warp < 2) {
 #pragma unroll
@@ -533,7 +586,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (tid == 0) {   // read out before the next head rewrites A^T / Tm (waited there)
+    if (tid == 0) {   // read out before the next head rewrites A / Tm (waited there)
       tma_store_2d(&map_wu, 0, wrow, stage_w);
       tma_store_2d(&map_wu, 64, wrow, stage_w + 8192);
       tma_store_commit();
