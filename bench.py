@@ -124,12 +124,14 @@ class ClockSampler:
 
 # ------------------------------------------------------------------- CPU oracle leg
 
-def cpu_oracle_prefill(p: W.PrefillInputs, target_s: float = 12.0, max_tokens: int = 4096):
+def cpu_oracle_prefill(p: W.PrefillInputs, target_s: float = 12.0, max_tokens: int = 4096,
+                       threads: int = 0):
     """Time the fp64 oracle on the first tokens of the same 64K sequence (all 48 heads,
-    conv included), sized to about ``target_s`` seconds. Returns (tok/s, threads, sample)."""
+    conv included), sized to about ``target_s`` seconds, on ``threads`` host threads (0: all
+    cores). Returns (tok/s, threads, sample)."""
     import oracle
     sh = p.shape
-    threads = oracle.default_threads()
+    threads = threads or oracle.default_threads()
 
     def run(n):
         x = p.x[:n].float().numpy(); w = p.conv_w.float().numpy()
@@ -145,6 +147,87 @@ def cpu_oracle_prefill(p: W.PrefillInputs, target_s: float = 12.0, max_tokens: i
     return n / dt, threads, f"first {n} tokens of the 65536-token 27B-shaped sequence, all 48 heads, conv included"
 
 
+# ------------------------------------------------------------ per-workload report
+
+def _median_ms(fn, stream, warmup=5, reps=20):
+    """Median device time of fn() over reps runs after warmup runs (CUDA events)."""
+    for _ in range(warmup):
+        fn()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+    ts = []
+    for i in range(reps):
+        ev[i].record(stream)
+        fn()
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    ts = [ev[i].elapsed_time(ev[i + 1]) for i in range(reps)]
+    return statistics.median(ts)
+
+
+def _roof(ms, flops, nbytes, tc_tflops, hbm_gbs):
+    t_tc = flops / (tc_tflops * 1e12) * 1e3 if flops else 0.0
+    t_hbm = nbytes / (hbm_gbs * 1e9) * 1e3
+    t_roof = max(t_tc, t_hbm)
+    return {"t_roof_ms": t_roof, "roofline_frac": t_roof / ms, "bound": "tensor" if t_tc > t_hbm else "hbm",
+            "tflops": flops / (ms / 1e3) / 1e12 if flops else None, "gbs": nbytes / (ms / 1e3) / 1e9}
+
+
+def measure_configs(gdn, dev, stream, hbm_gbs, tc_sust):
+    """Every benchmark workload, timed as CUDA-event medians of 20 runs after 5 warm-ups:
+    the layer (conv + prefill) for the prefill workloads, the 100-step block for decode.
+    Roofline fraction = t_roof / t_measured with t_roof = max(flops / sustained bf16 peak,
+    bytes / HBM copy peak); flops in the chunked-form count, bytes = pre-conv x in, o out,
+    g and beta in (plus initial and final states where given)."""
+    out = []
+
+    def layer(p: W.PrefillInputs, name: str, note: str = ""):
+        sh = p.shape
+        x = p.x.to(dev); w = p.conv_w.to(dev); g = p.g.to(dev); b = p.beta.to(dev)
+        cu = p.cu_seqlens.to(dev) if p.cu_seqlens is not None else None
+        s0 = p.initial_state.to(dev) if p.initial_state is not None else None
+        n = p.n_seq
+        fin = torch.empty((n, sh.Hv, sh.dv, sh.dk), dtype=torch.float32, device=dev)
+        y = torch.empty_like(x)
+        o = torch.empty((p.T, sh.Hv, sh.dv), dtype=x.dtype, device=dev)
+        ws_n = gdn.gdn_chunk_prefill_workspace_size(p.T, n, sh.Hk, sh.Hv, sh.dk, sh.dv, x.dtype)
+        ws = torch.empty(max(ws_n, 1), dtype=torch.uint8, device=dev)
+        fn = lambda: gdn.prefill_layer(x, w, g, b, sh.Hk, sh.Hv, sh.dk, cu_seqlens=cu, initial_state=s0,
+                                       final_state=fin, y=y, o=o, workspace=ws)
+        ms = _median_ms(fn, stream)
+        T = p.T
+        rec = {"workload": name, "tokens": T, "sequences": n, "ms": ms, "tokens_per_s": T / (ms / 1e3),
+               "dtype": "f32" if x.dtype == torch.float32 else "bf16"}
+        if x.dtype == torch.bfloat16:
+            nbytes = prefill_bytes_per_token(sh) * T + (2 if s0 is not None else 1) * fin.numel() * 4
+            rec.update(_roof(ms, prefill_flops_per_token(sh) * T, nbytes, tc_sust, hbm_gbs))
+        if note:
+            rec["note"] = note
+        out.append(rec)
+        del x, w, g, b, y, o, ws, fin
+
+    layer(W.tiny_layer(), "tiny fp32 layer: T=64, Hk=Hv=2, d=16",
+          "correctness gate; fp32 token-recurrent path; time only")
+    layer(W.qwen35_9b_prefill(8192), "Qwen3.5-9B-shaped layer prefill: T=8192, Hk 16, Hv 32, d 128")
+    layer(W.qwen35_27b_prefill(65536), "Qwen3.5-27B-shaped layer prefill: T=65536, Hk 16, Hv 48, d 128")
+    layer(W.qwen35_27b_varlen(32), "Qwen3.5-27B-shaped varlen prefill: 32 sequences (log-uniform 512..32768), nonzero initial states")
+
+    dcd = W.qwen35_27b_decode(256, 100)
+    sh = dcd.shape
+    xs = [t.to(dev) for t in dcd.xs]; gs = [t.to(dev) for t in dcd.gs]; bs = [t.to(dev) for t in dcd.betas]
+    cs = dcd.conv_state.to(dev); st = dcd.state.to(dev); cw = dcd.conv_w.to(dev)
+    do = torch.empty((256, sh.Hv, sh.dv), dtype=xs[0].dtype, device=dev)
+
+    def block():
+        for t in range(100):
+            gdn.gdn_decode_step(xs[t], cw, cs, gs[t], bs[t], st, sh.Hk, do)
+    ms = _median_ms(block, stream, warmup=2, reps=20) / 100
+    rec = {"workload": "Qwen3.5-27B-shaped decode: B=256 x 1 token, 100-step block (per step)",
+           "tokens": 256, "sequences": 256, "ms": ms, "tokens_per_s": 256 / (ms / 1e3), "dtype": "bf16"}
+    rec.update(_roof(ms, 0, decode_bytes(256, sh), tc_sust, hbm_gbs))
+    out.append(rec)
+    return out
+
+
 # --------------------------------------------------------------------------- main
 
 def parse():
@@ -157,6 +240,8 @@ def parse():
     ap.add_argument("--decode-batch", type=int, default=B_DECODE)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-workload report (run after the timed region, N = 1 only)")
     return ap.parse_args()
 
 
@@ -345,7 +430,15 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v_cpu, threads, sample = cpu_oracle_prefill(p)
-        cpu = {"value": v_cpu, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample}
+        v_one, _, sample_one = cpu_oracle_prefill(p, target_s=4.0, max_tokens=1024, threads=1)
+        cpu = {"value": v_cpu, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample,
+               "value_1_thread": v_one, "sample_1_thread": sample_one}
+
+    configs = None
+    if rank == 0 and world == 1 and not args.no_configs:
+        del x, y, o, ws, dst, dx, dg, db, dcs, do
+        torch.cuda.empty_cache()
+        configs = measure_configs(gdn, dev, stream, hbm_gbs, tc_sust)
 
     if rank == 0:
         line = {
@@ -370,6 +463,7 @@ def main():
             "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,
+            "configs": configs,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
