@@ -246,15 +246,20 @@ def parse():
 
 
 def dist_setup(n_gpus):
+    """One process per GPU (torchrun's RANK / WORLD_SIZE / LOCAL_RANK); NCCL on GPUs, gloo
+    where there is no GPU (the CPU-only reference arm and the multi-process tests)."""
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        timeout = datetime.timedelta(seconds=120)
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=timeout)
     return rank, world, local
 
 
