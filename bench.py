@@ -62,6 +62,14 @@ def decode_bytes(B, sh=SHAPE):
             + 2 * B * sh.Hv * 4 + Cc * 4 * 2)
 
 
+def decode_tokens_bytes(B, n_tok, sh=SHAPE):
+    """A multi-token call: each state read and written once, n_tok tokens of x, g, beta, o."""
+    Cc = sh.conv_channels
+    state = B * sh.Hv * sh.dv * sh.dk * 4
+    return (2 * state + n_tok * B * Cc * 2 + 2 * B * 3 * Cc * 2 + n_tok * B * sh.Hv * sh.dv * 2
+            + n_tok * 2 * B * sh.Hv * 4 + Cc * 4 * 2)
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -224,6 +232,23 @@ def measure_configs(gdn, dev, stream, hbm_gbs, tc_sust):
     rec = {"workload": "Qwen3.5-27B-shaped decode: B=256 x 1 token, 100-step block (per step)",
            "tokens": 256, "sequences": 256, "ms": ms, "tokens_per_s": 256 / (ms / 1e3), "dtype": "bf16"}
     rec.update(_roof(ms, 0, decode_bytes(256, sh), tc_sust, hbm_gbs))
+    out.append(rec)
+
+    # multi-token decode / verify: 4 tokens per sequence per call (25 calls = 100 tokens)
+    n_tok = 4
+    xt = [torch.stack(xs[i:i + n_tok], 1) for i in range(0, 100, n_tok)]
+    gt = [torch.stack(gs[i:i + n_tok], 1) for i in range(0, 100, n_tok)]
+    bt = [torch.stack(bs[i:i + n_tok], 1) for i in range(0, 100, n_tok)]
+    ot = torch.empty((256, n_tok, sh.Hv, sh.dv), dtype=xs[0].dtype, device=dev)
+
+    def block4():
+        for i in range(len(xt)):
+            gdn.gdn_decode_tokens(xt[i], cw, cs, gt[i], bt[i], st, sh.Hk, ot)
+    ms = _median_ms(block4, stream, warmup=2, reps=20) / len(xt)
+    rec = {"workload": "Qwen3.5-27B-shaped multi-token decode: B=256 x 4 tokens per call (per call)",
+           "tokens": 256 * n_tok, "sequences": 256, "ms": ms, "tokens_per_s": 256 * n_tok / (ms / 1e3),
+           "dtype": "bf16"}
+    rec.update(_roof(ms, 0, decode_tokens_bytes(256, n_tok, sh), tc_sust, hbm_gbs))
     out.append(rec)
     return out
 

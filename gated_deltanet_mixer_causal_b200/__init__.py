@@ -5,7 +5,8 @@ package marshals torch tensors into it. The library is loaded on first use and a
 library raises -- there is no fallback.
 
 Entry points (same names as the C ABI): ``gdn_conv1d_silu``, ``gdn_chunk_prefill``,
-``gdn_chunk_prefill_workspace_size``, ``gdn_decode_step``; ``prefill_layer`` chains the
+``gdn_chunk_prefill_workspace_size``, ``gdn_chunk_prefill_noalloc``, ``gdn_decode_step``,
+``gdn_decode_tokens``; ``prefill_layer`` chains the
 conv and the chunked prefill over one packed batch without copies.
 """
 from __future__ import annotations
@@ -15,10 +16,12 @@ from typing import Optional
 import torch
 
 from ._lib import (GDNError, LIB_PATH, gdn_chunk_prefill, gdn_chunk_prefill_noalloc,
-                   gdn_chunk_prefill_workspace_size, gdn_conv1d_silu, gdn_decode_step, lib)
+                   gdn_chunk_prefill_workspace_size, gdn_conv1d_silu, gdn_decode_step,
+                   gdn_decode_tokens, lib)
 
 __all__ = ["GDNError", "LIB_PATH", "lib", "gdn_conv1d_silu", "gdn_chunk_prefill",
            "gdn_chunk_prefill_workspace_size", "gdn_chunk_prefill_noalloc", "gdn_decode_step",
+           "gdn_decode_tokens",
            "prefill_layer", "qkv_views"]
 
 

@@ -33,6 +33,8 @@ SIGNATURES = {
                                           _P, _SZ, _P]),
     "gdn_decode_step": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _I32, _I32,
                                         _I32, _I32, _I32, _F32, _P]),
+    "gdn_decode_tokens": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _I32, _I32, _I32,
+                                         _I32, _I32, _I32, _F32, _P]),
     "gdn_chunk_prefill_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int, _I64, _I32,
                                                   _I32, _I32, _I32, _I64, _I64, _P, _I32, _P, _P,
                                                   _F32, _I32, _P]),
@@ -232,4 +234,29 @@ def gdn_decode_step(x: torch.Tensor, conv_w: torch.Tensor, conv_state: torch.Ten
     _check(lib().gdn_decode_step(_ptr(x), _ptr(conv_w), _ptr(conv_state), _ptr(g), _ptr(beta),
                                  _ptr(state), _ptr(o), _dtype_code(x), B, Hk, Hv, dk, dv,
                                  float(scale), _stream(dev)), "gdn_decode_step")
+    return o
+
+
+def gdn_decode_tokens(x: torch.Tensor, conv_w: torch.Tensor, conv_state: torch.Tensor,
+                      g: torch.Tensor, beta: torch.Tensor, state: torch.Tensor, Hk: int,
+                      o: Optional[torch.Tensor] = None, scale: float = 1.0) -> torch.Tensor:
+    """n_tok (1..8) consecutive tokens per sequence, x [B, n_tok, Cc]; conv_state and state
+    are updated in place. Returns o [B, n_tok, Hv, dv]."""
+    B, n_tok, Cc = x.shape
+    _, Hv, dv, dk = state.shape
+    dev = x.device
+    if Cc != 2 * Hk * dk + Hv * dv:
+        raise ValueError(f"x has {Cc} channels, expected 2*Hk*dk + Hv*dv = {2 * Hk * dk + Hv * dv}")
+    _need(x, "x", device=dev)
+    _need(conv_w, "conv_w", (Cc, 4), x.dtype, dev)
+    _need(conv_state, "conv_state", (B, 3, Cc), x.dtype, dev)
+    _need(g, "g", (B, n_tok, Hv), torch.float32, dev)
+    _need(beta, "beta", (B, n_tok, Hv), torch.float32, dev)
+    _need(state, "state", (B, Hv, dv, dk), torch.float32, dev)
+    if o is None:
+        o = torch.empty((B, n_tok, Hv, dv), dtype=x.dtype, device=dev)
+    _need(o, "o", (B, n_tok, Hv, dv), x.dtype, dev)
+    _check(lib().gdn_decode_tokens(_ptr(x), _ptr(conv_w), _ptr(conv_state), _ptr(g), _ptr(beta),
+                                   _ptr(state), _ptr(o), _dtype_code(x), B, n_tok, Hk, Hv, dk, dv,
+                                   float(scale), _stream(dev)), "gdn_decode_tokens")
     return o

@@ -204,4 +204,45 @@ gdn_status_t gdn_decode_step(const void* x, const void* conv_w, void* conv_state
                      "decode_step launch");
 }
 
+gdn_status_t gdn_decode_tokens(const void* x, const void* conv_w, void* conv_state, const float* g,
+                               const float* beta, float* state, void* o, gdn_dtype_t dt, int32_t B,
+                               int32_t n_tok, int32_t Hk, int32_t Hv, int32_t dk, int32_t dv,
+                               float scale, gdn_stream_t stream) {
+  if (!valid_dtype(dt)) return fail(GDN_ERR_UNSUPPORTED, "decode_tokens: unknown dtype %d", (int)dt);
+  if (B < 0) return fail(GDN_ERR_INVALID_ARG, "decode_tokens: B = %d < 0", B);
+  if (n_tok < 1 || n_tok > 8) return fail(GDN_ERR_INVALID_ARG, "decode_tokens: n_tok = %d outside [1, 8]", n_tok);
+  if (Hk <= 0 || Hv <= 0) return fail(GDN_ERR_INVALID_ARG, "decode_tokens: Hk, Hv must be > 0");
+  if (Hv % Hk != 0) return fail(GDN_ERR_UNSUPPORTED, "decode_tokens: Hv %% Hk != 0 (%d, %d)", Hv, Hk);
+  if (dk != dv || !supported_head_dim(dk))
+    return fail(GDN_ERR_UNSUPPORTED, "decode_tokens: head dims dk=%d dv=%d (need dk = dv in {16,32,64,128})", dk, dv);
+  const int64_t G = Hv / Hk;
+  if ((int64_t)n_tok * ((2 + G) * dk + G * dk) * 4 > 227 * 1024)
+    return fail(GDN_ERR_UNSUPPORTED, "decode_tokens: %d tokens of %lld value heads per key head exceed shared memory",
+                n_tok, (long long)G);
+  if ((int64_t)B * Hk > 0x7fffffffLL) return fail(GDN_ERR_INVALID_ARG, "decode_tokens: B * Hk too large");
+  if (B == 0) return ok();
+  if (!x || !conv_w || !conv_state || !g || !beta || !state || !o)
+    return fail(GDN_ERR_INVALID_ARG, "decode_tokens: all pointers must be non-null");
+  if (!aligned16(x) || !aligned16(conv_w) || !aligned16(conv_state) || !aligned16(g) ||
+      !aligned16(beta) || !aligned16(state) || !aligned16(o))
+    return fail(GDN_ERR_INVALID_ARG, "decode_tokens: pointers must be 16-byte aligned");
+  const size_t es = elt_size(dt);
+  const int64_t Cc = 2LL * Hk * dk + (int64_t)Hv * dv;
+  const size_t xb = (size_t)B * n_tok * Cc * es, csb = (size_t)B * 3 * Cc * es;
+  const size_t stb = (size_t)B * Hv * dv * dk * 4, ob = (size_t)B * n_tok * Hv * dv * es;
+  const size_t gb = (size_t)B * n_tok * Hv * 4, wb = (size_t)Cc * 4 * es;
+  const void* ro[4] = {x, conv_w, g, beta};
+  const size_t rob[4] = {xb, wb, gb, gb};
+  for (int i = 0; i < 4; ++i)
+    if (overlap(ro[i], rob[i], conv_state, csb) || overlap(ro[i], rob[i], state, stb) ||
+        overlap(ro[i], rob[i], o, ob))
+      return fail(GDN_ERR_INVALID_ARG, "decode_tokens: an output overlaps an input");
+  if (overlap(conv_state, csb, state, stb) || overlap(conv_state, csb, o, ob) ||
+      overlap(state, stb, o, ob))
+    return fail(GDN_ERR_INVALID_ARG, "decode_tokens: conv_state, state and o must not overlap");
+  return cuda_status(gdn::launch_decode_tokens((int)dt, x, conv_w, conv_state, g, beta, state, o, B,
+                                               n_tok, Hk, Hv, dk, scale, (cudaStream_t)stream),
+                     "decode_tokens launch");
+}
+
 }  // extern "C"

@@ -20,6 +20,11 @@ cudaError_t launch_decode_step(int dtype, const void* x, const void* conv_w, voi
                                const float* g, const float* beta, float* state, void* o,
                                int32_t B, int32_t Hk, int32_t Hv, int32_t d, float scale,
                                cudaStream_t stream);
+// n_tok (1..8) tokens per sequence; x [B, n_tok, Cc], g/beta [B, n_tok, Hv], o [B, n_tok, Hv, d]
+cudaError_t launch_decode_tokens(int dtype, const void* x, const void* conv_w, void* conv_state,
+                                 const float* g, const float* beta, float* state, void* o,
+                                 int32_t B, int32_t n_tok, int32_t Hk, int32_t Hv, int32_t d,
+                                 float scale, cudaStream_t stream);
 
 // Token-by-token fp32 recurrence (SIMT): the fp32-activation prefill path.
 cudaError_t launch_prefill_recurrent(int dtype, const void* q, const void* k, const void* v,

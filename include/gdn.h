@@ -196,6 +196,33 @@ gdn_status_t gdn_decode_step(const void* x, const void* conv_w, void* conv_state
                              gdn_dtype_t dt, int32_t B, int32_t Hk, int32_t Hv,
                              int32_t dk, int32_t dv, float scale, gdn_stream_t stream);
 
+/*
+ * gdn_decode_tokens -- n_tok consecutive tokens (1 <= n_tok <= 8) for each of B sequences,
+ * conv taps and states updated in place: a multi-token decode or speculative verify step.
+ *
+ * Defined as n_tok applications of gdn_decode_step's update (Qwen3.5 page, section 5 and the
+ * conv of the config footnote), token t of every sequence before token t + 1: the result
+ * equals n_tok calls of gdn_decode_step, and a prefill of B sequences of n_tok tokens from
+ * the same states. Each state is read and written once per call (Qwen3.5 page, section 8:
+ * decode is bound by moving the fixed-size state).
+ *
+ * x           [B, n_tok, Cc] dtype dt, the tokens' pre-conv q|k|v in order.
+ * conv_w      [Cc, 4] dtype dt.
+ * conv_state  [B, 3, Cc] dtype dt, read and updated in place (advances by n_tok taps).
+ * g, beta     [B, n_tok, Hv] fp32.
+ * state       [B, Hv, dv, dk] fp32, read and updated in place.
+ * o           [B, n_tok, Hv, dv] dtype dt.
+ * All tokens are committed: a caller that rejects speculative tokens keeps a copy of the
+ * states from before the call. Returns GDN_OK, GDN_ERR_INVALID_ARG (n_tok outside [1, 8],
+ * null, misaligned or overlapping buffers), GDN_ERR_UNSUPPORTED (as gdn_decode_step, or a
+ * head group whose n_tok tokens exceed one CTA's shared memory), GDN_ERR_CUDA. B = 0 is a
+ * no-op.
+ */
+gdn_status_t gdn_decode_tokens(const void* x, const void* conv_w, void* conv_state,
+                               const float* g, const float* beta, float* state, void* o,
+                               gdn_dtype_t dt, int32_t B, int32_t n_tok, int32_t Hk, int32_t Hv,
+                               int32_t dk, int32_t dv, float scale, gdn_stream_t stream);
+
 #ifdef __cplusplus
 }  /* extern "C" */
 #endif

@@ -168,6 +168,23 @@ def decode_step(x, conv_w, conv_state, g, beta, state, Hk, Hv, dk, dv, scale=1.0
                          n_threads)
 
 
+def decode_tokens(x, conv_w, conv_state, g, beta, state, Hk, Hv, dk, dv, scale=1.0,
+                  n_threads=None):
+    """n consecutive tokens for each of B sequences: the prefill of B sequences of n tokens
+    that start from the carried conv taps and recurrent states.
+
+    x [B, n, Cc]; conv_state [B, 3, Cc]; g, beta [B, n, Hv]; state [B, Hv, dv, dk].
+    Returns (o [B, n, Hv, dv], new_state, new_conv_state); inputs are not modified.
+    """
+    x = np.asarray(x)
+    B, n, Cc = x.shape
+    cu = np.arange(0, (B + 1) * n, n, dtype=np.int32)
+    o, S, cs = layer_prefill(x.reshape(B * n, Cc), conv_w, np.asarray(g).reshape(B * n, Hv),
+                             np.asarray(beta).reshape(B * n, Hv), Hk, Hv, dk, dv, cu, state,
+                             conv_state, scale, n_threads)
+    return o.reshape(B, n, Hv, dv), S, cs
+
+
 def layer_state_bytes(Hv, dk, dv, state_bytes, conv_channels, conv_taps, conv_bytes) -> int:
     """Per-layer constant footprint of one sequence: Hv dv x dk matrices plus the conv
     buffer (channels x taps elements)."""

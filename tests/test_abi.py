@@ -127,6 +127,30 @@ def test_decode_validation(L):
     assert _decode(L, cs=FAKE + 16) == _lib.GDN_ERR_INVALID_ARG               # conv_state over x
 
 
+def _decode_tokens(L, **kw):
+    a = dict(x=FAKE, w=FAKE + (1 << 30), cs=FAKE + (2 << 30), g=FAKE + (3 << 30),
+             b=FAKE + (4 << 30), st=FAKE + (5 << 30), o=FAKE + (6 << 30), dt=1, B=8, n=4, Hk=2,
+             Hv=4, dk=32, dv=32)
+    a.update(kw)
+    return L.gdn_decode_tokens(a["x"], a["w"], a["cs"], a["g"], a["b"], a["st"], a["o"], a["dt"],
+                               a["B"], a["n"], a["Hk"], a["Hv"], a["dk"], a["dv"], 1.0, None)
+
+
+def test_decode_tokens_validation(L):
+    assert _decode_tokens(L, n=0) == _lib.GDN_ERR_INVALID_ARG
+    assert _decode_tokens(L, n=9) == _lib.GDN_ERR_INVALID_ARG
+    assert _decode_tokens(L, B=-1) == _lib.GDN_ERR_INVALID_ARG
+    assert _decode_tokens(L, B=0) == _lib.GDN_OK                       # no-op, nothing launched
+    assert _decode_tokens(L, dk=24, dv=24) == _lib.GDN_ERR_UNSUPPORTED
+    assert _decode_tokens(L, Hv=5) == _lib.GDN_ERR_UNSUPPORTED
+    # 8 tokens of 32 value heads of 128 per key head need more than one CTA's shared memory
+    assert _decode_tokens(L, n=8, Hk=1, Hv=32, dk=128, dv=128) == _lib.GDN_ERR_UNSUPPORTED
+    assert _decode_tokens(L, st=None) == _lib.GDN_ERR_INVALID_ARG
+    # x holds B * n tokens: a conv_state placed inside it overlaps
+    assert _decode_tokens(L, cs=FAKE + 8 * 3 * 256 * 2) == _lib.GDN_ERR_INVALID_ARG
+    assert _decode_tokens(L, o=FAKE + (5 << 30) + 128) == _lib.GDN_ERR_INVALID_ARG   # o inside state
+
+
 def test_python_binding_refuses_cpu_tensors():
     import torch
     x = torch.zeros(8, 64, dtype=torch.bfloat16)

@@ -287,3 +287,68 @@ def test_decode_matches_prefill_on_gpu(cuda_device):
     o_d = torch.stack(outs, 1).reshape(16, sh.Hv, sh.dv)
     assert worst_head_o(np64(o_d), np64(o_p), [0, 8, 16]) <= BF16_TOL
     assert worst_head_state(np64(st), np64(fin)) <= BF16_TOL
+
+
+# ------------------------------------------------------------ multi-token decode
+
+@pytest.mark.parametrize("n_tok", [1, 2, 3, 5, 8])
+def test_decode_tokens_fp32_small(cuda_device, n_tok):
+    """n_tok tokens per sequence in one call against the oracle (fp32, element by element);
+    n_tok < 3 keeps old taps in the new conv state, n_tok >= 3 replaces them all."""
+    sh = W.LayerShape(2, 4, 32, 32)
+    d = W.make_decode(sh, B=3, steps=n_tok, seed=43 + n_tok, dtype=torch.float32)
+    x = torch.stack(d.xs, 1); g = torch.stack(d.gs, 1); b = torch.stack(d.betas, 1)
+    cs = d.conv_state.to(cuda_device).clone()
+    st = d.state.to(cuda_device).clone()
+    o = gdn.gdn_decode_tokens(x.to(cuda_device), d.conv_w.to(cuda_device), cs, g.to(cuda_device),
+                              b.to(cuda_device), st, sh.Hk)
+    torch.cuda.synchronize()
+    o_r, st_r, cs_r = oracle.decode_tokens(x.numpy(), d.conv_w.numpy(), d.conv_state.numpy(),
+                                           g.numpy(), b.numpy(), d.state.numpy(), sh.Hk, sh.Hv,
+                                           sh.dk, sh.dv)
+    assert o.shape == (3, n_tok, sh.Hv, sh.dv)
+    assert max_rel(np64(o), o_r) <= FP32_TOL
+    assert max_rel(np64(st), st_r) <= FP32_TOL
+    np.testing.assert_array_equal(np64(cs), cs_r)
+
+
+@pytest.mark.parametrize("n_tok", [4, 8])
+def test_decode_tokens_27b_bf16(cuda_device, n_tok):
+    """27B-shaped heads, 16 sequences, n_tok tokens each in one call, every head against the
+    oracle (bf16 tolerance); the conv taps are copies and must match exactly."""
+    d = W.make_decode(W.QWEN35_27B, B=16, steps=n_tok, seed=44)
+    sh = d.shape
+    x = torch.stack(d.xs, 1); g = torch.stack(d.gs, 1); b = torch.stack(d.betas, 1)
+    cs = d.conv_state.to(cuda_device).clone()
+    st = d.state.to(cuda_device).clone()
+    o = gdn.gdn_decode_tokens(x.to(cuda_device), d.conv_w.to(cuda_device), cs, g.to(cuda_device),
+                              b.to(cuda_device), st, sh.Hk)
+    torch.cuda.synchronize()
+    o_r, st_r, cs_r = oracle.decode_tokens(x.float().numpy(), d.conv_w.float().numpy(),
+                                           d.conv_state.float().numpy(), g.numpy(), b.numpy(),
+                                           d.state.numpy(), sh.Hk, sh.Hv, sh.dk, sh.dv)
+    o_g, st_g = np64(o), np64(st)
+    for j in range(16):
+        for h in range(sh.Hv):
+            assert frob_rel(o_g[j, :, h], o_r[j, :, h]) <= BF16_TOL, (j, h)
+            assert frob_rel(st_g[j, h], st_r[j, h]) <= BF16_TOL, (j, h)
+    np.testing.assert_array_equal(np64(cs), cs_r)
+
+
+def test_decode_tokens_equals_single_steps_on_gpu(cuda_device):
+    """Four tokens in one call agree with four gdn_decode_step calls (both on the GPU, the
+    same per-row arithmetic)."""
+    d = W.make_decode(W.QWEN35_27B, B=8, steps=4, seed=45)
+    sh = d.shape
+    w = d.conv_w.to(cuda_device)
+    cs1 = d.conv_state.to(cuda_device).clone(); st1 = d.state.to(cuda_device).clone()
+    outs = [gdn.gdn_decode_step(d.xs[t].to(cuda_device), w, cs1, d.gs[t].to(cuda_device),
+                                d.betas[t].to(cuda_device), st1, sh.Hk) for t in range(4)]
+    cs4 = d.conv_state.to(cuda_device).clone(); st4 = d.state.to(cuda_device).clone()
+    o4 = gdn.gdn_decode_tokens(torch.stack(d.xs, 1).to(cuda_device), w, cs4,
+                               torch.stack(d.gs, 1).to(cuda_device),
+                               torch.stack(d.betas, 1).to(cuda_device), st4, sh.Hk)
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(np64(o4), np64(torch.stack(outs, 1)), rtol=1e-2, atol=1e-3)
+    assert max_rel(np64(st4), np64(st1)) <= 1e-5
+    assert torch.equal(cs4, cs1)

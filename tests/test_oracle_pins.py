@@ -306,6 +306,27 @@ def test_decode_steps_equal_prefill(oracle_mod):
     np.testing.assert_array_equal(cs_d, xs[-3:].transpose(1, 0, 2))
 
 
+def test_decode_tokens_equal_single_steps(oracle_mod):
+    """A multi-token decode call equals its tokens taken one decode step at a time, with
+    o[b, t] the output of sequence b's t-th token."""
+    r = rng(18)
+    B, n, Hk, Hv, d = 3, 5, 1, 2, 4
+    Cc = 2 * Hk * d + Hv * d
+    w = r.standard_normal((Cc, 4))
+    S = r.standard_normal((B, Hv, d, d)) * 0.1
+    cs = r.standard_normal((B, 3, Cc))
+    xs = r.standard_normal((B, n, Cc)); gs = r.uniform(-0.3, 0, (B, n, Hv))
+    bs = expit(r.standard_normal((B, n, Hv)))
+    o_m, S_m, cs_m = oracle.decode_tokens(xs, w, cs, gs, bs, S, Hk, Hv, d, d)
+    S_d, cs_d = S.copy(), cs.copy()
+    for t in range(n):
+        o, S_d, cs_d = oracle.decode_step(xs[:, t], w, cs_d, gs[:, t], bs[:, t], S_d, Hk, Hv, d, d)
+        np.testing.assert_allclose(o_m[:, t], o, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(S_m, S_d, rtol=1e-13, atol=1e-14)
+    np.testing.assert_array_equal(cs_m, cs_d)
+    np.testing.assert_array_equal(cs_m, xs[:, -3:])
+
+
 def test_empty_sequence_passes_state_through(oracle_mod):
     r = rng(17)
     q, k, v, g, beta, S0 = _random_case(r, 4, 1, 1, 3)
