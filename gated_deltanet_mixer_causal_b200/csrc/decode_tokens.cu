@@ -11,7 +11,7 @@
 //  1. conv + SiLU of the call's tokens over this key head's channels: the three carried taps
 //     and the n_tok new inputs form one window; the taps advance by n_tok, in place;
 //  2. q_t, k_t L2-normalised per token in shared memory, read per token by the row loop;
-//  3. each warp streams whole state rows: per token t, with s the current row,
+//  3. the warps stream the state rows (D / 16 lanes per row): per token t, with s the row,
 //       sk = s.k_t, sq = s.q_t;  u = beta_t (v_t,i - alpha_t sk);  s <- alpha_t s + u k_t
 //       o_t,i = scale (alpha_t sq + u (k_t.q_t))
 #include "common.cuh"
@@ -22,33 +22,8 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kRowUnroll = 4;      // rows per warp iteration, all of one value head
 constexpr int kMaxTok = 8;
 constexpr float kEps = 1e-6f;
-
-template <int VEC> struct Row;
-template <> struct Row<4> {
-  static __device__ __forceinline__ void load(const float* p, float (&s)[4]) {
-    const float4 v = __ldcs(reinterpret_cast<const float4*>(p));
-    s[0] = v.x; s[1] = v.y; s[2] = v.z; s[3] = v.w;
-  }
-  static __device__ __forceinline__ void store(float* p, const float (&s)[4]) {
-    __stcs(reinterpret_cast<float4*>(p), make_float4(s[0], s[1], s[2], s[3]));
-  }
-};
-template <> struct Row<2> {
-  static __device__ __forceinline__ void load(const float* p, float (&s)[2]) {
-    const float2 v = __ldcs(reinterpret_cast<const float2*>(p));
-    s[0] = v.x; s[1] = v.y;
-  }
-  static __device__ __forceinline__ void store(float* p, const float (&s)[2]) {
-    __stcs(reinterpret_cast<float2*>(p), make_float2(s[0], s[1]));
-  }
-};
-template <> struct Row<1> {
-  static __device__ __forceinline__ void load(const float* p, float (&s)[1]) { s[0] = __ldcs(p); }
-  static __device__ __forceinline__ void store(float* p, const float (&s)[1]) { __stcs(p, s[0]); }
-};
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads, 3)
@@ -146,61 +121,60 @@ decode_tokens_kernel(const T* __restrict__ x, const T* __restrict__ conv_w, T* _
   }
   __syncthreads();
 
-  // 3. stream the G * D state rows of this CTA, each through every token.
+  // 3. stream the G * D state rows of this CTA, each through every token. A row is split
+  //    over L = D / 16 lanes of 16 columns each, so its dot products need log2(L) shuffle
+  //    rounds; a warp takes 32 / L consecutive rows per pass. Lane seg of a row holds the
+  //    float4 columns j * 4L + 4 seg (j < 4): for each of its four loads the row's lanes
+  //    cover one contiguous 16L-float span, so every access is a full line.
+  constexpr int SEG = 16;
+  constexpr int L = D / SEG;
+  constexpr int RPW = 32 / L;
   const int rows = G * D;
-  for (int r0 = warp * kRowUnroll; r0 < rows; r0 += kWarps * kRowUnroll) {
-    const int h = hk * G + r0 / D;          // kRowUnroll divides D: one value head per group
-    float s[kRowUnroll][VEC];
-    float* ptr[kRowUnroll];
+  const int seg = lane % L;
+  for (int r0 = warp * RPW; r0 < rows; r0 += kWarps * RPW) {
+    const int r = r0 + lane / L;
+    const bool live = r < rows;
+    const int h = hk * G + (live ? r : 0) / D;
+    float* ptr = state + ((b * Hv + h) * (int64_t)D + (live ? r : 0) % D) * D + seg * 4;
+    float s[SEG];
 #pragma unroll
-    for (int u = 0; u < kRowUnroll; ++u) {
-      const int r = r0 + u;
-      ptr[u] = state + ((b * Hv + h) * (int64_t)D + r % D) * D + lane * VEC;
-      if (r < rows && active) Row<VEC>::load(ptr[u], s[u]);
-      else {
-#pragma unroll
-        for (int j = 0; j < VEC; ++j) s[u][j] = 0.f;
-      }
+    for (int j = 0; j < SEG; j += 4) {
+      const float4 v = live ? __ldcs(reinterpret_cast<const float4*>(ptr + j * L)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      s[j] = v.x; s[j + 1] = v.y; s[j + 2] = v.z; s[j + 3] = v.w;
     }
 #pragma unroll
     for (int t = 0; t < kMaxTok; ++t) {
       if (t >= n_tok) break;
-      float qh[VEC], kh[VEC];
+      const float* qt = ys + t * n_local + seg * 4;
+      const float* kt = qt + D;
+      float kv[SEG], a = 0.f, c = 0.f;
 #pragma unroll
-      for (int j = 0; j < VEC; ++j) {
-        qh[j] = active ? ys[t * n_local + lane * VEC + j] : 0.f;
-        kh[j] = active ? ys[t * n_local + D + lane * VEC + j] : 0.f;
-      }
-      const float kqh = kqs[t];
-      float sk[kRowUnroll], sq[kRowUnroll];
-#pragma unroll
-      for (int u = 0; u < kRowUnroll; ++u) {
-        float a = 0.f, c = 0.f;
-#pragma unroll
-        for (int j = 0; j < VEC; ++j) { a = fmaf(s[u][j], kh[j], a); c = fmaf(s[u][j], qh[j], c); }
-        sk[u] = a; sq[u] = c;
+      for (int j = 0; j < SEG; j += 4) {
+        const float4 k4 = *reinterpret_cast<const float4*>(kt + j * L);
+        const float4 q4 = *reinterpret_cast<const float4*>(qt + j * L);
+        kv[j] = k4.x; kv[j + 1] = k4.y; kv[j + 2] = k4.z; kv[j + 3] = k4.w;
+        a = fmaf(s[j], k4.x, a); a = fmaf(s[j + 1], k4.y, a); a = fmaf(s[j + 2], k4.z, a); a = fmaf(s[j + 3], k4.w, a);
+        c = fmaf(s[j], q4.x, c); c = fmaf(s[j + 1], q4.y, c); c = fmaf(s[j + 2], q4.z, c); c = fmaf(s[j + 3], q4.w, c);
       }
 #pragma unroll
-      for (int m = 16; m >= 1; m >>= 1)
+      for (int m = L / 2; m >= 1; m >>= 1) {   // within the row's L lanes
+        a += __shfl_xor_sync(0xffffffffu, a, m);
+        c += __shfl_xor_sync(0xffffffffu, c, m);
+      }
+      if (live) {
+        const float alpha = expf(g[(b * n_tok + t) * Hv + h]);
+        const float bt = beta[(b * n_tok + t) * Hv + h];
+        const float uu = bt * (ys[t * n_local + 2 * D + r] - alpha * a);
 #pragma unroll
-        for (int u = 0; u < kRowUnroll; ++u) {
-          sk[u] += __shfl_xor_sync(0xffffffffu, sk[u], m);
-          sq[u] += __shfl_xor_sync(0xffffffffu, sq[u], m);
-        }
-      const float alpha = expf(g[(b * n_tok + t) * Hv + h]);
-      const float bt = beta[(b * n_tok + t) * Hv + h];
-#pragma unroll
-      for (int u = 0; u < kRowUnroll; ++u) {
-        const int r = r0 + u;
-        const float uu = r < rows ? bt * (ys[t * n_local + 2 * D + r] - alpha * sk[u]) : 0.f;
-#pragma unroll
-        for (int j = 0; j < VEC; ++j) s[u][j] = fmaf(alpha, s[u][j], uu * kh[j]);
-        if (lane == 0 && r < rows) os[t * rows + r] = scale * fmaf(alpha, sq[u], uu * kqh);
+        for (int j = 0; j < SEG; ++j) s[j] = fmaf(alpha, s[j], uu * kv[j]);
+        if (seg == 0) os[t * rows + r] = scale * fmaf(alpha, c, uu * kqs[t]);
       }
     }
+    if (live) {
 #pragma unroll
-    for (int u = 0; u < kRowUnroll; ++u)
-      if (r0 + u < rows && active) Row<VEC>::store(ptr[u], s[u]);
+      for (int j = 0; j < SEG; j += 4)
+        __stcs(reinterpret_cast<float4*>(ptr + j * L), make_float4(s[j], s[j + 1], s[j + 2], s[j + 3]));
+    }
   }
   __syncthreads();
 
