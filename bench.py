@@ -55,9 +55,9 @@ def conv_bytes(T, sh=SHAPE):
     return 2 * T * sh.conv_channels * 2 + sh.conv_channels * 4 * 2
 
 
-def decode_bytes(B, sh=SHAPE):
+def decode_bytes(B, sh=SHAPE, state_bytes=4):
     Cc = sh.conv_channels
-    state = B * sh.Hv * sh.dv * sh.dk * 4
+    state = B * sh.Hv * sh.dv * sh.dk * state_bytes
     return (2 * state + B * Cc * 2 + 2 * B * 3 * Cc * 2 + B * sh.Hv * sh.dv * 2
             + 2 * B * sh.Hv * 4 + Cc * 4 * 2)
 
@@ -233,6 +233,19 @@ def measure_configs(gdn, dev, stream, hbm_gbs, tc_sust):
            "tokens": 256, "sequences": 256, "ms": ms, "tokens_per_s": 256 / (ms / 1e3), "dtype": "bf16"}
     rec.update(_roof(ms, 0, decode_bytes(256, sh), tc_sust, hbm_gbs))
     out.append(rec)
+
+    # the same 100-step block with the states stored in bf16
+    st16 = st.to(torch.bfloat16)
+
+    def block16():
+        for t in range(100):
+            gdn.gdn_decode_step(xs[t], cw, cs, gs[t], bs[t], st16, sh.Hk, do)
+    ms = _median_ms(block16, stream, warmup=2, reps=20) / 100
+    rec = {"workload": "Qwen3.5-27B-shaped decode, bf16 states: B=256 x 1 token, 100-step block (per step)",
+           "tokens": 256, "sequences": 256, "ms": ms, "tokens_per_s": 256 / (ms / 1e3), "dtype": "bf16"}
+    rec.update(_roof(ms, 0, decode_bytes(256, sh, state_bytes=2), tc_sust, hbm_gbs))
+    out.append(rec)
+    del st16
 
     # multi-token decode / verify: 4 tokens per sequence per call (25 calls = 100 tokens)
     n_tok = 4

@@ -35,6 +35,10 @@ SIGNATURES = {
                                         _I32, _I32, _I32, _F32, _P]),
     "gdn_decode_tokens": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _I32, _I32, _I32,
                                          _I32, _I32, _I32, _F32, _P]),
+    "gdn_decode_step_ex": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int, _P, ctypes.c_int,
+                                          _I32, _I32, _I32, _I32, _I32, _F32, _P]),
+    "gdn_decode_tokens_ex": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int, _P, ctypes.c_int,
+                                            _I32, _I32, _I32, _I32, _I32, _I32, _F32, _P]),
     "gdn_chunk_prefill_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int, _I64, _I32,
                                                   _I32, _I32, _I32, _I64, _I64, _P, _I32, _P, _P,
                                                   _F32, _I32, _P]),
@@ -216,7 +220,8 @@ def gdn_chunk_prefill_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
 def gdn_decode_step(x: torch.Tensor, conv_w: torch.Tensor, conv_state: torch.Tensor,
                     g: torch.Tensor, beta: torch.Tensor, state: torch.Tensor, Hk: int,
                     o: Optional[torch.Tensor] = None, scale: float = 1.0) -> torch.Tensor:
-    """One decode token per sequence; conv_state and state are updated in place."""
+    """One decode token per sequence; conv_state and state are updated in place. The state
+    is fp32, or bf16 (stored in bf16, updated in fp32)."""
     B, Cc = x.shape
     _, Hv, dv, dk = state.shape
     dev = x.device
@@ -227,13 +232,13 @@ def gdn_decode_step(x: torch.Tensor, conv_w: torch.Tensor, conv_state: torch.Ten
     _need(conv_state, "conv_state", (B, 3, Cc), x.dtype, dev)
     _need(g, "g", (B, Hv), torch.float32, dev)
     _need(beta, "beta", (B, Hv), torch.float32, dev)
-    _need(state, "state", (B, Hv, dv, dk), torch.float32, dev)
+    _need(state, "state", (B, Hv, dv, dk), None, dev)
     if o is None:
         o = torch.empty((B, Hv, dv), dtype=x.dtype, device=dev)
     _need(o, "o", (B, Hv, dv), x.dtype, dev)
-    _check(lib().gdn_decode_step(_ptr(x), _ptr(conv_w), _ptr(conv_state), _ptr(g), _ptr(beta),
-                                 _ptr(state), _ptr(o), _dtype_code(x), B, Hk, Hv, dk, dv,
-                                 float(scale), _stream(dev)), "gdn_decode_step")
+    _check(lib().gdn_decode_step_ex(_ptr(x), _ptr(conv_w), _ptr(conv_state), _ptr(g), _ptr(beta),
+                                    _ptr(state), _dtype_code(state), _ptr(o), _dtype_code(x), B,
+                                    Hk, Hv, dk, dv, float(scale), _stream(dev)), "gdn_decode_step")
     return o
 
 
@@ -241,7 +246,7 @@ def gdn_decode_tokens(x: torch.Tensor, conv_w: torch.Tensor, conv_state: torch.T
                       g: torch.Tensor, beta: torch.Tensor, state: torch.Tensor, Hk: int,
                       o: Optional[torch.Tensor] = None, scale: float = 1.0) -> torch.Tensor:
     """n_tok (1..8) consecutive tokens per sequence, x [B, n_tok, Cc]; conv_state and state
-    are updated in place. Returns o [B, n_tok, Hv, dv]."""
+    (fp32, or bf16 storage) are updated in place. Returns o [B, n_tok, Hv, dv]."""
     B, n_tok, Cc = x.shape
     _, Hv, dv, dk = state.shape
     dev = x.device
@@ -252,11 +257,12 @@ def gdn_decode_tokens(x: torch.Tensor, conv_w: torch.Tensor, conv_state: torch.T
     _need(conv_state, "conv_state", (B, 3, Cc), x.dtype, dev)
     _need(g, "g", (B, n_tok, Hv), torch.float32, dev)
     _need(beta, "beta", (B, n_tok, Hv), torch.float32, dev)
-    _need(state, "state", (B, Hv, dv, dk), torch.float32, dev)
+    _need(state, "state", (B, Hv, dv, dk), None, dev)
     if o is None:
         o = torch.empty((B, n_tok, Hv, dv), dtype=x.dtype, device=dev)
     _need(o, "o", (B, n_tok, Hv, dv), x.dtype, dev)
-    _check(lib().gdn_decode_tokens(_ptr(x), _ptr(conv_w), _ptr(conv_state), _ptr(g), _ptr(beta),
-                                   _ptr(state), _ptr(o), _dtype_code(x), B, n_tok, Hk, Hv, dk, dv,
-                                   float(scale), _stream(dev)), "gdn_decode_tokens")
+    _check(lib().gdn_decode_tokens_ex(_ptr(x), _ptr(conv_w), _ptr(conv_state), _ptr(g), _ptr(beta),
+                                      _ptr(state), _dtype_code(state), _ptr(o), _dtype_code(x), B,
+                                      n_tok, Hk, Hv, dk, dv, float(scale), _stream(dev)),
+           "gdn_decode_tokens")
     return o

@@ -1,4 +1,5 @@
-// decode_step.cu -- one token for each of B sequences, conv taps and fp32 states in place.
+// decode_step.cu -- one token for each of B sequences, conv taps and states in place (states
+// stored in fp32, or in bf16 with fp32 arithmetic).
 //
 // Workload (Qwen3.5 page, section 8): decode is a state-update stream -- every token reads,
 // modifies and writes each fixed-size fp32 state. It is HBM-bound: per (sequence, value
@@ -24,8 +25,10 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kRowUnroll = 4;      // rows per warp iteration (loads in flight)
 constexpr float kEps = 1e-6f;
 
-template <int VEC> struct RowIO;
-template <> struct RowIO<4> {
+// VEC consecutive state values of one row, streamed (evict-first): fp32 storage, or bf16
+// storage widened to fp32 for the arithmetic and rounded once on the store.
+template <typename S, int VEC> struct RowIO;
+template <> struct RowIO<float, 4> {
   static __device__ __forceinline__ void load(const float* p, float (&s)[4]) {
     float4 v = __ldcs(reinterpret_cast<const float4*>(p));
     s[0] = v.x; s[1] = v.y; s[2] = v.z; s[3] = v.w;
@@ -34,7 +37,7 @@ template <> struct RowIO<4> {
     __stcs(reinterpret_cast<float4*>(p), make_float4(s[0], s[1], s[2], s[3]));
   }
 };
-template <> struct RowIO<2> {
+template <> struct RowIO<float, 2> {
   static __device__ __forceinline__ void load(const float* p, float (&s)[2]) {
     float2 v = __ldcs(reinterpret_cast<const float2*>(p));
     s[0] = v.x; s[1] = v.y;
@@ -43,16 +46,43 @@ template <> struct RowIO<2> {
     __stcs(reinterpret_cast<float2*>(p), make_float2(s[0], s[1]));
   }
 };
-template <> struct RowIO<1> {
+template <> struct RowIO<float, 1> {
   static __device__ __forceinline__ void load(const float* p, float (&s)[1]) { s[0] = __ldcs(p); }
   static __device__ __forceinline__ void store(float* p, const float (&s)[1]) { __stcs(p, s[0]); }
 };
+template <> struct RowIO<bf16, 4> {
+  static __device__ __forceinline__ void load(const bf16* p, float (&s)[4]) {
+    const uint2 u = __ldcs(reinterpret_cast<const uint2*>(p));
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+    s[0] = a.x; s[1] = a.y; s[2] = b.x; s[3] = b.y;
+  }
+  static __device__ __forceinline__ void store(bf16* p, const float (&s)[4]) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(s[0], s[1]), b = __floats2bfloat162_rn(s[2], s[3]);
+    __stcs(reinterpret_cast<uint2*>(p), make_uint2(*reinterpret_cast<uint32_t*>(&a), *reinterpret_cast<uint32_t*>(&b)));
+  }
+};
+template <> struct RowIO<bf16, 2> {
+  static __device__ __forceinline__ void load(const bf16* p, float (&s)[2]) {
+    const unsigned int u = __ldcs(reinterpret_cast<const unsigned int*>(p));
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u));
+    s[0] = a.x; s[1] = a.y;
+  }
+  static __device__ __forceinline__ void store(bf16* p, const float (&s)[2]) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(s[0], s[1]);
+    __stcs(reinterpret_cast<unsigned int*>(p), *reinterpret_cast<unsigned int*>(&a));
+  }
+};
+template <> struct RowIO<bf16, 1> {
+  static __device__ __forceinline__ void load(const bf16* p, float (&s)[1]) { s[0] = __bfloat162float(p[0]); }
+  static __device__ __forceinline__ void store(bf16* p, const float (&s)[1]) { p[0] = __float2bfloat16_rn(s[0]); }
+};
 
-template <typename T, int D>
+template <typename T, int D, typename S>
 __global__ void __launch_bounds__(kThreads)
 decode_step_kernel(const T* __restrict__ x, const T* __restrict__ conv_w, T* __restrict__ conv_state,
                    const float* __restrict__ g, const float* __restrict__ beta,
-                   float* __restrict__ state, T* __restrict__ o, int32_t Hk, int32_t Hv,
+                   S* __restrict__ state, T* __restrict__ o, int32_t Hk, int32_t Hv,
                    float scale) {
   constexpr int VEC = D >= 32 ? D / 32 : 1;
   const int G = Hv / Hk;
@@ -119,13 +149,13 @@ decode_step_kernel(const T* __restrict__ x, const T* __restrict__ conv_w, T* __r
   const int rows = G * D;
   for (int r0 = warp * kRowUnroll; r0 < rows; r0 += kWarps * kRowUnroll) {
     float s[kRowUnroll][VEC];
-    float* ptr[kRowUnroll];
+    S* ptr[kRowUnroll];
 #pragma unroll
     for (int u = 0; u < kRowUnroll; ++u) {
       const int r = r0 + u;
       const int h = hk * G + r / D, i = r % D;
       ptr[u] = state + ((b * Hv + h) * (int64_t)D + i) * D + lane * VEC;
-      if (r < rows && active) RowIO<VEC>::load(ptr[u], s[u]);
+      if (r < rows && active) RowIO<S, VEC>::load(ptr[u], s[u]);
       else {
 #pragma unroll
         for (int j = 0; j < VEC; ++j) s[u][j] = 0.f;
@@ -156,7 +186,7 @@ decode_step_kernel(const T* __restrict__ x, const T* __restrict__ conv_w, T* __r
       const float uu = bt * (ys[2 * D + r] - alpha * sk[u]);
 #pragma unroll
       for (int j = 0; j < VEC; ++j) s[u][j] = fmaf(alpha, s[u][j], uu * kh[j]);
-      if (active) RowIO<VEC>::store(ptr[u], s[u]);
+      if (active) RowIO<S, VEC>::store(ptr[u], s[u]);
       if (lane == 0) os[r] = scale * fmaf(alpha, sq[u], uu * kqh);
     }
   }
@@ -167,45 +197,50 @@ decode_step_kernel(const T* __restrict__ x, const T* __restrict__ conv_w, T* __r
   for (int e = threadIdx.x; e < rows; e += kThreads) ob[e] = from_f<T>(os[e]);
 }
 
-template <typename T, int D>
+template <typename T, int D, typename S>
 cudaError_t launch_typed(const void* x, const void* w, void* cs, const float* g, const float* beta,
-                         float* state, void* o, int32_t B, int32_t Hk, int32_t Hv, float scale,
+                         void* state, void* o, int32_t B, int32_t Hk, int32_t Hv, float scale,
                          cudaStream_t st) {
   const int G = Hv / Hk;
   const size_t smem = sizeof(float) * (size_t)((2 + G) * D + G * D);
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(decode_step_kernel<T, D>,
+    cudaError_t e = cudaFuncSetAttribute(decode_step_kernel<T, D, S>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
   dim3 grid((unsigned)((int64_t)B * Hk));
-  decode_step_kernel<T, D><<<grid, kThreads, smem, st>>>(
-      (const T*)x, (const T*)w, (T*)cs, g, beta, state, (T*)o, Hk, Hv, scale);
+  decode_step_kernel<T, D, S><<<grid, kThreads, smem, st>>>(
+      (const T*)x, (const T*)w, (T*)cs, g, beta, (S*)state, (T*)o, Hk, Hv, scale);
   return cudaGetLastError();
 }
 
-template <typename T>
+template <typename T, typename S>
 cudaError_t launch_d(const void* x, const void* w, void* cs, const float* g, const float* beta,
-                     float* state, void* o, int32_t B, int32_t Hk, int32_t Hv, int32_t d,
+                     void* state, void* o, int32_t B, int32_t Hk, int32_t Hv, int32_t d,
                      float scale, cudaStream_t st) {
   switch (d) {
-    case 16: return launch_typed<T, 16>(x, w, cs, g, beta, state, o, B, Hk, Hv, scale, st);
-    case 32: return launch_typed<T, 32>(x, w, cs, g, beta, state, o, B, Hk, Hv, scale, st);
-    case 64: return launch_typed<T, 64>(x, w, cs, g, beta, state, o, B, Hk, Hv, scale, st);
-    default: return launch_typed<T, 128>(x, w, cs, g, beta, state, o, B, Hk, Hv, scale, st);
+    case 16: return launch_typed<T, 16, S>(x, w, cs, g, beta, state, o, B, Hk, Hv, scale, st);
+    case 32: return launch_typed<T, 32, S>(x, w, cs, g, beta, state, o, B, Hk, Hv, scale, st);
+    case 64: return launch_typed<T, 64, S>(x, w, cs, g, beta, state, o, B, Hk, Hv, scale, st);
+    default: return launch_typed<T, 128, S>(x, w, cs, g, beta, state, o, B, Hk, Hv, scale, st);
   }
 }
 
 }  // namespace
 
 cudaError_t launch_decode_step(int dtype, const void* x, const void* conv_w, void* conv_state,
-                               const float* g, const float* beta, float* state, void* o,
-                               int32_t B, int32_t Hk, int32_t Hv, int32_t d, float scale,
+                               const float* g, const float* beta, void* state, int state_dtype,
+                               void* o, int32_t B, int32_t Hk, int32_t Hv, int32_t d, float scale,
                                cudaStream_t stream) {
   if (B == 0) return cudaSuccess;
-  if (dtype == kF32)
-    return launch_d<float>(x, conv_w, conv_state, g, beta, state, o, B, Hk, Hv, d, scale, stream);
-  return launch_d<bf16>(x, conv_w, conv_state, g, beta, state, o, B, Hk, Hv, d, scale, stream);
+  if (dtype == kF32) {
+    if (state_dtype == kF32)
+      return launch_d<float, float>(x, conv_w, conv_state, g, beta, state, o, B, Hk, Hv, d, scale, stream);
+    return launch_d<float, bf16>(x, conv_w, conv_state, g, beta, state, o, B, Hk, Hv, d, scale, stream);
+  }
+  if (state_dtype == kF32)
+    return launch_d<bf16, float>(x, conv_w, conv_state, g, beta, state, o, B, Hk, Hv, d, scale, stream);
+  return launch_d<bf16, bf16>(x, conv_w, conv_state, g, beta, state, o, B, Hk, Hv, d, scale, stream);
 }
 
 }  // namespace gdn

@@ -1,5 +1,6 @@
 // decode_tokens.cu -- n_tok (1..8) consecutive tokens for each of B sequences, conv taps and
-// fp32 states in place: a multi-token decode / speculative verify step.
+// states in place (fp32, or bf16 storage with fp32 arithmetic): a multi-token decode /
+// speculative verify step.
 //
 // Same update as the single-token step (Qwen3.5 page, section 5: decay, then the delta
 // write along k; section 8: decode is a state-update stream), applied n_tok times. The
@@ -25,11 +26,31 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kMaxTok = 8;
 constexpr float kEps = 1e-6f;
 
-template <typename T, int D>
+// Four consecutive state values, streamed (evict-first): fp32 storage, or bf16 storage
+// widened to fp32 for the arithmetic and rounded once on the store.
+template <typename S> struct Quad;
+template <> struct Quad<float> {
+  static __device__ __forceinline__ float4 load(const float* p) { return __ldcs(reinterpret_cast<const float4*>(p)); }
+  static __device__ __forceinline__ void store(float* p, float4 v) { __stcs(reinterpret_cast<float4*>(p), v); }
+};
+template <> struct Quad<bf16> {
+  static __device__ __forceinline__ float4 load(const bf16* p) {
+    const uint2 u = __ldcs(reinterpret_cast<const uint2*>(p));
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+  }
+  static __device__ __forceinline__ void store(bf16* p, float4 v) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+    __stcs(reinterpret_cast<uint2*>(p), make_uint2(*reinterpret_cast<uint32_t*>(&a), *reinterpret_cast<uint32_t*>(&b)));
+  }
+};
+
+template <typename T, int D, typename S>
 __global__ void __launch_bounds__(kThreads, 3)
 decode_tokens_kernel(const T* __restrict__ x, const T* __restrict__ conv_w, T* __restrict__ conv_state,
                      const float* __restrict__ g, const float* __restrict__ beta,
-                     float* __restrict__ state, T* __restrict__ o, int32_t Hk, int32_t Hv,
+                     S* __restrict__ state, T* __restrict__ o, int32_t Hk, int32_t Hv,
                      int32_t n_tok, float scale) {
   constexpr int VEC = D >= 32 ? D / 32 : 1;
   const int G = Hv / Hk;
@@ -135,11 +156,11 @@ decode_tokens_kernel(const T* __restrict__ x, const T* __restrict__ conv_w, T* _
     const int r = r0 + lane / L;
     const bool live = r < rows;
     const int h = hk * G + (live ? r : 0) / D;
-    float* ptr = state + ((b * Hv + h) * (int64_t)D + (live ? r : 0) % D) * D + seg * 4;
+    S* ptr = state + ((b * Hv + h) * (int64_t)D + (live ? r : 0) % D) * D + seg * 4;
     float s[SEG];
 #pragma unroll
     for (int j = 0; j < SEG; j += 4) {
-      const float4 v = live ? __ldcs(reinterpret_cast<const float4*>(ptr + j * L)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 v = live ? Quad<S>::load(ptr + j * L) : make_float4(0.f, 0.f, 0.f, 0.f);
       s[j] = v.x; s[j + 1] = v.y; s[j + 2] = v.z; s[j + 3] = v.w;
     }
 #pragma unroll
@@ -173,7 +194,7 @@ decode_tokens_kernel(const T* __restrict__ x, const T* __restrict__ conv_w, T* _
     if (live) {
 #pragma unroll
       for (int j = 0; j < SEG; j += 4)
-        __stcs(reinterpret_cast<float4*>(ptr + j * L), make_float4(s[j], s[j + 1], s[j + 2], s[j + 3]));
+        Quad<S>::store(ptr + j * L, make_float4(s[j], s[j + 1], s[j + 2], s[j + 3]));
     }
   }
   __syncthreads();
@@ -185,44 +206,49 @@ decode_tokens_kernel(const T* __restrict__ x, const T* __restrict__ conv_w, T* _
   }
 }
 
-template <typename T, int D>
+template <typename T, int D, typename S>
 cudaError_t launch_typed(const void* x, const void* w, void* cs, const float* g, const float* beta,
-                         float* state, void* o, int32_t B, int32_t n_tok, int32_t Hk, int32_t Hv,
+                         void* state, void* o, int32_t B, int32_t n_tok, int32_t Hk, int32_t Hv,
                          float scale, cudaStream_t st) {
   const int G = Hv / Hk;
   const size_t smem = sizeof(float) * (size_t)n_tok * ((2 + G) * D + G * D + 1);
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(decode_tokens_kernel<T, D>,
+    cudaError_t e = cudaFuncSetAttribute(decode_tokens_kernel<T, D, S>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
   dim3 grid((unsigned)((int64_t)B * Hk));
-  decode_tokens_kernel<T, D><<<grid, kThreads, smem, st>>>(
-      (const T*)x, (const T*)w, (T*)cs, g, beta, state, (T*)o, Hk, Hv, n_tok, scale);
+  decode_tokens_kernel<T, D, S><<<grid, kThreads, smem, st>>>(
+      (const T*)x, (const T*)w, (T*)cs, g, beta, (S*)state, (T*)o, Hk, Hv, n_tok, scale);
   return cudaGetLastError();
 }
 
-template <typename T>
+template <typename T, typename S>
 cudaError_t launch_d(const void* x, const void* w, void* cs, const float* g, const float* beta,
-                     float* state, void* o, int32_t B, int32_t n_tok, int32_t Hk, int32_t Hv,
+                     void* state, void* o, int32_t B, int32_t n_tok, int32_t Hk, int32_t Hv,
                      int32_t d, float scale, cudaStream_t st) {
   switch (d) {
-    case 16: return launch_typed<T, 16>(x, w, cs, g, beta, state, o, B, n_tok, Hk, Hv, scale, st);
-    case 32: return launch_typed<T, 32>(x, w, cs, g, beta, state, o, B, n_tok, Hk, Hv, scale, st);
-    case 64: return launch_typed<T, 64>(x, w, cs, g, beta, state, o, B, n_tok, Hk, Hv, scale, st);
-    default: return launch_typed<T, 128>(x, w, cs, g, beta, state, o, B, n_tok, Hk, Hv, scale, st);
+    case 16: return launch_typed<T, 16, S>(x, w, cs, g, beta, state, o, B, n_tok, Hk, Hv, scale, st);
+    case 32: return launch_typed<T, 32, S>(x, w, cs, g, beta, state, o, B, n_tok, Hk, Hv, scale, st);
+    case 64: return launch_typed<T, 64, S>(x, w, cs, g, beta, state, o, B, n_tok, Hk, Hv, scale, st);
+    default: return launch_typed<T, 128, S>(x, w, cs, g, beta, state, o, B, n_tok, Hk, Hv, scale, st);
   }
 }
 
 }  // namespace
 
 cudaError_t launch_decode_tokens(int dtype, const void* x, const void* conv_w, void* conv_state,
-                                 const float* g, const float* beta, float* state, void* o,
-                                 int32_t B, int32_t n_tok, int32_t Hk, int32_t Hv, int32_t d,
+                                 const float* g, const float* beta, void* state, int state_dtype,
+                                 void* o, int32_t B, int32_t n_tok, int32_t Hk, int32_t Hv, int32_t d,
                                  float scale, cudaStream_t stream) {
-  if (dtype == kF32)
-    return launch_d<float>(x, conv_w, conv_state, g, beta, state, o, B, n_tok, Hk, Hv, d, scale, stream);
-  return launch_d<bf16>(x, conv_w, conv_state, g, beta, state, o, B, n_tok, Hk, Hv, d, scale, stream);
+  if (dtype == kF32) {
+    if (state_dtype == kF32)
+      return launch_d<float, float>(x, conv_w, conv_state, g, beta, state, o, B, n_tok, Hk, Hv, d, scale, stream);
+    return launch_d<float, bf16>(x, conv_w, conv_state, g, beta, state, o, B, n_tok, Hk, Hv, d, scale, stream);
+  }
+  if (state_dtype == kF32)
+    return launch_d<bf16, float>(x, conv_w, conv_state, g, beta, state, o, B, n_tok, Hk, Hv, d, scale, stream);
+  return launch_d<bf16, bf16>(x, conv_w, conv_state, g, beta, state, o, B, n_tok, Hk, Hv, d, scale, stream);
 }
 
 }  // namespace gdn

@@ -168,11 +168,12 @@ gdn_status_t gdn_chunk_prefill(const void* q, const void* k, const void* v, cons
                      "chunk_prefill launch");
 }
 
-gdn_status_t gdn_decode_step(const void* x, const void* conv_w, void* conv_state, const float* g,
-                             const float* beta, float* state, void* o, gdn_dtype_t dt, int32_t B,
-                             int32_t Hk, int32_t Hv, int32_t dk, int32_t dv, float scale,
-                             gdn_stream_t stream) {
+gdn_status_t gdn_decode_step_ex(const void* x, const void* conv_w, void* conv_state, const float* g,
+                                const float* beta, void* state, gdn_dtype_t state_dt, void* o,
+                                gdn_dtype_t dt, int32_t B, int32_t Hk, int32_t Hv, int32_t dk,
+                                int32_t dv, float scale, gdn_stream_t stream) {
   if (!valid_dtype(dt)) return fail(GDN_ERR_UNSUPPORTED, "decode_step: unknown dtype %d", (int)dt);
+  if (!valid_dtype(state_dt)) return fail(GDN_ERR_UNSUPPORTED, "decode_step: unknown state dtype %d", (int)state_dt);
   if (B < 0) return fail(GDN_ERR_INVALID_ARG, "decode_step: B = %d < 0", B);
   if (Hk <= 0 || Hv <= 0) return fail(GDN_ERR_INVALID_ARG, "decode_step: Hk, Hv must be > 0");
   if (Hv % Hk != 0) return fail(GDN_ERR_UNSUPPORTED, "decode_step: Hv %% Hk != 0 (%d, %d)", Hv, Hk);
@@ -188,7 +189,7 @@ gdn_status_t gdn_decode_step(const void* x, const void* conv_w, void* conv_state
   const size_t es = elt_size(dt);
   const int64_t Cc = 2LL * Hk * dk + (int64_t)Hv * dv;
   const size_t xb = (size_t)B * Cc * es, csb = (size_t)B * 3 * Cc * es;
-  const size_t stb = (size_t)B * Hv * dv * dk * 4, ob = (size_t)B * Hv * dv * es;
+  const size_t stb = (size_t)B * Hv * dv * dk * elt_size(state_dt), ob = (size_t)B * Hv * dv * es;
   const size_t gb = (size_t)B * Hv * 4, wb = (size_t)Cc * 4 * es;
   const void* ro[4] = {x, conv_w, g, beta};
   const size_t rob[4] = {xb, wb, gb, gb};
@@ -199,16 +200,26 @@ gdn_status_t gdn_decode_step(const void* x, const void* conv_w, void* conv_state
   if (overlap(conv_state, csb, state, stb) || overlap(conv_state, csb, o, ob) ||
       overlap(state, stb, o, ob))
     return fail(GDN_ERR_INVALID_ARG, "decode_step: conv_state, state and o must not overlap");
-  return cuda_status(gdn::launch_decode_step((int)dt, x, conv_w, conv_state, g, beta, state, o, B,
-                                             Hk, Hv, dk, scale, (cudaStream_t)stream),
+  return cuda_status(gdn::launch_decode_step((int)dt, x, conv_w, conv_state, g, beta, state,
+                                             (int)state_dt, o, B, Hk, Hv, dk, scale,
+                                             (cudaStream_t)stream),
                      "decode_step launch");
 }
 
-gdn_status_t gdn_decode_tokens(const void* x, const void* conv_w, void* conv_state, const float* g,
-                               const float* beta, float* state, void* o, gdn_dtype_t dt, int32_t B,
-                               int32_t n_tok, int32_t Hk, int32_t Hv, int32_t dk, int32_t dv,
-                               float scale, gdn_stream_t stream) {
+gdn_status_t gdn_decode_step(const void* x, const void* conv_w, void* conv_state, const float* g,
+                             const float* beta, float* state, void* o, gdn_dtype_t dt, int32_t B,
+                             int32_t Hk, int32_t Hv, int32_t dk, int32_t dv, float scale,
+                             gdn_stream_t stream) {
+  return gdn_decode_step_ex(x, conv_w, conv_state, g, beta, state, GDN_F32, o, dt, B, Hk, Hv, dk,
+                            dv, scale, stream);
+}
+
+gdn_status_t gdn_decode_tokens_ex(const void* x, const void* conv_w, void* conv_state, const float* g,
+                                  const float* beta, void* state, gdn_dtype_t state_dt, void* o,
+                                  gdn_dtype_t dt, int32_t B, int32_t n_tok, int32_t Hk, int32_t Hv,
+                                  int32_t dk, int32_t dv, float scale, gdn_stream_t stream) {
   if (!valid_dtype(dt)) return fail(GDN_ERR_UNSUPPORTED, "decode_tokens: unknown dtype %d", (int)dt);
+  if (!valid_dtype(state_dt)) return fail(GDN_ERR_UNSUPPORTED, "decode_tokens: unknown state dtype %d", (int)state_dt);
   if (B < 0) return fail(GDN_ERR_INVALID_ARG, "decode_tokens: B = %d < 0", B);
   if (n_tok < 1 || n_tok > 8) return fail(GDN_ERR_INVALID_ARG, "decode_tokens: n_tok = %d outside [1, 8]", n_tok);
   if (Hk <= 0 || Hv <= 0) return fail(GDN_ERR_INVALID_ARG, "decode_tokens: Hk, Hv must be > 0");
@@ -216,7 +227,7 @@ gdn_status_t gdn_decode_tokens(const void* x, const void* conv_w, void* conv_sta
   if (dk != dv || !supported_head_dim(dk))
     return fail(GDN_ERR_UNSUPPORTED, "decode_tokens: head dims dk=%d dv=%d (need dk = dv in {16,32,64,128})", dk, dv);
   const int64_t G = Hv / Hk;
-  if ((int64_t)n_tok * ((2 + G) * dk + G * dk) * 4 > 227 * 1024)
+  if ((int64_t)n_tok * ((2 + G) * dk + G * dk + 1) * 4 > 227 * 1024)
     return fail(GDN_ERR_UNSUPPORTED, "decode_tokens: %d tokens of %lld value heads per key head exceed shared memory",
                 n_tok, (long long)G);
   if ((int64_t)B * Hk > 0x7fffffffLL) return fail(GDN_ERR_INVALID_ARG, "decode_tokens: B * Hk too large");
@@ -229,7 +240,7 @@ gdn_status_t gdn_decode_tokens(const void* x, const void* conv_w, void* conv_sta
   const size_t es = elt_size(dt);
   const int64_t Cc = 2LL * Hk * dk + (int64_t)Hv * dv;
   const size_t xb = (size_t)B * n_tok * Cc * es, csb = (size_t)B * 3 * Cc * es;
-  const size_t stb = (size_t)B * Hv * dv * dk * 4, ob = (size_t)B * n_tok * Hv * dv * es;
+  const size_t stb = (size_t)B * Hv * dv * dk * elt_size(state_dt), ob = (size_t)B * n_tok * Hv * dv * es;
   const size_t gb = (size_t)B * n_tok * Hv * 4, wb = (size_t)Cc * 4 * es;
   const void* ro[4] = {x, conv_w, g, beta};
   const size_t rob[4] = {xb, wb, gb, gb};
@@ -240,9 +251,18 @@ gdn_status_t gdn_decode_tokens(const void* x, const void* conv_w, void* conv_sta
   if (overlap(conv_state, csb, state, stb) || overlap(conv_state, csb, o, ob) ||
       overlap(state, stb, o, ob))
     return fail(GDN_ERR_INVALID_ARG, "decode_tokens: conv_state, state and o must not overlap");
-  return cuda_status(gdn::launch_decode_tokens((int)dt, x, conv_w, conv_state, g, beta, state, o, B,
-                                               n_tok, Hk, Hv, dk, scale, (cudaStream_t)stream),
+  return cuda_status(gdn::launch_decode_tokens((int)dt, x, conv_w, conv_state, g, beta, state,
+                                               (int)state_dt, o, B, n_tok, Hk, Hv, dk, scale,
+                                               (cudaStream_t)stream),
                      "decode_tokens launch");
+}
+
+gdn_status_t gdn_decode_tokens(const void* x, const void* conv_w, void* conv_state, const float* g,
+                               const float* beta, float* state, void* o, gdn_dtype_t dt, int32_t B,
+                               int32_t n_tok, int32_t Hk, int32_t Hv, int32_t dk, int32_t dv,
+                               float scale, gdn_stream_t stream) {
+  return gdn_decode_tokens_ex(x, conv_w, conv_state, g, beta, state, GDN_F32, o, dt, B, n_tok, Hk,
+                              Hv, dk, dv, scale, stream);
 }
 
 }  // extern "C"

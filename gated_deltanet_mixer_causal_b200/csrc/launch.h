@@ -16,14 +16,15 @@ cudaError_t launch_conv1d_silu(int dtype, const void* x, void* y, const void* w,
                                const void* conv_state_in, void* conv_state_out,
                                cudaStream_t stream);
 
+// state_dtype: kF32, or kBF16 for bf16 state storage (fp32 arithmetic)
 cudaError_t launch_decode_step(int dtype, const void* x, const void* conv_w, void* conv_state,
-                               const float* g, const float* beta, float* state, void* o,
-                               int32_t B, int32_t Hk, int32_t Hv, int32_t d, float scale,
+                               const float* g, const float* beta, void* state, int state_dtype,
+                               void* o, int32_t B, int32_t Hk, int32_t Hv, int32_t d, float scale,
                                cudaStream_t stream);
 // n_tok (1..8) tokens per sequence; x [B, n_tok, Cc], g/beta [B, n_tok, Hv], o [B, n_tok, Hv, d]
 cudaError_t launch_decode_tokens(int dtype, const void* x, const void* conv_w, void* conv_state,
-                                 const float* g, const float* beta, float* state, void* o,
-                                 int32_t B, int32_t n_tok, int32_t Hk, int32_t Hv, int32_t d,
+                                 const float* g, const float* beta, void* state, int state_dtype,
+                                 void* o, int32_t B, int32_t n_tok, int32_t Hk, int32_t Hv, int32_t d,
                                  float scale, cudaStream_t stream);
 
 // Token-by-token fp32 recurrence (SIMT): the fp32-activation prefill path.

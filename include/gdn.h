@@ -223,6 +223,29 @@ gdn_status_t gdn_decode_tokens(const void* x, const void* conv_w, void* conv_sta
                                gdn_dtype_t dt, int32_t B, int32_t n_tok, int32_t Hk, int32_t Hv,
                                int32_t dk, int32_t dv, float scale, gdn_stream_t stream);
 
+/*
+ * gdn_decode_step_ex, gdn_decode_tokens_ex -- gdn_decode_step and gdn_decode_tokens with the
+ * recurrent state stored as state_dt: GDN_F32 (the calls above), or GDN_BF16, which halves
+ * the bytes that dominate decode (Qwen3.5 page, section 8: decode moves the fixed-size state
+ * every token). With GDN_BF16 each state element is widened to fp32 on load, the update is
+ * computed in fp32 as for GDN_F32, and the result is rounded to bf16 (nearest, ties to even)
+ * once per call when it is stored: gdn_decode_tokens_ex rounds after all n_tok tokens.
+ *
+ * state       [B, Hv, dv, dk] of state_dt, 16-byte aligned, read and updated in place.
+ * Every other argument, and the return codes, as in gdn_decode_step / gdn_decode_tokens
+ * (GDN_ERR_UNSUPPORTED also for an unknown state_dt).
+ */
+gdn_status_t gdn_decode_step_ex(const void* x, const void* conv_w, void* conv_state,
+                                const float* g, const float* beta, void* state,
+                                gdn_dtype_t state_dt, void* o, gdn_dtype_t dt, int32_t B,
+                                int32_t Hk, int32_t Hv, int32_t dk, int32_t dv, float scale,
+                                gdn_stream_t stream);
+gdn_status_t gdn_decode_tokens_ex(const void* x, const void* conv_w, void* conv_state,
+                                  const float* g, const float* beta, void* state,
+                                  gdn_dtype_t state_dt, void* o, gdn_dtype_t dt, int32_t B,
+                                  int32_t n_tok, int32_t Hk, int32_t Hv, int32_t dk, int32_t dv,
+                                  float scale, gdn_stream_t stream);
+
 #ifdef __cplusplus
 }  /* extern "C" */
 #endif

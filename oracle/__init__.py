@@ -154,26 +154,37 @@ def layer_prefill(x, conv_w, g, beta, Hk, Hv, dk, dv, cu_seqlens=None, initial_s
     return o, fin, conv_out
 
 
+def round_bf16(a):
+    """Round to the nearest bfloat16 value (ties to even), returned as float64: the storage
+    of a bf16 state between decode calls."""
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float64)).to(torch.bfloat16).to(
+        torch.float64).numpy()
+
+
 def decode_step(x, conv_w, conv_state, g, beta, state, Hk, Hv, dk, dv, scale=1.0,
-                n_threads=None):
+                n_threads=None, state_dtype="f32"):
     """One token for each of B sequences: a decode step is the prefill of B sequences
     of length one that start from the carried conv taps and recurrent states.
 
     x [B, Cc]; conv_state [B, 3, Cc]; g, beta [B, Hv]; state [B, Hv, dv, dk].
+    state_dtype "bf16": the state is stored in bf16, so the new state is rounded to bf16.
     Returns (o [B, Hv, dv], new_state, new_conv_state); inputs are not modified.
     """
     B = np.asarray(x).shape[0]
     cu = np.arange(B + 1, dtype=np.int32)
-    return layer_prefill(x, conv_w, g, beta, Hk, Hv, dk, dv, cu, state, conv_state, scale,
-                         n_threads)
+    o, S, cs = layer_prefill(x, conv_w, g, beta, Hk, Hv, dk, dv, cu, state, conv_state, scale,
+                             n_threads)
+    return o, (round_bf16(S) if state_dtype == "bf16" else S), cs
 
 
 def decode_tokens(x, conv_w, conv_state, g, beta, state, Hk, Hv, dk, dv, scale=1.0,
-                  n_threads=None):
+                  n_threads=None, state_dtype="f32"):
     """n consecutive tokens for each of B sequences: the prefill of B sequences of n tokens
     that start from the carried conv taps and recurrent states.
 
     x [B, n, Cc]; conv_state [B, 3, Cc]; g, beta [B, n, Hv]; state [B, Hv, dv, dk].
+    state_dtype "bf16": the state is stored in bf16, rounded once after the n tokens.
     Returns (o [B, n, Hv, dv], new_state, new_conv_state); inputs are not modified.
     """
     x = np.asarray(x)
@@ -182,7 +193,7 @@ def decode_tokens(x, conv_w, conv_state, g, beta, state, Hk, Hv, dk, dv, scale=1
     o, S, cs = layer_prefill(x.reshape(B * n, Cc), conv_w, np.asarray(g).reshape(B * n, Hv),
                              np.asarray(beta).reshape(B * n, Hv), Hk, Hv, dk, dv, cu, state,
                              conv_state, scale, n_threads)
-    return o.reshape(B, n, Hv, dv), S, cs
+    return o.reshape(B, n, Hv, dv), (round_bf16(S) if state_dtype == "bf16" else S), cs
 
 
 def layer_state_bytes(Hv, dk, dv, state_bytes, conv_channels, conv_taps, conv_bytes) -> int:

@@ -151,6 +151,24 @@ def test_decode_tokens_validation(L):
     assert _decode_tokens(L, o=FAKE + (5 << 30) + 128) == _lib.GDN_ERR_INVALID_ARG   # o inside state
 
 
+def test_decode_state_dtype_validation(L):
+    def step(state_dt, **kw):
+        a = dict(x=FAKE, w=FAKE + (1 << 30), cs=FAKE + (2 << 30), g=FAKE + (3 << 30),
+                 b=FAKE + (4 << 30), st=FAKE + (5 << 30), o=FAKE + (6 << 30), B=8)
+        a.update(kw)
+        return L.gdn_decode_step_ex(a["x"], a["w"], a["cs"], a["g"], a["b"], a["st"], state_dt,
+                                    a["o"], 1, a["B"], 2, 4, 32, 32, 1.0, None)
+    assert step(7) == _lib.GDN_ERR_UNSUPPORTED
+    assert step(1, B=0) == _lib.GDN_OK
+    # a bf16 state of 8 x 4 x 32 x 32 is 64 KB: o placed 40 KB in overlaps only as bf16 ... and
+    # as fp32 (128 KB); 72 KB in overlaps the fp32 state but not the bf16 one
+    assert step(1, o=FAKE + (5 << 30) + 40 * 1024) == _lib.GDN_ERR_INVALID_ARG
+    assert step(0, o=FAKE + (5 << 30) + 72 * 1024) == _lib.GDN_ERR_INVALID_ARG
+    assert L.gdn_decode_tokens_ex(FAKE, FAKE + (1 << 30), FAKE + (2 << 30), FAKE + (3 << 30),
+                                  FAKE + (4 << 30), FAKE + (5 << 30), 9, FAKE + (6 << 30), 1, 8, 4,
+                                  2, 4, 32, 32, 1.0, None) == _lib.GDN_ERR_UNSUPPORTED
+
+
 def test_python_binding_refuses_cpu_tensors():
     import torch
     x = torch.zeros(8, 64, dtype=torch.bfloat16)

@@ -352,3 +352,55 @@ def test_decode_tokens_equals_single_steps_on_gpu(cuda_device):
     np.testing.assert_allclose(np64(o4), np64(torch.stack(outs, 1)), rtol=1e-2, atol=1e-3)
     assert max_rel(np64(st4), np64(st1)) <= 1e-5
     assert torch.equal(cs4, cs1)
+
+
+# ---------------------------------------------------------------- bf16 states
+
+def test_decode_bf16_state_27b(cuda_device):
+    """27B-shaped heads, 16 sequences, 20 single-token steps with the states stored in bf16;
+    the oracle rounds its state to bf16 after every step. Checked every 5th step."""
+    d = W.make_decode(W.QWEN35_27B, B=16, steps=20, seed=46)
+    sh = d.shape
+    st_r = oracle.round_bf16(d.state.numpy())
+    st = torch.from_numpy(st_r).to(torch.bfloat16).to(cuda_device)
+    cs = d.conv_state.to(cuda_device).clone()
+    cs_r = d.conv_state.float().numpy().astype(np.float64)
+    w = d.conv_w.to(cuda_device)
+    for t in range(20):
+        o = gdn.gdn_decode_step(d.xs[t].to(cuda_device), w, cs, d.gs[t].to(cuda_device),
+                                d.betas[t].to(cuda_device), st, sh.Hk)
+        o_r, st_r, cs_r = oracle.decode_step(d.xs[t].float().numpy(), d.conv_w.float().numpy(),
+                                             cs_r, d.gs[t].numpy(), d.betas[t].numpy(), st_r,
+                                             sh.Hk, sh.Hv, sh.dk, sh.dv, state_dtype="bf16")
+        if (t + 1) % 5 == 0:
+            torch.cuda.synchronize()
+            o_g, st_g = np64(o), np64(st)
+            for j in range(16):
+                for h in range(sh.Hv):
+                    assert frob_rel(o_g[j, h], o_r[j, h]) <= BF16_TOL, (t, j, h)
+                    assert frob_rel(st_g[j, h], st_r[j, h]) <= BF16_TOL, (t, j, h)
+            np.testing.assert_array_equal(np64(cs), cs_r)
+    assert st.dtype == torch.bfloat16
+
+
+@pytest.mark.parametrize("n_tok", [1, 4])
+def test_decode_tokens_bf16_state_27b(cuda_device, n_tok):
+    """n_tok tokens in one call with a bf16 state (rounded once, after the last token)."""
+    d = W.make_decode(W.QWEN35_27B, B=16, steps=n_tok, seed=47)
+    sh = d.shape
+    x = torch.stack(d.xs, 1); g = torch.stack(d.gs, 1); b = torch.stack(d.betas, 1)
+    s0 = oracle.round_bf16(d.state.numpy())
+    st = torch.from_numpy(s0).to(torch.bfloat16).to(cuda_device)
+    cs = d.conv_state.to(cuda_device).clone()
+    o = gdn.gdn_decode_tokens(x.to(cuda_device), d.conv_w.to(cuda_device), cs, g.to(cuda_device),
+                              b.to(cuda_device), st, sh.Hk)
+    torch.cuda.synchronize()
+    o_r, st_r, cs_r = oracle.decode_tokens(x.float().numpy(), d.conv_w.float().numpy(),
+                                           d.conv_state.float().numpy(), g.numpy(), b.numpy(), s0,
+                                           sh.Hk, sh.Hv, sh.dk, sh.dv, state_dtype="bf16")
+    o_g, st_g = np64(o), np64(st)
+    for j in range(16):
+        for h in range(sh.Hv):
+            assert frob_rel(o_g[j, :, h], o_r[j, :, h]) <= BF16_TOL, (j, h)
+            assert frob_rel(st_g[j, h], st_r[j, h]) <= BF16_TOL, (j, h)
+    np.testing.assert_array_equal(np64(cs), cs_r)

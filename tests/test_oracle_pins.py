@@ -327,6 +327,23 @@ def test_decode_tokens_equal_single_steps(oracle_mod):
     np.testing.assert_array_equal(cs_m, xs[:, -3:])
 
 
+def test_bf16_state_rounding(oracle_mod):
+    """bf16 keeps 8 significant bits: exact halfway cases go to the even neighbour, bf16
+    values are fixed points, and every value moves by at most half a unit in the last place."""
+    u = 2.0 ** -7                                      # ulp of bf16 in [1, 2)
+    cases = {1.0 + u / 2: 1.0, 1.0 + 1.5 * u: 1.0 + 2 * u, 1.0 + 0.49 * u: 1.0,
+             -(1.0 + 2.5 * u): -(1.0 + 2 * u),
+             3.0 * 2.0 ** -133: 3.0 * 2.0 ** -133,     # subnormal: a multiple of 2^-133
+             3.0 * 2.0 ** -140: 0.0}                   # below half the smallest subnormal
+    for v, want in cases.items():
+        assert oracle.round_bf16(np.array([v]))[0] == want, v
+    r = rng(19).standard_normal(10000) * 10.0 ** rng(20).uniform(-6, 6, 10000)
+    b = oracle.round_bf16(r)
+    np.testing.assert_array_equal(oracle.round_bf16(b), b)
+    ulp = 2.0 ** (np.floor(np.log2(np.abs(r))) - 7)
+    assert np.all(np.abs(b - r) <= ulp / 2)
+
+
 def test_empty_sequence_passes_state_through(oracle_mod):
     r = rng(17)
     q, k, v, g, beta, S0 = _random_case(r, 4, 1, 1, 3)
