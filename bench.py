@@ -524,8 +524,8 @@ def gdn_prefill_launches() -> int:
 # of each kernel on the small case (T = 8192, decode batch 64), per unit processed (token
 # for the prefill kernels and the conv, sequence for the decode step), scaled to the
 # benchmark's launch; None when the kernel changed since the capture.
-TRAFFIC_PER_UNIT = {"prefill": None, "conv": None,
-                    "decode": 354.37e6 / 64}
+TRAFFIC_PER_UNIT = {"prefill": (375.06e6 + 405.27e6) / 8192, "conv": 289.54e6 / 8192,
+                    "decode": 355.05e6 / 64}
 
 
 def traffic(kernel: str, units: int):
