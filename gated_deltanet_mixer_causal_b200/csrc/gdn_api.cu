@@ -50,8 +50,10 @@ bool supported_head_dim(int32_t d) { return d == 16 || d == 32 || d == 64 || d =
 
 // bf16 activations with 128-wide heads (and at most 8 value heads per key head) run the
 // chunked tensor-core prefill; everything else runs the token-by-token fp32 kernel.
-bool use_tensor_core_prefill(gdn_dtype_t dt, int32_t d, int32_t Hk, int32_t Hv) {
-  return dt == GDN_BF16 && d == 128 && Hv / Hk <= gdn::kPrefillTcMaxG;
+// The tensor-core prefill folds the q/k L2 norm into its factors; inputs used as given
+// (qk_l2norm = 0) take the token-recurrent path.
+bool use_tensor_core_prefill(gdn_dtype_t dt, int32_t d, int32_t Hk, int32_t Hv, int32_t qk_l2norm = 1) {
+  return dt == GDN_BF16 && d == 128 && Hv / Hk <= gdn::kPrefillTcMaxG && qk_l2norm != 0;
 }
 
 }  // namespace
@@ -153,7 +155,7 @@ gdn_status_t gdn_chunk_prefill(const void* q, const void* k, const void* v, cons
   if (workspace_bytes < need || (need > 0 && workspace == nullptr))
     return fail(GDN_ERR_WORKSPACE, "chunk_prefill: workspace %zu bytes < %zu needed", workspace_bytes, need);
   if (T == 0 && final_state == nullptr) return ok();
-  if (use_tensor_core_prefill(dt, dk, Hk, Hv)) {
+  if (use_tensor_core_prefill(dt, dk, Hk, Hv, qk_l2norm)) {
     if (!aligned16(workspace) || ((uintptr_t)workspace & 255u) != 0)
       return fail(GDN_ERR_INVALID_ARG, "chunk_prefill: workspace must be 256-byte aligned");
     return cuda_status(gdn::launch_prefill_chunk_tc(q, k, v, g, beta, o, T, Hk, Hv, qk_stride, v_stride,

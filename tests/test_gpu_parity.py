@@ -143,6 +143,27 @@ def test_prefill_bf16_varlen_with_state(cuda_device):
     np.testing.assert_array_equal(np64(cs), cs_ref)
 
 
+def test_prefill_bf16_d128_without_l2norm(cuda_device):
+    """bf16 heads of 128 with q and k used as given (qk_l2norm = 0): the shape the
+    tensor-core path serves, but with the flag off, against the oracle without the norm.
+    Keys are drawn at norm ~1 so the un-normalised delta rule stays bounded."""
+    sh = W.LayerShape(2, 4, 128, 128)
+    r = W.make_recurrence(sh, 200, seed=48, dtype=torch.float32, init_std=0.02)
+    q = (r.q / np.sqrt(sh.dk)).to(torch.bfloat16)
+    k = (r.k / np.sqrt(sh.dk)).to(torch.bfloat16)
+    v = r.v.to(torch.bfloat16)
+    fin = torch.empty((1, sh.Hv, sh.dv, sh.dk), dtype=torch.float32, device=cuda_device)
+    o = gdn.gdn_chunk_prefill(q.to(cuda_device), k.to(cuda_device), v.to(cuda_device),
+                              r.g.to(cuda_device), r.beta.to(cuda_device), None,
+                              r.initial_state.to(cuda_device), fin, 1.0, False)
+    torch.cuda.synchronize()
+    o_r, fin_r = oracle.recurrence(q.float().numpy(), k.float().numpy(), v.float().numpy(),
+                                   r.g.numpy(), r.beta.numpy(), initial_state=r.initial_state.numpy(),
+                                   l2norm=False)
+    assert worst_head_o(np64(o), o_r, [0, 200]) <= BF16_TOL
+    assert worst_head_state(np64(fin), fin_r) <= BF16_TOL
+
+
 def test_prefill_final_state_in_place(cuda_device):
     p = W.make_prefill(W.QWEN35_9B, 70, seed=34, init_std=0.02)
     sh = p.shape
