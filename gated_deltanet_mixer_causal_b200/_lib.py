@@ -31,6 +31,9 @@ SIGNATURES = {
     "gdn_chunk_prefill": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int, _I64, _I32, _I32,
                                           _I32, _I32, _I64, _I64, _P, _I32, _P, _P, _F32, _I32,
                                           _P, _SZ, _P]),
+    "gdn_chunk_prefill_ex": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int, _I64, _I32, _I32,
+                                             _I32, _I32, _I64, _I64, _P, _I32, _P, _P, _F32, _I32,
+                                             _I32, _P, _P, _I64, _P, _SZ, _P]),
     "gdn_decode_step": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _I32, _I32,
                                         _I32, _I32, _I32, _F32, _P]),
     "gdn_decode_tokens": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _I32, _I32, _I32,
@@ -152,11 +155,15 @@ def gdn_chunk_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torc
                       initial_state: Optional[torch.Tensor] = None,
                       final_state: Optional[torch.Tensor] = None, scale: float = 1.0,
                       qk_l2norm: bool = True, o: Optional[torch.Tensor] = None,
-                      workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+                      workspace: Optional[torch.Tensor] = None, block_tokens: int = 0,
+                      block_states: Optional[torch.Tensor] = None,
+                      block_rows: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Gated delta rule over packed sequences (see include/gdn.h). Returns o [T, Hv, dv].
 
     q, k: [T, Hk, dk] and v: [T, Hv, dv] may be token-strided views (e.g. of the conv
-    output). ``final_state`` (fp32 [N, Hv, dv, dk]) is written when given.
+    output). ``final_state`` (fp32 [N, Hv, dv, dk]) is written when given. With
+    ``block_tokens`` > 0 (a multiple of 64) the state after every block_tokens tokens of
+    sequence n goes to ``block_states`` (fp32 [R, Hv, dv, dk]) rows block_rows[n], +1, ...
     """
     T, Hk, dk = q.shape
     _, Hv, dv = v.shape
@@ -179,10 +186,21 @@ def gdn_chunk_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torc
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib().gdn_chunk_prefill(
+    n_rows = 0
+    if block_tokens:
+        if block_states is None or block_rows is None:
+            raise ValueError("block_tokens needs block_states and block_rows")
+        _need(block_states, "block_states", dtype=torch.float32, device=dev)
+        if tuple(block_states.shape[1:]) != (Hv, dv, dk):
+            raise ValueError(f"block_states has shape {tuple(block_states.shape)}, expected [R, {Hv}, {dv}, {dk}]")
+        _need(block_rows, "block_rows", (n_seq,), torch.int32, dev)
+        n_rows = block_states.shape[0]
+    _check(lib().gdn_chunk_prefill_ex(
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(o), _dtype_code(q), T, Hk, Hv, dk, dv,
         qs, vs, _ptr(cu_seqlens), n_seq, _ptr(initial_state), _ptr(final_state), float(scale),
-        int(bool(qk_l2norm)), _ptr(workspace), ws_bytes, _stream(dev)), "gdn_chunk_prefill")
+        int(bool(qk_l2norm)), int(block_tokens), _ptr(block_states if block_tokens else None),
+        _ptr(block_rows if block_tokens else None), n_rows, _ptr(workspace), ws_bytes,
+        _stream(dev)), "gdn_chunk_prefill")
     return o
 
 

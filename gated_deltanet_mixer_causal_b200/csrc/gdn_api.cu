@@ -114,13 +114,14 @@ size_t gdn_chunk_prefill_workspace_size(int64_t T, int32_t n_seq, int32_t Hk, in
   return use_tensor_core_prefill(dt, dk, Hk, Hv) ? gdn::prefill_chunk_tc_workspace(T, n_seq, Hv) : 0;
 }
 
-gdn_status_t gdn_chunk_prefill(const void* q, const void* k, const void* v, const float* g,
-                               const float* beta, void* o, gdn_dtype_t dt, int64_t T,
-                               int32_t Hk, int32_t Hv, int32_t dk, int32_t dv, int64_t qk_stride,
-                               int64_t v_stride, const int32_t* cu_seqlens, int32_t n_seq,
-                               const float* initial_state, float* final_state, float scale,
-                               int32_t qk_l2norm, void* workspace, size_t workspace_bytes,
-                               gdn_stream_t stream) {
+gdn_status_t gdn_chunk_prefill_ex(const void* q, const void* k, const void* v, const float* g,
+                                  const float* beta, void* o, gdn_dtype_t dt, int64_t T,
+                                  int32_t Hk, int32_t Hv, int32_t dk, int32_t dv, int64_t qk_stride,
+                                  int64_t v_stride, const int32_t* cu_seqlens, int32_t n_seq,
+                                  const float* initial_state, float* final_state, float scale,
+                                  int32_t qk_l2norm, int32_t block_tokens, float* block_states,
+                                  const int32_t* block_rows, int64_t n_block_rows, void* workspace,
+                                  size_t workspace_bytes, gdn_stream_t stream) {
   if (!valid_dtype(dt)) return fail(GDN_ERR_UNSUPPORTED, "chunk_prefill: unknown dtype %d", (int)dt);
   if (T < 0) return fail(GDN_ERR_INVALID_ARG, "chunk_prefill: T = %lld < 0", (long long)T);
   if (Hk <= 0 || Hv <= 0) return fail(GDN_ERR_INVALID_ARG, "chunk_prefill: Hk, Hv must be > 0");
@@ -151,6 +152,27 @@ gdn_status_t gdn_chunk_prefill(const void* q, const void* k, const void* v, cons
     return fail(GDN_ERR_INVALID_ARG, "chunk_prefill: o overlaps an input or a state");
   if (final_state != initial_state && overlap(initial_state, stb, final_state, stb))
     return fail(GDN_ERR_INVALID_ARG, "chunk_prefill: final_state partially overlaps initial_state");
+  gdn::BlockStates blocks;
+  if (block_tokens < 0 || block_tokens % 64 != 0)
+    return fail(GDN_ERR_INVALID_ARG, "chunk_prefill: block_tokens = %d must be 0 or a positive multiple of 64",
+                block_tokens);
+  if (block_tokens > 0) {
+    if (!block_states || !block_rows || n_block_rows < 1)
+      return fail(GDN_ERR_INVALID_ARG, "chunk_prefill: block states need block_states, block_rows and n_block_rows >= 1");
+    if (!aligned16(block_states))
+      return fail(GDN_ERR_INVALID_ARG, "chunk_prefill: block_states must be 16-byte aligned");
+    const size_t bsb = (size_t)n_block_rows * Hv * dv * dk * 4;
+    if (overlap(block_states, bsb, q, qkb) || overlap(block_states, bsb, k, qkb) ||
+        overlap(block_states, bsb, v, vb) || overlap(block_states, bsb, g, gb) ||
+        overlap(block_states, bsb, beta, gb) || overlap(block_states, bsb, o, ob) ||
+        overlap(block_states, bsb, initial_state, stb) || overlap(block_states, bsb, final_state, stb) ||
+        overlap(block_states, bsb, block_rows, (size_t)n_seq * 4))
+      return fail(GDN_ERR_INVALID_ARG, "chunk_prefill: block_states overlaps another buffer");
+    blocks.block_tokens = block_tokens;
+    blocks.states = block_states;
+    blocks.rows = block_rows;
+    blocks.n_rows = n_block_rows;
+  }
   const size_t need = gdn_chunk_prefill_workspace_size(T, n_seq, Hk, Hv, dk, dv, dt);
   if (workspace_bytes < need || (need > 0 && workspace == nullptr))
     return fail(GDN_ERR_WORKSPACE, "chunk_prefill: workspace %zu bytes < %zu needed", workspace_bytes, need);
@@ -160,14 +182,26 @@ gdn_status_t gdn_chunk_prefill(const void* q, const void* k, const void* v, cons
       return fail(GDN_ERR_INVALID_ARG, "chunk_prefill: workspace must be 256-byte aligned");
     return cuda_status(gdn::launch_prefill_chunk_tc(q, k, v, g, beta, o, T, Hk, Hv, qk_stride, v_stride,
                                                     cu_seqlens, n_seq, initial_state, final_state,
-                                                    scale, workspace, (cudaStream_t)stream),
+                                                    scale, blocks, workspace, (cudaStream_t)stream),
                        "chunk_prefill (tensor-core) launch");
   }
   return cuda_status(gdn::launch_prefill_recurrent((int)dt, q, k, v, g, beta, o, T, Hk, Hv, dk,
                                                    qk_stride, v_stride, cu_seqlens, n_seq,
                                                    initial_state, final_state, scale, qk_l2norm,
-                                                   (cudaStream_t)stream),
+                                                   blocks, (cudaStream_t)stream),
                      "chunk_prefill launch");
+}
+
+gdn_status_t gdn_chunk_prefill(const void* q, const void* k, const void* v, const float* g,
+                               const float* beta, void* o, gdn_dtype_t dt, int64_t T,
+                               int32_t Hk, int32_t Hv, int32_t dk, int32_t dv, int64_t qk_stride,
+                               int64_t v_stride, const int32_t* cu_seqlens, int32_t n_seq,
+                               const float* initial_state, float* final_state, float scale,
+                               int32_t qk_l2norm, void* workspace, size_t workspace_bytes,
+                               gdn_stream_t stream) {
+  return gdn_chunk_prefill_ex(q, k, v, g, beta, o, dt, T, Hk, Hv, dk, dv, qk_stride, v_stride,
+                              cu_seqlens, n_seq, initial_state, final_state, scale, qk_l2norm, 0,
+                              nullptr, nullptr, 0, workspace, workspace_bytes, stream);
 }
 
 gdn_status_t gdn_decode_step_ex(const void* x, const void* conv_w, void* conv_state, const float* g,

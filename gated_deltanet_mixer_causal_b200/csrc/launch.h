@@ -27,13 +27,24 @@ cudaError_t launch_decode_tokens(int dtype, const void* x, const void* conv_w, v
                                  void* o, int32_t B, int32_t n_tok, int32_t Hk, int32_t Hv, int32_t d,
                                  float scale, cudaStream_t stream);
 
+// States at block boundaries (prefix caching): after every block_tokens tokens of a sequence
+// (block_tokens a positive multiple of 64; 0 = none), its state goes to row
+// block_rows[n] + m - 1 of block_states [n_block_rows, Hv, dv, dk] fp32 for the m-th
+// boundary; rows outside [0, n_block_rows) are skipped.
+struct BlockStates {
+  int32_t block_tokens = 0;
+  float* states = nullptr;
+  const int32_t* rows = nullptr;
+  int64_t n_rows = 0;
+};
+
 // Token-by-token fp32 recurrence (SIMT): the fp32-activation prefill path.
 cudaError_t launch_prefill_recurrent(int dtype, const void* q, const void* k, const void* v,
                                      const float* g, const float* beta, void* o, int64_t T,
                                      int32_t Hk, int32_t Hv, int32_t d, int64_t qk_stride,
                                      int64_t v_stride, const int32_t* cu, int32_t n_seq,
                                      const float* init, float* final_state, float scale,
-                                     int32_t l2norm, cudaStream_t stream);
+                                     int32_t l2norm, BlockStates blocks, cudaStream_t stream);
 
 // Chunked WY/UT prefill on tcgen05 (bf16 activations, dk = dv = 128, at most
 // kPrefillTcMaxG value heads per key head). Needs
@@ -44,6 +55,6 @@ cudaError_t launch_prefill_chunk_tc(const void* q, const void* k, const void* v,
                                     const float* beta, void* o, int64_t T, int32_t Hk, int32_t Hv,
                                     int64_t qk_stride, int64_t v_stride, const int32_t* cu,
                                     int32_t n_seq, const float* init, float* fin, float scale,
-                                    void* workspace, cudaStream_t stream);
+                                    BlockStates blocks, void* workspace, cudaStream_t stream);
 
 }  // namespace gdn

@@ -638,7 +638,7 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
                    const __grid_constant__ CUtensorMap map_wu, const __grid_constant__ CUtensorMap map_mq,
                    const int32_t* __restrict__ cu, int32_t n_seq, int64_t T, int32_t Hk, int32_t Hv,
                    const uint8_t* __restrict__ ws_ro, int* err_word, const float* init, float* fin,
-                   bf16* __restrict__ o, float scale) {
+                   bf16* __restrict__ o, float scale, BlockStates blocks) {
   const Ws L = ws_layout(T, n_seq, Hv);
   const int32_t* prefix = reinterpret_cast<const int32_t*>(ws_ro + L.prefix);
   const int tile = blockIdx.x % NT;
@@ -850,6 +850,15 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
           s[e] = fmaf(decay_last, s[e], __uint_as_float(d0[e]) + __uint_as_float(d1[e]));
         store_state_bf16();
       }
+      // the state after a full chunk that ends a block of the sequence (prefix caching)
+      if (blocks.block_tokens > 0 && len == C && ((int64_t)(c + 1) * C) % blocks.block_tokens == 0) {
+        const int64_t brow = (int64_t)blocks.rows[n] + (int64_t)(c + 1) * C / blocks.block_tokens - 1;
+        if (brow >= 0 && brow < blocks.n_rows) {
+          float* dst = blocks.states + ((brow * Hv + h) * D + tile * DT + half * SJ) * (int64_t)D + lrow;
+#pragma unroll
+          for (int j = 0; j < SJ; ++j) dst[(int64_t)j * D] = s[j];
+        }
+      }
       fence_async_smem();
       tc_fence_before();
       warp_arrive(bar_S);
@@ -937,7 +946,7 @@ cudaError_t launch_prefill_chunk_tc(const void* q, const void* k, const void* v,
                                     const float* beta, void* o, int64_t T, int32_t Hk, int32_t Hv,
                                     int64_t qk_stride, int64_t v_stride, const int32_t* cu,
                                     int32_t n_seq, const float* init, float* fin, float scale,
-                                    void* workspace, cudaStream_t stream) {
+                                    BlockStates blocks, void* workspace, cudaStream_t stream) {
   static uint64_t attrs_set = 0;   // one bit per device that has the smem attributes
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -970,7 +979,7 @@ cudaError_t launch_prefill_chunk_tc(const void* q, const void* k, const void* v,
   dim3 gc((unsigned)((int64_t)n_seq * Hv * NT));
   chunk_chain_kernel<<<gc, kChainThreads, kChainSmem, stream>>>(mq, mk, mwu, mmq, cu, n_seq, T, Hk, Hv, ws,
                                                               reinterpret_cast<int*>(ws + L.err), init, fin,
-                                                              static_cast<bf16*>(o), scale);
+                                                              static_cast<bf16*>(o), scale, blocks);
   return cudaGetLastError();
 }
 

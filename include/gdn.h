@@ -141,6 +141,34 @@ gdn_status_t gdn_chunk_prefill(const void* q, const void* k, const void* v,
                                void* workspace, size_t workspace_bytes, gdn_stream_t stream);
 
 /*
+ * gdn_chunk_prefill_ex -- gdn_chunk_prefill that also stores each sequence's state at block
+ * boundaries, for prefix caching (a block's cached state lets a later request that shares
+ * the prefix resume from it; the state after token t is the S_t of the Qwen3.5 page,
+ * section 5).
+ *
+ * block_tokens  0: no block states (the other three block arguments are ignored); else a
+ *               positive multiple of 64 (the chunk length, so boundaries fall on chunk ends).
+ * block_states  fp32 [n_block_rows, Hv, dv, dk], 16-byte aligned: after the first
+ *               m * block_tokens tokens of sequence n (m >= 1, m * block_tokens <= its
+ *               length) its state is written to row block_rows[n] + m - 1. A sequence whose
+ *               length is a multiple of block_tokens also gets its final state there.
+ * block_rows    int32 [n_seq] device array: the first row of each sequence. Rows outside
+ *               [0, n_block_rows) are skipped, not an error.
+ * Other arguments and return codes as gdn_chunk_prefill; GDN_ERR_INVALID_ARG also for a
+ * bad block_tokens, missing block buffers or block_states overlapping another buffer.
+ */
+gdn_status_t gdn_chunk_prefill_ex(const void* q, const void* k, const void* v,
+                                  const float* g, const float* beta, void* o,
+                                  gdn_dtype_t dt, int64_t T, int32_t Hk, int32_t Hv,
+                                  int32_t dk, int32_t dv, int64_t qk_stride, int64_t v_stride,
+                                  const int32_t* cu_seqlens, int32_t n_seq,
+                                  const float* initial_state, float* final_state,
+                                  float scale, int32_t qk_l2norm, int32_t block_tokens,
+                                  float* block_states, const int32_t* block_rows,
+                                  int64_t n_block_rows, void* workspace, size_t workspace_bytes,
+                                  gdn_stream_t stream);
+
+/*
  * gdn_chunk_prefill_noalloc -- gdn_chunk_prefill for callers that cannot allocate.
  *
  * The pages have no counterpart to this call; it is a convenience of this library.

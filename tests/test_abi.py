@@ -169,6 +169,24 @@ def test_decode_state_dtype_validation(L):
                                   2, 4, 32, 32, 1.0, None) == _lib.GDN_ERR_UNSUPPORTED
 
 
+def test_prefill_block_state_validation(L):
+    def call(bt, bs, br, nr, **kw):
+        a = dict(q=FAKE, k=FAKE + 256, v=FAKE + (1 << 30), g=FAKE + (2 << 30), b=FAKE + (3 << 30),
+                 o=FAKE + (4 << 30), fin=FAKE + (5 << 30))
+        a.update(kw)
+        return L.gdn_chunk_prefill_ex(a["q"], a["k"], a["v"], a["g"], a["b"], a["o"], 0, 128, 2,
+                                      4, 32, 32, 128, 128, None, 1, None, a["fin"], 1.0, 1, bt, bs,
+                                      br, nr, None, 0, None)
+    rows = FAKE + (7 << 30)
+    assert call(-64, FAKE + (6 << 30), rows, 4) == _lib.GDN_ERR_INVALID_ARG
+    assert call(96, FAKE + (6 << 30), rows, 4) == _lib.GDN_ERR_INVALID_ARG      # not a multiple of 64
+    assert call(64, None, rows, 4) == _lib.GDN_ERR_INVALID_ARG
+    assert call(64, FAKE + (6 << 30), None, 4) == _lib.GDN_ERR_INVALID_ARG
+    assert call(64, FAKE + (6 << 30), rows, 0) == _lib.GDN_ERR_INVALID_ARG
+    assert call(64, FAKE + (6 << 30) + 8, rows, 4) == _lib.GDN_ERR_INVALID_ARG  # misaligned
+    assert call(64, FAKE + (5 << 30) + 4096, rows, 4) == _lib.GDN_ERR_INVALID_ARG  # inside final_state
+
+
 def test_python_binding_refuses_cpu_tensors():
     import torch
     x = torch.zeros(8, 64, dtype=torch.bfloat16)

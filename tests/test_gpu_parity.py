@@ -425,3 +425,68 @@ def test_decode_tokens_bf16_state_27b(cuda_device, n_tok):
             assert frob_rel(o_g[j, :, h], o_r[j, :, h]) <= BF16_TOL, (j, h)
             assert frob_rel(st_g[j, h], st_r[j, h]) <= BF16_TOL, (j, h)
     np.testing.assert_array_equal(np64(cs), cs_r)
+
+
+# ------------------------------------------------------- states at block boundaries
+
+def _block_state_reference(r, lengths, block, rows, n_rows, l2norm=True):
+    """Oracle state after each block of each sequence: the recurrence over that prefix."""
+    ref = {}
+    cu = np.concatenate([[0], np.cumsum(lengths)])
+    for n, L in enumerate(lengths):
+        for m in range(1, L // block + 1):
+            row = rows[n] + m - 1
+            if not 0 <= row < n_rows:
+                continue
+            a, b = cu[n], cu[n] + m * block
+            _, fin = oracle.recurrence(r.q[a:b].float().numpy(), r.k[a:b].float().numpy(),
+                                       r.v[a:b].float().numpy(), r.g[a:b].numpy(), r.beta[a:b].numpy(),
+                                       initial_state=r.initial_state[n:n + 1].numpy(), l2norm=l2norm)
+            ref[row] = fin[0]
+    return ref
+
+
+def _run_with_blocks(r, dev, block, rows, n_rows):
+    sh = r.shape
+    n = r.cu_seqlens.numel() - 1
+    bs = torch.full((n_rows, sh.Hv, sh.dv, sh.dk), float("nan"), dtype=torch.float32, device=dev)
+    fin = torch.empty((n, sh.Hv, sh.dv, sh.dk), dtype=torch.float32, device=dev)
+    args = (r.q.to(dev), r.k.to(dev), r.v.to(dev), r.g.to(dev), r.beta.to(dev), r.cu_seqlens.to(dev),
+            r.initial_state.to(dev))
+    o = gdn.gdn_chunk_prefill(*args, fin, 1.0, True, block_tokens=block, block_states=bs,
+                              block_rows=torch.tensor(rows, dtype=torch.int32, device=dev))
+    fin0 = torch.empty_like(fin)
+    o0 = gdn.gdn_chunk_prefill(*args, fin0, 1.0, True)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o0) and torch.equal(fin, fin0)   # block states change nothing else
+    return np64(bs)
+
+
+def test_prefill_block_states_bf16(cuda_device):
+    """Tensor-core path (bf16, heads of 128): block states of four packed sequences, one of
+    them shorter than a block and one a multiple of the block, against oracle prefixes."""
+    lengths, block = [300, 128, 1000, 64], 128
+    r = W.make_recurrence(W.LayerShape(2, 4, 128, 128), 0, seed=49, dtype=torch.bfloat16,
+                          init_std=0.02, lengths=lengths)
+    rows = [0, 2, 3, 10]
+    got = _run_with_blocks(r, cuda_device, block, rows, 10)
+    ref = _block_state_reference(r, lengths, block, rows, 10)
+    assert sorted(ref) == list(range(10))
+    for row, s_ref in ref.items():
+        for h in range(4):
+            assert frob_rel(got[row, h], s_ref[h]) <= BF16_TOL, (row, h)
+
+
+def test_prefill_block_states_fp32_rows_out_of_range(cuda_device):
+    """Token-recurrent path (fp32): block states against oracle prefixes; rows past the end
+    of block_states are skipped and the buffer's other rows stay untouched."""
+    lengths, block = [150, 64, 200], 64
+    r = W.make_recurrence(W.LayerShape(2, 2, 16, 16), 0, seed=50, dtype=torch.float32,
+                          init_std=0.1, lengths=lengths)
+    rows, n_rows = [0, 3, 4], 6        # sequence 2's third boundary would be row 6: skipped;
+    got = _run_with_blocks(r, cuda_device, block, rows, n_rows)   # row 2 is never written
+    ref = _block_state_reference(r, lengths, block, rows, n_rows)
+    assert sorted(ref) == [0, 1, 3, 4, 5]
+    for row, s_ref in ref.items():
+        assert max_rel(got[row], s_ref) <= FP32_TOL, row
+    assert np.isnan(got[2]).all()
