@@ -4,10 +4,11 @@ The compute runs in ``libgdn.so`` (hand-written CUDA, C ABI in ``include/gdn.h``
 package marshals torch tensors into it. The library is loaded on first use and a missing
 library raises -- there is no fallback.
 
-Entry points (same names as the C ABI): ``gdn_conv1d_silu``, ``gdn_chunk_prefill``,
-``gdn_chunk_prefill_workspace_size``, ``gdn_chunk_prefill_noalloc``, ``gdn_decode_step``,
-``gdn_decode_tokens``; ``prefill_layer`` chains the
-conv and the chunked prefill over one packed batch without copies.
+Entry points (same names as the C ABI): ``gdn_conv1d_silu``, ``gdn_chunk_prefill`` (states at
+block boundaries on request), ``gdn_chunk_prefill_workspace_size``,
+``gdn_chunk_prefill_noalloc``, ``gdn_decode_step`` and ``gdn_decode_tokens`` (fp32 or bf16
+states, taken from the state tensor); ``prefill_layer`` chains the conv and the chunked
+prefill over one packed batch without copies.
 """
 from __future__ import annotations
 

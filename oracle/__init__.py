@@ -13,6 +13,11 @@ stabilisers, alpha/beta per token and per head) and the config footnote (16 K / 
 heads x 128, conv kernel 4, fp32 state); "Hybrid Mamba-Transformer MoE"
 (sotaaz.com), section "Gated DeltaNet" (the ungated DeltaNet update).
 
+Decode entry points are prefills: ``decode_step`` of B sequences of one token,
+``decode_tokens`` of B sequences of n tokens, from the carried conv taps and states. A state
+stored in bf16 between calls (a serving option; the pages' model keeps fp32 states) is
+modelled by rounding the fp64 result with ``round_bf16`` once per call.
+
 Every function here is pinned by tests in ``tests/test_oracle_pins.py``.
 """
 from __future__ import annotations
