@@ -1,0 +1,92 @@
+"""Context-parallel prefill of one sequence split across ranks: the exchange and the fold
+run as gloo ranks on the CPU with the oracle as the per-segment prefill (exact in fp64); on
+one GPU the same pieces run with the library's prefill, segment by segment."""
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+sys.path.insert(0, os.path.join(ROOT, "tests"))
+
+from gated_deltanet_mixer_causal_b200 import context_parallel as cp  # noqa: E402
+from gated_deltanet_mixer_causal_b200 import workloads as W  # noqa: E402
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _oracle_prefill(q, k, v, g, beta, initial_state):
+    import oracle
+    o, fin = oracle.recurrence(q.double().numpy(), k.double().numpy(), v.double().numpy(),
+                               g.double().numpy(), beta.double().numpy(),
+                               initial_state=initial_state.double().numpy(), l2norm=True)
+    return torch.from_numpy(o), torch.from_numpy(fin)
+
+
+def _sequence(T, seed):
+    return W.make_recurrence(W.LayerShape(2, 4, 8, 8), T, seed=seed, dtype=torch.float32,
+                             init_std=0.1)
+
+
+def _worker(rank, world, port, lengths, seed, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        r = _sequence(sum(lengths), seed)
+        a = sum(lengths[:rank]); b = a + lengths[rank]
+        o, fin = cp.cp_prefill(r.q[a:b], r.k[a:b], r.v[a:b], r.g[a:b], r.beta[a:b],
+                               initial_state=r.initial_state, prefill=_oracle_prefill)
+        out[rank] = (o.numpy(), fin.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("lengths", [[40, 57], [33, 1, 70]])
+def test_cp_prefill_gloo_equals_one_run(oracle_mod, lengths):
+    world, seed = len(lengths), 51 + len(lengths)
+    out = mp.get_context("spawn").Manager().dict()
+    mp.spawn(_worker, args=(world, _free_port(), lengths, seed, out), nprocs=world, join=True)
+    r = _sequence(sum(lengths), seed)
+    o_ref, fin_ref = _oracle_prefill(r.q, r.k, r.v, r.g, r.beta, r.initial_state)
+    o = np.concatenate([out[i][0] for i in range(world)])
+    np.testing.assert_allclose(o, o_ref.numpy(), rtol=1e-10, atol=1e-12)
+    for i in range(world):
+        np.testing.assert_allclose(out[i][1], fin_ref.numpy(), rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_cp_pieces_on_gpu(cuda_device, dtype):
+    """Two segments on one GPU (summaries, fold, second pass) against one prefill of the
+    whole sequence: fp32 (token-recurrent path) at 1e-4, bf16 heads of 128 (tensor-core
+    path) at the bf16 tolerance."""
+    from parity import BF16_TOL, FP32_TOL, frob_rel, max_rel, np64
+    r = W.make_recurrence(W.LayerShape(2, 4, 128, 128), 700, seed=53, dtype=dtype, init_std=0.02)
+    dev = cuda_device
+    q, k, v, g, b = (t.to(dev) for t in (r.q, r.k, r.v, r.g, r.beta))
+    s0 = r.initial_state.to(dev)
+    prefill = cp._library_prefill(1.0, True)
+    cuts = [(0, 300), (300, 700)]
+    sums = [cp.segment_summary(q[a:e], k[a:e], v[a:e], g[a:e], b[a:e], prefill) for a, e in cuts]
+    states = cp.fold(sums, s0)
+    o_cp = torch.cat([prefill(q[a:e], k[a:e], v[a:e], g[a:e], b[a:e], states[i].contiguous())[0]
+                      for i, (a, e) in enumerate(cuts)])
+    o_one, fin_one = prefill(q, k, v, g, b, s0)
+    torch.cuda.synchronize()
+    if dtype == torch.float32:
+        assert max_rel(np64(o_cp), np64(o_one)) <= FP32_TOL
+        assert max_rel(np64(states[-1]), np64(fin_one)) <= FP32_TOL
+    else:
+        for h in range(4):
+            assert frob_rel(np64(o_cp)[:, h], np64(o_one)[:, h]) <= BF16_TOL, h
+            assert frob_rel(np64(states[-1])[0, h], np64(fin_one)[0, h]) <= BF16_TOL, h
