@@ -34,6 +34,8 @@ SIGNATURES = {
     "gdn_chunk_prefill_ex": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int, _I64, _I32, _I32,
                                              _I32, _I32, _I64, _I64, _P, _I32, _P, _P, _F32, _I32,
                                              _I32, _P, _P, _I64, _P, _SZ, _P]),
+    "gdn_prefill_status": (ctypes.c_int, [_P, _P]),
+    "gdn_prefill_noalloc_status": (ctypes.c_int, [_P]),
     "gdn_decode_step": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _I32, _I32,
                                         _I32, _I32, _I32, _F32, _P]),
     "gdn_decode_tokens": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _I32, _I32, _I32,
@@ -157,13 +159,14 @@ def gdn_chunk_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torc
                       qk_l2norm: bool = True, o: Optional[torch.Tensor] = None,
                       workspace: Optional[torch.Tensor] = None, block_tokens: int = 0,
                       block_states: Optional[torch.Tensor] = None,
-                      block_rows: Optional[torch.Tensor] = None) -> torch.Tensor:
+                      block_rows: Optional[torch.Tensor] = None, check: bool = False) -> torch.Tensor:
     """Gated delta rule over packed sequences (see include/gdn.h). Returns o [T, Hv, dv].
 
     q, k: [T, Hk, dk] and v: [T, Hv, dv] may be token-strided views (e.g. of the conv
     output). ``final_state`` (fp32 [N, Hv, dv, dk]) is written when given. With
     ``block_tokens`` > 0 (a multiple of 64) the state after every block_tokens tokens of
     sequence n goes to ``block_states`` (fp32 [R, Hv, dv, dk]) rows block_rows[n], +1, ...
+    ``check``: wait for the call and raise GDNError if a bounded device-side wait gave up.
     """
     T, Hk, dk = q.shape
     _, Hv, dv = v.shape
@@ -201,7 +204,22 @@ def gdn_chunk_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torc
         int(bool(qk_l2norm)), int(block_tokens), _ptr(block_states if block_tokens else None),
         _ptr(block_rows if block_tokens else None), n_rows, _ptr(workspace), ws_bytes,
         _stream(dev)), "gdn_chunk_prefill")
+    if check and workspace is not None:
+        gdn_prefill_status(workspace)
     return o
+
+
+def gdn_prefill_status(workspace: torch.Tensor) -> None:
+    """Wait for the last prefill that used ``workspace`` and raise GDNError(GDN_ERR_TIMEOUT)
+    if one of its bounded device-side waits gave up (its outputs are then invalid)."""
+    _check(lib().gdn_prefill_status(_ptr(workspace), _stream(workspace.device)), "gdn_prefill_status")
+
+
+def gdn_prefill_noalloc_status(device: Optional[torch.device] = None) -> None:
+    """gdn_prefill_status for gdn_chunk_prefill_noalloc's static scratch on ``device``."""
+    dev = device or torch.device("cuda", torch.cuda.current_device())
+    with torch.cuda.device(dev):
+        _check(lib().gdn_prefill_noalloc_status(_stream(dev)), "gdn_prefill_noalloc_status")
 
 
 def gdn_chunk_prefill_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,

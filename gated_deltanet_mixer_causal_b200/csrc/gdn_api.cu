@@ -185,11 +185,27 @@ gdn_status_t gdn_chunk_prefill_ex(const void* q, const void* k, const void* v, c
                                                     scale, blocks, workspace, (cudaStream_t)stream),
                        "chunk_prefill (tensor-core) launch");
   }
+  if (workspace != nullptr && workspace_bytes >= sizeof(int)) {   // no wait can fail here
+    const cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(int), (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_status(e, "chunk_prefill: clearing the status word");
+  }
   return cuda_status(gdn::launch_prefill_recurrent((int)dt, q, k, v, g, beta, o, T, Hk, Hv, dk,
                                                    qk_stride, v_stride, cu_seqlens, n_seq,
                                                    initial_state, final_state, scale, qk_l2norm,
                                                    blocks, (cudaStream_t)stream),
                      "chunk_prefill launch");
+}
+
+gdn_status_t gdn_prefill_status(const void* workspace, gdn_stream_t stream) {
+  if (workspace == nullptr) return fail(GDN_ERR_INVALID_ARG, "prefill_status: workspace is NULL");
+  int word = 0;
+  cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost,
+                                  (cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_status(e, "prefill_status");
+  if (word == 0) return ok();
+  return fail(GDN_ERR_TIMEOUT, "prefill_status: a bounded device-side wait gave up (%s, code %d); "
+              "the outputs of that call are invalid", gdn::prefill_chunk_tc_error_string(word), word);
 }
 
 gdn_status_t gdn_chunk_prefill(const void* q, const void* k, const void* v, const float* g,

@@ -938,6 +938,16 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, ui
 
 }  // namespace
 
+const char* prefill_chunk_tc_error_string(int code) {
+  switch (code) {
+    case kErrIntraTma: return "intra-chunk kernel: a TMA load did not land";
+    case kErrIntraMma: return "intra-chunk kernel: an MMA did not complete";
+    case kErrChainTma: return "chain kernel: a TMA load did not land";
+    case kErrChainMma: return "chain kernel: an MMA or a warp handoff did not complete";
+    default: return "unknown wait";
+  }
+}
+
 size_t prefill_chunk_tc_workspace(int64_t T, int32_t n_seq, int32_t Hv) {
   return ws_layout(T, n_seq, Hv).total;
 }

@@ -72,3 +72,9 @@ extern "C" gdn_status_t gdn_chunk_prefill_noalloc(
                            cu_seqlens, n_seq, initial_state, final_state, scale, qk_l2norm,
                            scratch, kNoallocScratchBytes, stream);
 }
+
+extern "C" gdn_status_t gdn_prefill_noalloc_status(gdn_stream_t stream) {
+  void* scratch = nullptr;
+  if (scratch_for_current_device(&scratch) != cudaSuccess) return GDN_ERR_CUDA;
+  return gdn_prefill_status(scratch, stream);
+}

@@ -48,7 +48,7 @@ typedef enum {
   GDN_ERR_UNSUPPORTED = 2,   /* valid but not built: head size, dtype, Hv % Hk != 0 */
   GDN_ERR_WORKSPACE = 3,     /* workspace too small (see the *_workspace_size query) */
   GDN_ERR_CUDA = 4,          /* a CUDA launch or runtime call failed */
-  GDN_ERR_TIMEOUT = 5        /* reserved: a bounded device-side wait gave up */
+  GDN_ERR_TIMEOUT = 5        /* a bounded device-side wait gave up (gdn_prefill_status) */
 } gdn_status_t;
 
 typedef enum {
@@ -139,6 +139,20 @@ gdn_status_t gdn_chunk_prefill(const void* q, const void* k, const void* v,
                                const float* initial_state, float* final_state,
                                float scale, int32_t qk_l2norm,
                                void* workspace, size_t workspace_bytes, gdn_stream_t stream);
+
+/*
+ * gdn_prefill_status -- whether the last gdn_chunk_prefill / gdn_chunk_prefill_ex that used
+ * this workspace completed its device-side waits. The tensor-core kernels bound every wait
+ * (for a TMA load or an MMA) and, when one gives up, record a code in the workspace's first
+ * int and return early instead of hanging; the call itself has already returned GDN_OK.
+ * This waits for the work queued on `stream`, reads that word and returns GDN_OK, or
+ * GDN_ERR_TIMEOUT (the outputs of that call are invalid; gdn_last_error() names the kernel
+ * and the wait), GDN_ERR_INVALID_ARG for a NULL workspace, GDN_ERR_CUDA if the read fails.
+ * gdn_prefill_noalloc_status is the same for gdn_chunk_prefill_noalloc's static scratch on
+ * the current device.
+ */
+gdn_status_t gdn_prefill_status(const void* workspace, gdn_stream_t stream);
+gdn_status_t gdn_prefill_noalloc_status(gdn_stream_t stream);
 
 /*
  * gdn_chunk_prefill_ex -- gdn_chunk_prefill that also stores each sequence's state at block

@@ -187,6 +187,10 @@ def test_prefill_block_state_validation(L):
     assert call(64, FAKE + (5 << 30) + 4096, rows, 4) == _lib.GDN_ERR_INVALID_ARG  # inside final_state
 
 
+def test_prefill_status_needs_a_workspace(L):
+    assert L.gdn_prefill_status(None, None) == _lib.GDN_ERR_INVALID_ARG
+
+
 def test_python_binding_refuses_cpu_tensors():
     import torch
     x = torch.zeros(8, 64, dtype=torch.bfloat16)

@@ -164,6 +164,21 @@ def test_prefill_bf16_d128_without_l2norm(cuda_device):
     assert worst_head_state(np64(fin), fin_r) <= BF16_TOL
 
 
+def test_prefill_status_after_a_call(cuda_device):
+    """The status word of a completed tensor-core prefill reads OK, also through check=True;
+    a recurrent-path call that was handed a workspace leaves it cleared."""
+    sh = W.LayerShape(2, 4, 128, 128)
+    r = W.make_recurrence(sh, 300, seed=54, dtype=torch.bfloat16)
+    args = [t.to(cuda_device) for t in (r.q, r.k, r.v, r.g, r.beta)]
+    need = gdn.gdn_chunk_prefill_workspace_size(300, 1, sh.Hk, sh.Hv, sh.dk, sh.dv, torch.bfloat16)
+    ws = torch.full((need,), 0xFF, dtype=torch.uint8, device=cuda_device)   # garbage on entry
+    gdn.gdn_chunk_prefill(*args, workspace=ws, check=True)
+    gdn.gdn_prefill_status(ws)
+    ws.fill_(0xFF)
+    gdn.gdn_chunk_prefill(*args, qk_l2norm=False, workspace=ws)   # token-recurrent path
+    gdn.gdn_prefill_status(ws)
+
+
 def test_prefill_final_state_in_place(cuda_device):
     p = W.make_prefill(W.QWEN35_9B, 70, seed=34, init_std=0.02)
     sh = p.shape

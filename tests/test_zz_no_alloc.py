@@ -48,6 +48,7 @@ def test_noalloc_matches_workspace_entry_point(cuda_device):
         fin = torch.full_like(init, float("nan"))
         o = torch.full((p.T, sh.Hv, sh.dv), float("nan"), dtype=q.dtype, device=dev)
         gdn.gdn_chunk_prefill_noalloc(q, k, v, g, beta, cu, init, fin, o=o)
+        gdn.gdn_prefill_noalloc_status(dev)   # every bounded wait of the call completed
         torch.cuda.synchronize()
         cu_np = p.cu_seqlens.numpy()
         assert worst_head_o(np64(o), np64(o_ref), cu_np) <= BF16_TOL
