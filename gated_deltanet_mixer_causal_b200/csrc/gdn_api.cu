@@ -50,6 +50,13 @@ bool supported_head_dim(int32_t d) { return d == 16 || d == 32 || d == 64 || d =
 
 // bf16 activations with 128-wide heads (and at most 8 value heads per key head) run the
 // chunked tensor-core prefill; everything else runs the token-by-token fp32 kernel.
+// TMA coordinates are 32-bit: the tensor-core prefill addresses tokens and workspace rows
+// (chunk slot x value head x 128) with int32, which bounds the tokens of one call.
+bool tc_rows_fit(int64_t T, int32_t n_seq, int32_t Hv) {
+  const int64_t slots = (T + 63) / 64 + (n_seq < 1 ? 1 : n_seq);
+  return T <= 0x7fffffffLL && slots * Hv * 128 <= 0x7fffffffLL;
+}
+
 // The tensor-core prefill folds the q/k L2 norm into its factors; inputs used as given
 // (qk_l2norm = 0) take the token-recurrent path.
 bool use_tensor_core_prefill(gdn_dtype_t dt, int32_t d, int32_t Hk, int32_t Hv, int32_t qk_l2norm = 1) {
@@ -111,7 +118,8 @@ size_t gdn_chunk_prefill_workspace_size(int64_t T, int32_t n_seq, int32_t Hk, in
       !supported_head_dim(dk))
     return SIZE_MAX;
   if (n_seq < 1) n_seq = 1;
-  return use_tensor_core_prefill(dt, dk, Hk, Hv) ? gdn::prefill_chunk_tc_workspace(T, n_seq, Hv) : 0;
+  if (!use_tensor_core_prefill(dt, dk, Hk, Hv)) return 0;
+  return tc_rows_fit(T, n_seq, Hv) ? gdn::prefill_chunk_tc_workspace(T, n_seq, Hv) : SIZE_MAX;
 }
 
 gdn_status_t gdn_chunk_prefill_ex(const void* q, const void* k, const void* v, const float* g,
@@ -173,11 +181,15 @@ gdn_status_t gdn_chunk_prefill_ex(const void* q, const void* k, const void* v, c
     blocks.rows = block_rows;
     blocks.n_rows = n_block_rows;
   }
-  const size_t need = gdn_chunk_prefill_workspace_size(T, n_seq, Hk, Hv, dk, dv, dt);
+  const bool tensor_core = use_tensor_core_prefill(dt, dk, Hk, Hv, qk_l2norm);
+  if (tensor_core && !tc_rows_fit(T, n_seq, Hv))
+    return fail(GDN_ERR_UNSUPPORTED, "chunk_prefill: %lld tokens of %d value heads exceed the 32-bit "
+                "TMA coordinates of one call; split the batch", (long long)T, Hv);
+  const size_t need = tensor_core ? gdn::prefill_chunk_tc_workspace(T, n_seq, Hv) : 0;
   if (workspace_bytes < need || (need > 0 && workspace == nullptr))
     return fail(GDN_ERR_WORKSPACE, "chunk_prefill: workspace %zu bytes < %zu needed", workspace_bytes, need);
   if (T == 0 && final_state == nullptr) return ok();
-  if (use_tensor_core_prefill(dt, dk, Hk, Hv, qk_l2norm)) {
+  if (tensor_core) {
     if (!aligned16(workspace) || ((uintptr_t)workspace & 255u) != 0)
       return fail(GDN_ERR_INVALID_ARG, "chunk_prefill: workspace must be 256-byte aligned");
     return cuda_status(gdn::launch_prefill_chunk_tc(q, k, v, g, beta, o, T, Hk, Hv, qk_stride, v_stride,

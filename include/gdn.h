@@ -98,7 +98,9 @@ gdn_status_t gdn_conv1d_silu(const void* x, void* y, gdn_dtype_t dt, const void*
 /*
  * gdn_chunk_prefill_workspace_size -- bytes of device workspace gdn_chunk_prefill needs
  * for these sizes (0 is a valid answer); an upper bound, since calls with qk_l2norm = 0
- * need none. Returns SIZE_MAX for unsupported shapes.
+ * need none. Returns SIZE_MAX for unsupported shapes, including bf16 heads of 128 whose
+ * chunk rows (about T / 64 x Hv x 128) pass 2^31 - 1: the tensor-core path addresses them
+ * with 32-bit TMA coordinates, so such a batch is split into several calls.
  */
 size_t gdn_chunk_prefill_workspace_size(int64_t T, int32_t n_seq, int32_t Hk, int32_t Hv,
                                         int32_t dk, int32_t dv, gdn_dtype_t dt);

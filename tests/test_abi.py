@@ -187,6 +187,20 @@ def test_prefill_block_state_validation(L):
     assert call(64, FAKE + (5 << 30) + 4096, rows, 4) == _lib.GDN_ERR_INVALID_ARG  # inside final_state
 
 
+def test_prefill_beyond_32bit_coordinates_is_refused(L):
+    """bf16 heads of 128: the tensor-core path's rows are int32 TMA coordinates, so a batch
+    whose chunk rows pass 2^31 is unsupported (and says so before any launch); the same size
+    with the norm off takes the token-recurrent path, which needs no workspace."""
+    T, Hk, Hv, d = 30_000_000, 16, 48, 128
+    assert L.gdn_chunk_prefill_workspace_size(T, 1, Hk, Hv, d, d, _lib.GDN_BF16) == 2 ** 64 - 1
+    assert L.gdn_chunk_prefill_workspace_size(1_000_000, 1, Hk, Hv, d, d, _lib.GDN_BF16) < 2 ** 40
+    # q, k, v as views of one conv output (hundreds of GB at this T); g, beta, o far apart
+    st = L.gdn_chunk_prefill(FAKE, FAKE, FAKE, FAKE + (1 << 40), FAKE + (1 << 40) + (1 << 34),
+                             FAKE + (1 << 41), _lib.GDN_BF16, T, Hk, Hv, d, d, 2 * Hk * d + Hv * d,
+                             2 * Hk * d + Hv * d, None, 1, None, None, 1.0, 1, None, 0, None)
+    assert st == _lib.GDN_ERR_UNSUPPORTED and "split the batch" in L.gdn_last_error().decode()
+
+
 def test_prefill_status_needs_a_workspace(L):
     assert L.gdn_prefill_status(None, None) == _lib.GDN_ERR_INVALID_ARG
 
