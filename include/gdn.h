@@ -12,13 +12,15 @@
  *   o_t    = scale * S_t q_t
  *
  * One recurrent state S (dv x dk, fp32, row index = value dimension) exists per sequence
- * and value head. Value head h reads key head h / (Hv / Hk).
+ * and value head; the _ex decode calls can store it in bf16 instead. Value head h reads key
+ * head h / (Hv / Hk).
  *
  * Conventions shared by every entry point
  * ---------------------------------------
  * Pointers: device pointers unless stated; 16-byte aligned; tensors row-major and dense
  *   unless a stride argument says otherwise. The caller owns every buffer, including the
- *   workspace; the library allocates no device memory and keeps no state between calls.
+ *   workspace; the library allocates no device memory and keeps no state between calls
+ *   (except gdn_chunk_prefill_noalloc's static scratch, which it owns for its lifetime).
  * Streams: every call is asynchronous on `stream` (NULL = the legacy default stream) and
  *   returns once its kernels are enqueued. Inputs must stay valid until they complete.
  * Errors: arguments are validated before anything is launched; an invalid call returns a
@@ -45,15 +47,17 @@ typedef struct CUstream_st* gdn_stream_t;
 typedef enum {
   GDN_OK = 0,
   GDN_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, aliasing, bad cu_seqlens */
-  GDN_ERR_UNSUPPORTED = 2,   /* valid but not built: head size, dtype, Hv % Hk != 0 */
+  GDN_ERR_UNSUPPORTED = 2,   /* valid but not built: head size, dtype, Hv % Hk != 0, or a
+                                size beyond a path's limits */
   GDN_ERR_WORKSPACE = 3,     /* workspace too small (see the *_workspace_size query) */
   GDN_ERR_CUDA = 4,          /* a CUDA launch or runtime call failed */
   GDN_ERR_TIMEOUT = 5        /* a bounded device-side wait gave up (gdn_prefill_status) */
 } gdn_status_t;
 
 typedef enum {
-  GDN_F32 = 0,               /* fp32 activations (the state is always fp32) */
-  GDN_BF16 = 1               /* bf16 activations, fp32 math and state */
+  GDN_F32 = 0,               /* fp32 activations; fp32 state */
+  GDN_BF16 = 1               /* bf16 activations, fp32 math and state (as a state_dt of
+                                the _ex decode calls: bf16 state storage, fp32 math) */
 } gdn_dtype_t;
 
 /* Static string naming a status code. Never NULL. */
