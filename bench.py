@@ -87,9 +87,14 @@ class ClockSampler:
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index: int):
+        """Samples go to $GDN_CLOCKS_DIR/clocks_gpu<i>.csv when that is set (to keep them),
+        else to a temporary file."""
+        import tempfile
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+        keep = os.environ.get("GDN_CLOCKS_DIR")
+        self.path = (os.path.join(keep, f"clocks_gpu{gpu_index}.csv") if keep else
+                     os.path.join(tempfile.gettempdir(), f"gdn_clocks_gpu{gpu_index}_{os.getpid()}.csv"))
 
     def start(self):
         try:

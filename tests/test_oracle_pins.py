@@ -175,7 +175,7 @@ def test_brute_force_product_expansion(oracle_mod, d, T):
 
 def test_alpha_one_is_the_deltanet_update(oracle_mod):
     """g = 0 reduces to S_t = S_{t-1} - beta (S_{t-1} k) k^T + beta v k^T (the ungated
-    DeltaNet of the sotaaz survey), checked through the product expansion with alpha=1."""
+    DeltaNet of the sotaaz page), checked through the product expansion with alpha=1."""
     r = rng(9)
     q, k, v, _, beta, S0 = _random_case(r, 6, 1, 1, 3)
     g = np.zeros((6, 1))
