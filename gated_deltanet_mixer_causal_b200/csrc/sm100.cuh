@@ -1,5 +1,5 @@
 // sm100.cuh -- thin inline-PTX wrappers for the sm_100a features the chunked prefill uses:
-// mbarriers, TMA tile loads (no multicast), tcgen05 TMEM allocation, MMA, commit and loads.
+// mbarriers, TMA tile loads into this CTA only, tcgen05 TMEM allocation, MMA, commit and loads.
 //
 // Every wait is bounded: after kSpinLimit polls it gives up, records `code` in the
 // kernel's error word and returns false, so a mis-programmed transfer ends the kernel
@@ -65,7 +65,7 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-// 2D tiled load (no multicast) of the box at coordinates (x, y) into shared memory,
+// 2D tiled load, into this CTA only, of the box at coordinates (x, y) into shared memory,
 // completing `bar`'s transaction count. x * elementsize must be a multiple of 16 bytes.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int32_t x, int32_t y,
                                             uint64_t* bar) {
@@ -85,7 +85,7 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
-// 2D tiled store shared -> global of the box at (x, y) (no multicast); completion is
+// 2D tiled store shared -> global of the box at (x, y) (this CTA only); completion is
 // tracked by the issuing thread's bulk async-group.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int32_t x, int32_t y, const void* src) {
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];"
