@@ -38,26 +38,30 @@ def _sequence(T, seed):
                              init_std=0.1)
 
 
-def _worker(rank, world, port, lengths, seed, out):
+def _worker(rank, world, port, lengths, seed, with_state, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         r = _sequence(sum(lengths), seed)
         a = sum(lengths[:rank]); b = a + lengths[rank]
         o, fin = cp.cp_prefill(r.q[a:b], r.k[a:b], r.v[a:b], r.g[a:b], r.beta[a:b],
-                               initial_state=r.initial_state, prefill=_oracle_prefill)
+                               initial_state=r.initial_state if with_state else None,
+                               prefill=_oracle_prefill)
         out[rank] = (o.numpy(), fin.numpy())
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("lengths", [[40, 57], [33, 1, 70]])
-def test_cp_prefill_gloo_equals_one_run(oracle_mod, lengths):
+@pytest.mark.parametrize("lengths,with_state", [([40, 57], True), ([33, 1, 70], True),
+                                               ([64, 20], False)])
+def test_cp_prefill_gloo_equals_one_run(oracle_mod, lengths, with_state):
     world, seed = len(lengths), 51 + len(lengths)
     out = mp.get_context("spawn").Manager().dict()
-    mp.spawn(_worker, args=(world, _free_port(), lengths, seed, out), nprocs=world, join=True)
+    mp.spawn(_worker, args=(world, _free_port(), lengths, seed, with_state, out), nprocs=world,
+             join=True)
     r = _sequence(sum(lengths), seed)
-    o_ref, fin_ref = _oracle_prefill(r.q, r.k, r.v, r.g, r.beta, r.initial_state)
+    s0 = r.initial_state if with_state else torch.zeros_like(r.initial_state)
+    o_ref, fin_ref = _oracle_prefill(r.q, r.k, r.v, r.g, r.beta, s0)
     o = np.concatenate([out[i][0] for i in range(world)])
     np.testing.assert_allclose(o, o_ref.numpy(), rtol=1e-10, atol=1e-12)
     for i in range(world):
