@@ -53,7 +53,7 @@ def _worker(rank, world, port, lengths, seed, with_state, out):
 
 
 @pytest.mark.parametrize("lengths,with_state", [([40, 57], True), ([33, 1, 70], True),
-                                               ([64, 20], False)])
+                                               ([64, 20], False), ([20, 30, 10, 40], True)])
 def test_cp_prefill_gloo_equals_one_run(oracle_mod, lengths, with_state):
     world, seed = len(lengths), 51 + len(lengths)
     out = mp.get_context("spawn").Manager().dict()
