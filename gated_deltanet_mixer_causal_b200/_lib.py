@@ -32,8 +32,8 @@ SIGNATURES = {
                                           _I32, _I32, _I64, _I64, _P, _I32, _P, _P, _F32, _I32,
                                           _P, _SZ, _P]),
     "gdn_chunk_prefill_ex": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int, _I64, _I32, _I32,
-                                             _I32, _I32, _I64, _I64, _P, _I32, _P, _P, _F32, _I32,
-                                             _I32, _P, _P, _I64, _P, _SZ, _P]),
+                                             _I32, _I32, _I64, _I64, _P, _I32, _P, _P, ctypes.c_int,
+                                             _F32, _I32, _I32, _P, _P, _I64, _P, _SZ, _P]),
     "gdn_prefill_status": (ctypes.c_int, [_P, _P]),
     "gdn_prefill_noalloc_status": (ctypes.c_int, [_P]),
     "gdn_decode_step": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _I32, _I32,
@@ -44,6 +44,7 @@ SIGNATURES = {
                                           _I32, _I32, _I32, _I32, _I32, _F32, _P]),
     "gdn_decode_tokens_ex": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int, _P, ctypes.c_int,
                                             _I32, _I32, _I32, _I32, _I32, _I32, _F32, _P]),
+    "gdn_chunk_prefill_path": (_I32, [ctypes.c_int, _I32, _I32, _I32, _I32, _I32]),
     "gdn_chunk_prefill_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int, _I64, _I32,
                                                   _I32, _I32, _I32, _I64, _I64, _P, _I32, _P, _P,
                                                   _F32, _I32, _P]),
@@ -144,6 +145,20 @@ def gdn_chunk_prefill_workspace_size(T: int, n_seq: int, Hk: int, Hv: int, dk: i
     return int(n)
 
 
+PATH_NAMES = {0: "recurrent", 1: "chunked_tc"}
+
+
+def gdn_chunk_prefill_path(dtype: torch.dtype, Hk: int, Hv: int, dk: int, dv: int,
+                           qk_l2norm: bool = True) -> str:
+    """Which kernels gdn_chunk_prefill runs for these arguments: "chunked_tc" (the chunked
+    form on tcgen05 tensor cores) or "recurrent" (the token-by-token fp32 kernel)."""
+    code = GDN_BF16 if dtype == torch.bfloat16 else GDN_F32
+    p = lib().gdn_chunk_prefill_path(code, Hk, Hv, dk, dv, int(bool(qk_l2norm)))
+    if p < 0:
+        raise GDNError(GDN_ERR_UNSUPPORTED, "gdn_chunk_prefill_path", "unsupported shape")
+    return PATH_NAMES[p]
+
+
 def _row_view(t: torch.Tensor, name: str):
     """[T, H, d] with unit inner stride and dense heads; returns the token stride."""
     if t.dim() != 3 or t.stride(2) != 1 or t.stride(1) != t.shape[2]:
@@ -163,9 +178,11 @@ def gdn_chunk_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torc
     """Gated delta rule over packed sequences (see include/gdn.h). Returns o [T, Hv, dv].
 
     q, k: [T, Hk, dk] and v: [T, Hv, dv] may be token-strided views (e.g. of the conv
-    output). ``final_state`` (fp32 [N, Hv, dv, dk]) is written when given. With
-    ``block_tokens`` > 0 (a multiple of 64) the state after every block_tokens tokens of
-    sequence n goes to ``block_states`` (fp32 [R, Hv, dv, dk]) rows block_rows[n], +1, ...
+    output). ``final_state`` ([N, Hv, dv, dk]) is written when given. States are fp32, or
+    bf16 storage (fp32 math): the dtype of ``initial_state`` / ``final_state`` /
+    ``block_states``, which must agree. With ``block_tokens`` > 0 (a multiple of 64) the
+    state after every block_tokens tokens of sequence n goes to ``block_states``
+    ([R, Hv, dv, dk]) rows block_rows[n], +1, ...
     ``check``: wait for the call and raise GDNError if a bounded device-side wait gave up.
     """
     T, Hk, dk = q.shape
@@ -180,8 +197,12 @@ def gdn_chunk_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torc
     _need(g, "g", (T, Hv), torch.float32, dev)
     _need(beta, "beta", (T, Hv), torch.float32, dev)
     _need(cu_seqlens, "cu_seqlens", dtype=torch.int32, device=dev)
-    _need(initial_state, "initial_state", (n_seq, Hv, dv, dk), torch.float32, dev)
-    _need(final_state, "final_state", (n_seq, Hv, dv, dk), torch.float32, dev)
+    st_dtype = next((t.dtype for t in (initial_state, final_state, block_states if block_tokens else None)
+                     if t is not None), torch.float32)
+    if st_dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError(f"states must be fp32 or bf16, got {st_dtype}")
+    _need(initial_state, "initial_state", (n_seq, Hv, dv, dk), st_dtype, dev)
+    _need(final_state, "final_state", (n_seq, Hv, dv, dk), st_dtype, dev)
     if o is None:
         o = torch.empty((T, Hv, dv), dtype=q.dtype, device=dev)
     _need(o, "o", (T, Hv, dv), q.dtype, dev)
@@ -193,14 +214,15 @@ def gdn_chunk_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torc
     if block_tokens:
         if block_states is None or block_rows is None:
             raise ValueError("block_tokens needs block_states and block_rows")
-        _need(block_states, "block_states", dtype=torch.float32, device=dev)
+        _need(block_states, "block_states", dtype=st_dtype, device=dev)
         if tuple(block_states.shape[1:]) != (Hv, dv, dk):
             raise ValueError(f"block_states has shape {tuple(block_states.shape)}, expected [R, {Hv}, {dv}, {dk}]")
         _need(block_rows, "block_rows", (n_seq,), torch.int32, dev)
         n_rows = block_states.shape[0]
     _check(lib().gdn_chunk_prefill_ex(
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(o), _dtype_code(q), T, Hk, Hv, dk, dv,
-        qs, vs, _ptr(cu_seqlens), n_seq, _ptr(initial_state), _ptr(final_state), float(scale),
+        qs, vs, _ptr(cu_seqlens), n_seq, _ptr(initial_state), _ptr(final_state),
+        GDN_BF16 if st_dtype == torch.bfloat16 else GDN_F32, float(scale),
         int(bool(qk_l2norm)), int(block_tokens), _ptr(block_states if block_tokens else None),
         _ptr(block_rows if block_tokens else None), n_rows, _ptr(workspace), ws_bytes,
         _stream(dev)), "gdn_chunk_prefill")
@@ -236,20 +258,25 @@ def gdn_chunk_prefill_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     _, Hv, dv = v.shape
     dev = q.device
     n_seq = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
-    qs = _row_view(q, "q"); ks = _row_view(k, "k"); _row_view(v, "v")
+    qs = _row_view(q, "q"); ks = _row_view(k, "k"); vs = _row_view(v, "v")
     if k.shape != q.shape or ks != qs:
         raise ValueError("k must match q in shape and token stride")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, dtype=q.dtype, device=dev, dense=False)
     _need(g, "g", (T, Hv), torch.float32, dev)
     _need(beta, "beta", (T, Hv), torch.float32, dev)
+    _need(cu_seqlens, "cu_seqlens", dtype=torch.int32, device=dev)
     _need(initial_state, "initial_state", (n_seq, Hv, dv, dk), torch.float32, dev)
     _need(final_state, "final_state", (n_seq, Hv, dv, dk), torch.float32, dev)
     if o is None:
         o = torch.empty((T, Hv, dv), dtype=q.dtype, device=dev)
     _need(o, "o", (T, Hv, dv), q.dtype, dev)
-    _check(lib().gdn_chunk_prefill_noalloc(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(o), _dtype_code(q), T, Hk, Hv, dk, dv,
-        qs, v.stride(0), _ptr(cu_seqlens), n_seq, _ptr(initial_state), _ptr(final_state),
-        float(scale), int(bool(qk_l2norm)), _stream(dev)), "gdn_chunk_prefill_noalloc")
+    # the scratch array is per device: make the tensors' device current for the call
+    with torch.cuda.device(dev):
+        _check(lib().gdn_chunk_prefill_noalloc(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(o), _dtype_code(q), T, Hk, Hv,
+            dk, dv, qs, vs, _ptr(cu_seqlens), n_seq, _ptr(initial_state), _ptr(final_state),
+            float(scale), int(bool(qk_l2norm)), _stream(dev)), "gdn_chunk_prefill_noalloc")
     return o
 
 

@@ -17,6 +17,26 @@ template <typename T> __device__ __forceinline__ T from_f(float v);
 template <> __device__ __forceinline__ float from_f<float>(float v) { return v; }
 template <> __device__ __forceinline__ bf16 from_f<bf16>(float v) { return __float2bfloat16_rn(v); }
 
+// (a, b) as a bf16 pair hi (nearest, ties to even) and the bf16 pair lo of what hi left out,
+// so hi + lo carries about 16 significant bits: one paired conversion for each, the
+// widening of hi back to fp32 by bit operations.
+__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  hi = *reinterpret_cast<uint32_t*>(&h);
+  __nv_bfloat162 l = __floats2bfloat162_rn(a - __uint_as_float(hi << 16), b - __uint_as_float(hi & 0xFFFF0000u));
+  lo = *reinterpret_cast<uint32_t*>(&l);
+}
+
+// Recurrent-state elements in HBM: fp32, or bf16 storage (widened to fp32 on load, rounded
+// to nearest-even once on store).
+__device__ __forceinline__ float state_load(const void* p, int64_t i, bool bf) {
+  return bf ? __bfloat162float(static_cast<const bf16*>(p)[i]) : static_cast<const float*>(p)[i];
+}
+__device__ __forceinline__ void state_store(void* p, int64_t i, float v, bool bf) {
+  if (bf) static_cast<bf16*>(p)[i] = __float2bfloat16_rn(v);
+  else static_cast<float*>(p)[i] = v;
+}
+
 // N contiguous elements starting at p (p aligned to N * sizeof(T)), widened to fp32.
 template <typename T, int N> struct VecIO;
 

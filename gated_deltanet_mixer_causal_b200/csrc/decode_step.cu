@@ -8,8 +8,9 @@
 // One CTA owns one (sequence b, key head hk): the conv channels of that key head's q and k
 // and of its G = Hv/Hk value heads. Owning the channels makes the in-place tap shift
 // race-free without a second kernel. After the conv, SiLU and the q/k L2 norm (in shared
-// memory), each warp streams whole state rows (value index i): a row is 128 floats, one
-// float4 per lane, so a warp access is 512 contiguous bytes. Per row, with s the old row:
+// memory), each warp streams whole state rows (value index i): an fp32 row is 128 floats,
+// one float4 per lane, so a warp access is 512 contiguous bytes; a bf16 row (256 bytes) is
+// read by half a warp with 16-byte loads, two rows per access. Per row, with s the old row:
 //   sk = s.k, sq = s.q                  (one two-value warp reduction)
 //   u  = beta (v_i - alpha sk)          (delta write strength for this row)
 //   s' = alpha s + u k                  (decay, then the write along k)
@@ -50,16 +51,24 @@ template <> struct RowIO<float, 1> {
   static __device__ __forceinline__ void load(const float* p, float (&s)[1]) { s[0] = __ldcs(p); }
   static __device__ __forceinline__ void store(float* p, const float (&s)[1]) { __stcs(p, s[0]); }
 };
-template <> struct RowIO<bf16, 4> {
-  static __device__ __forceinline__ void load(const bf16* p, float (&s)[4]) {
-    const uint2 u = __ldcs(reinterpret_cast<const uint2*>(p));
-    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
-    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
-    s[0] = a.x; s[1] = a.y; s[2] = b.x; s[3] = b.y;
+template <> struct RowIO<bf16, 8> {
+  static __device__ __forceinline__ void load(const bf16* p, float (&s)[8]) {
+    const uint4 u = __ldcs(reinterpret_cast<const uint4*>(p));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+      s[2 * i] = f.x; s[2 * i + 1] = f.y;
+    }
   }
-  static __device__ __forceinline__ void store(bf16* p, const float (&s)[4]) {
-    __nv_bfloat162 a = __floats2bfloat162_rn(s[0], s[1]), b = __floats2bfloat162_rn(s[2], s[3]);
-    __stcs(reinterpret_cast<uint2*>(p), make_uint2(*reinterpret_cast<uint32_t*>(&a), *reinterpret_cast<uint32_t*>(&b)));
+  static __device__ __forceinline__ void store(bf16* p, const float (&s)[8]) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __nv_bfloat162 f = __floats2bfloat162_rn(s[2 * i], s[2 * i + 1]);
+      w[i] = *reinterpret_cast<uint32_t*>(&f);
+    }
+    __stcs(reinterpret_cast<uint4*>(p), make_uint4(w[0], w[1], w[2], w[3]));
   }
 };
 template <> struct RowIO<bf16, 2> {
@@ -78,13 +87,24 @@ template <> struct RowIO<bf16, 1> {
   static __device__ __forceinline__ void store(bf16* p, const float (&s)[1]) { p[0] = __float2bfloat16_rn(s[0]); }
 };
 
+// Lanes per state row: a row of 128 bf16 values (256 bytes) is read by 16 lanes with 16-byte
+// loads, two rows per warp access, so a warp instruction still moves 512 bytes and each
+// row's dot products reduce over 16 lanes (4 shuffle rounds); every other case uses the
+// whole warp per row.
+template <typename S, int D> struct RowShape {
+  static constexpr int VEC = (sizeof(S) == 2 && D == 128) ? 8 : (D >= 32 ? D / 32 : 1);
+  static constexpr int LPR = (sizeof(S) == 2 && D == 128) ? 16 : 32;
+};
+
 template <typename T, int D, typename S>
 __global__ void __launch_bounds__(kThreads)
 decode_step_kernel(const T* __restrict__ x, const T* __restrict__ conv_w, T* __restrict__ conv_state,
                    const float* __restrict__ g, const float* __restrict__ beta,
                    S* __restrict__ state, T* __restrict__ o, int32_t Hk, int32_t Hv,
                    float scale) {
-  constexpr int VEC = D >= 32 ? D / 32 : 1;
+  constexpr int VEC = RowShape<S, D>::VEC;
+  constexpr int LPR = RowShape<S, D>::LPR;   // lanes per row
+  constexpr int RPW = 32 / LPR;              // rows per warp access
   const int G = Hv / Hk;
   const int32_t Cc = 2 * Hk * D + Hv * D;
   const int64_t b = blockIdx.x / Hk;
@@ -127,34 +147,43 @@ decode_step_kernel(const T* __restrict__ x, const T* __restrict__ conv_w, T* __r
   }
   __syncthreads();
 
-  // 2. L2-normalised q and k, per warp, in registers (VEC columns per lane).
-  const bool active = lane * VEC < D;
+  // 2. L2-normalised q and k, per warp, in registers (VEC columns per lane; with LPR = 16
+  //    lanes l and l + 16 hold the same columns).
+  const int col = (lane % LPR) * VEC;
+  const bool active = col < D;
   float qh[VEC], kh[VEC];
   float qq = 0.f, kk = 0.f, kq = 0.f;
 #pragma unroll
   for (int j = 0; j < VEC; ++j) {
-    qh[j] = active ? ys[lane * VEC + j] : 0.f;
-    kh[j] = active ? ys[D + lane * VEC + j] : 0.f;
+    qh[j] = active ? ys[col + j] : 0.f;
+    kh[j] = active ? ys[D + col + j] : 0.f;
     qq = fmaf(qh[j], qh[j], qq);
     kk = fmaf(kh[j], kh[j], kk);
     kq = fmaf(kh[j], qh[j], kq);
   }
-  qq = warp_sum(qq); kk = warp_sum(kk); kq = warp_sum(kq);
+#pragma unroll
+  for (int m = LPR / 2; m >= 1; m >>= 1) {
+    qq += __shfl_xor_sync(0xffffffffu, qq, m);
+    kk += __shfl_xor_sync(0xffffffffu, kk, m);
+    kq += __shfl_xor_sync(0xffffffffu, kq, m);
+  }
   const float iq = 1.0f / sqrtf(qq + kEps), ik = 1.0f / sqrtf(kk + kEps);
 #pragma unroll
   for (int j = 0; j < VEC; ++j) { qh[j] *= iq; kh[j] *= ik; }
   const float kqh = kq * iq * ik;
 
-  // 3. stream the G * D state rows of this CTA.
+  // 3. stream the G * D state rows of this CTA: a warp takes kRowUnroll x RPW rows per
+  //    iteration (row r0 + u * RPW + lane / LPR in slot u).
   const int rows = G * D;
-  for (int r0 = warp * kRowUnroll; r0 < rows; r0 += kWarps * kRowUnroll) {
+  const int sub = lane / LPR;
+  for (int r0 = warp * kRowUnroll * RPW; r0 < rows; r0 += kWarps * kRowUnroll * RPW) {
     float s[kRowUnroll][VEC];
     S* ptr[kRowUnroll];
 #pragma unroll
     for (int u = 0; u < kRowUnroll; ++u) {
-      const int r = r0 + u;
+      const int r = r0 + u * RPW + sub;
       const int h = hk * G + r / D, i = r % D;
-      ptr[u] = state + ((b * Hv + h) * (int64_t)D + i) * D + lane * VEC;
+      ptr[u] = state + ((b * Hv + h) * (int64_t)D + i) * D + col;
       if (r < rows && active) RowIO<S, VEC>::load(ptr[u], s[u]);
       else {
 #pragma unroll
@@ -170,7 +199,7 @@ decode_step_kernel(const T* __restrict__ x, const T* __restrict__ conv_w, T* __r
       sk[u] = a; sq[u] = c;
     }
 #pragma unroll
-    for (int m = 16; m >= 1; m >>= 1)
+    for (int m = LPR / 2; m >= 1; m >>= 1)
 #pragma unroll
       for (int u = 0; u < kRowUnroll; ++u) {
         sk[u] += __shfl_xor_sync(0xffffffffu, sk[u], m);
@@ -178,8 +207,8 @@ decode_step_kernel(const T* __restrict__ x, const T* __restrict__ conv_w, T* __r
       }
 #pragma unroll
     for (int u = 0; u < kRowUnroll; ++u) {
-      const int r = r0 + u;
-      if (r >= rows) break;
+      const int r = r0 + u * RPW + sub;
+      if (r >= rows) continue;
       const int h = hk * G + r / D;
       const float alpha = expf(g[b * Hv + h]);
       const float bt = beta[b * Hv + h];
@@ -187,7 +216,7 @@ decode_step_kernel(const T* __restrict__ x, const T* __restrict__ conv_w, T* __r
 #pragma unroll
       for (int j = 0; j < VEC; ++j) s[u][j] = fmaf(alpha, s[u][j], uu * kh[j]);
       if (active) RowIO<S, VEC>::store(ptr[u], s[u]);
-      if (lane == 0) os[r] = scale * fmaf(alpha, sq[u], uu * kqh);
+      if (lane % LPR == 0) os[r] = scale * fmaf(alpha, sq[u], uu * kqh);
     }
   }
   __syncthreads();

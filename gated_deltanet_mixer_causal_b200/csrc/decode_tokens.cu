@@ -147,22 +147,36 @@ decode_tokens_kernel(const T* __restrict__ x, const T* __restrict__ conv_w, T* _
   //    rounds; a warp takes 32 / L consecutive rows per pass. Lane seg of a row holds the
   //    float4 columns j * 4L + 4 seg (j < 4): for each of its four loads the row's lanes
   //    cover one contiguous 16L-float span, so every access is a full line.
+  //    The next pass's rows are loaded before this pass's tokens run (software pipelining),
+  //    so each warp keeps a pass of loads in flight while it computes.
   constexpr int SEG = 16;
   constexpr int L = D / SEG;
   constexpr int RPW = 32 / L;
   const int rows = G * D;
   const int seg = lane % L;
+  auto row_ptr = [&](int r) {
+    const int rr = r < rows ? r : 0;
+    return state + ((b * Hv + hk * G + rr / D) * (int64_t)D + rr % D) * D + seg * 4;
+  };
+  auto load_row = [&](int r, float (&dst)[SEG]) {
+    S* p = row_ptr(r);
+#pragma unroll
+    for (int j = 0; j < SEG; j += 4) {
+      const float4 v = r < rows ? Quad<S>::load(p + j * L) : make_float4(0.f, 0.f, 0.f, 0.f);
+      dst[j] = v.x; dst[j + 1] = v.y; dst[j + 2] = v.z; dst[j + 3] = v.w;
+    }
+  };
+  float s_next[SEG];
+  load_row(warp * RPW + lane / L, s_next);
   for (int r0 = warp * RPW; r0 < rows; r0 += kWarps * RPW) {
     const int r = r0 + lane / L;
     const bool live = r < rows;
     const int h = hk * G + (live ? r : 0) / D;
-    S* ptr = state + ((b * Hv + h) * (int64_t)D + (live ? r : 0) % D) * D + seg * 4;
+    S* ptr = row_ptr(r);
     float s[SEG];
 #pragma unroll
-    for (int j = 0; j < SEG; j += 4) {
-      const float4 v = live ? Quad<S>::load(ptr + j * L) : make_float4(0.f, 0.f, 0.f, 0.f);
-      s[j] = v.x; s[j + 1] = v.y; s[j + 2] = v.z; s[j + 3] = v.w;
-    }
+    for (int j = 0; j < SEG; ++j) s[j] = s_next[j];
+    if (r0 + kWarps * RPW < rows) load_row(r + kWarps * RPW, s_next);
 #pragma unroll
     for (int t = 0; t < kMaxTok; ++t) {
       if (t >= n_tok) break;

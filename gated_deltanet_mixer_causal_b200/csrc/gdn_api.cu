@@ -7,7 +7,7 @@
 #include <stdio.h>
 #include <string.h>
 
-#include "../../include/gdn.h"
+#include "gdn.h"
 #include "launch.h"
 
 namespace {
@@ -65,6 +65,28 @@ bool use_tensor_core_prefill(gdn_dtype_t dt, int32_t d, int32_t Hk, int32_t Hv, 
 
 }  // namespace
 
+namespace gdn {
+
+size_t prefill_workspace_need(gdn_dtype_t dt, int64_t T, int32_t n_seq, int32_t Hk, int32_t Hv,
+                              int32_t dk, int32_t dv, int32_t qk_l2norm) {
+  if (!valid_dtype(dt) || T < 0 || Hk <= 0 || Hv <= 0 || Hv % Hk != 0 || dk != dv ||
+      !supported_head_dim(dk))
+    return SIZE_MAX;
+  if (n_seq < 1) n_seq = 1;
+  if (!use_tensor_core_prefill(dt, dk, Hk, Hv, qk_l2norm)) return 0;
+  return tc_rows_fit(T, n_seq, Hv) ? prefill_chunk_tc_workspace(T, n_seq, Hv) : SIZE_MAX;
+}
+
+gdn_status_t set_error(gdn_status_t s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+}  // namespace gdn
+
 extern "C" {
 
 const char* gdn_status_string(gdn_status_t s) {
@@ -114,23 +136,28 @@ gdn_status_t gdn_conv1d_silu(const void* x, void* y, gdn_dtype_t dt, const void*
 
 size_t gdn_chunk_prefill_workspace_size(int64_t T, int32_t n_seq, int32_t Hk, int32_t Hv,
                                         int32_t dk, int32_t dv, gdn_dtype_t dt) {
-  if (!valid_dtype(dt) || T < 0 || Hk <= 0 || Hv <= 0 || Hv % Hk != 0 || dk != dv ||
-      !supported_head_dim(dk))
-    return SIZE_MAX;
-  if (n_seq < 1) n_seq = 1;
-  if (!use_tensor_core_prefill(dt, dk, Hk, Hv)) return 0;
-  return tc_rows_fit(T, n_seq, Hv) ? gdn::prefill_chunk_tc_workspace(T, n_seq, Hv) : SIZE_MAX;
+  return gdn::prefill_workspace_need(dt, T, n_seq, Hk, Hv, dk, dv, 1);
+}
+
+int32_t gdn_chunk_prefill_path(gdn_dtype_t dt, int32_t Hk, int32_t Hv, int32_t dk, int32_t dv,
+                               int32_t qk_l2norm) {
+  if (!valid_dtype(dt) || Hk <= 0 || Hv <= 0 || Hv % Hk != 0 || dk != dv || !supported_head_dim(dk))
+    return -1;
+  return use_tensor_core_prefill(dt, dk, Hk, Hv, qk_l2norm) ? GDN_PATH_CHUNKED_TC : GDN_PATH_RECURRENT;
 }
 
 gdn_status_t gdn_chunk_prefill_ex(const void* q, const void* k, const void* v, const float* g,
                                   const float* beta, void* o, gdn_dtype_t dt, int64_t T,
                                   int32_t Hk, int32_t Hv, int32_t dk, int32_t dv, int64_t qk_stride,
                                   int64_t v_stride, const int32_t* cu_seqlens, int32_t n_seq,
-                                  const float* initial_state, float* final_state, float scale,
-                                  int32_t qk_l2norm, int32_t block_tokens, float* block_states,
+                                  const void* initial_state, void* final_state,
+                                  gdn_dtype_t state_dt, float scale, int32_t qk_l2norm,
+                                  int32_t block_tokens, void* block_states,
                                   const int32_t* block_rows, int64_t n_block_rows, void* workspace,
                                   size_t workspace_bytes, gdn_stream_t stream) {
   if (!valid_dtype(dt)) return fail(GDN_ERR_UNSUPPORTED, "chunk_prefill: unknown dtype %d", (int)dt);
+  if (!valid_dtype(state_dt))
+    return fail(GDN_ERR_UNSUPPORTED, "chunk_prefill: unknown state dtype %d", (int)state_dt);
   if (T < 0) return fail(GDN_ERR_INVALID_ARG, "chunk_prefill: T = %lld < 0", (long long)T);
   if (Hk <= 0 || Hv <= 0) return fail(GDN_ERR_INVALID_ARG, "chunk_prefill: Hk, Hv must be > 0");
   if (Hv % Hk != 0) return fail(GDN_ERR_UNSUPPORTED, "chunk_prefill: Hv %% Hk != 0 (%d, %d)", Hv, Hk);
@@ -153,7 +180,8 @@ gdn_status_t gdn_chunk_prefill_ex(const void* q, const void* k, const void* v, c
   const size_t ob = (size_t)T * Hv * dv * es;
   const size_t qkb = T > 0 ? ((size_t)(T - 1) * qk_stride + (size_t)Hk * dk) * es : 0;
   const size_t vb = T > 0 ? ((size_t)(T - 1) * v_stride + (size_t)Hv * dv) * es : 0;
-  const size_t gb = (size_t)T * Hv * 4, stb = (size_t)n_seq * Hv * dv * dk * 4;
+  const size_t sts = elt_size(state_dt);
+  const size_t gb = (size_t)T * Hv * 4, stb = (size_t)n_seq * Hv * dv * dk * sts;
   if (overlap(o, ob, q, qkb) || overlap(o, ob, k, qkb) || overlap(o, ob, v, vb) ||
       overlap(o, ob, g, gb) || overlap(o, ob, beta, gb) || overlap(o, ob, initial_state, stb) ||
       overlap(o, ob, final_state, stb))
@@ -169,7 +197,7 @@ gdn_status_t gdn_chunk_prefill_ex(const void* q, const void* k, const void* v, c
       return fail(GDN_ERR_INVALID_ARG, "chunk_prefill: block states need block_states, block_rows and n_block_rows >= 1");
     if (!aligned16(block_states))
       return fail(GDN_ERR_INVALID_ARG, "chunk_prefill: block_states must be 16-byte aligned");
-    const size_t bsb = (size_t)n_block_rows * Hv * dv * dk * 4;
+    const size_t bsb = (size_t)n_block_rows * Hv * dv * dk * sts;
     if (overlap(block_states, bsb, q, qkb) || overlap(block_states, bsb, k, qkb) ||
         overlap(block_states, bsb, v, vb) || overlap(block_states, bsb, g, gb) ||
         overlap(block_states, bsb, beta, gb) || overlap(block_states, bsb, o, ob) ||
@@ -194,7 +222,8 @@ gdn_status_t gdn_chunk_prefill_ex(const void* q, const void* k, const void* v, c
       return fail(GDN_ERR_INVALID_ARG, "chunk_prefill: workspace must be 256-byte aligned");
     return cuda_status(gdn::launch_prefill_chunk_tc(q, k, v, g, beta, o, T, Hk, Hv, qk_stride, v_stride,
                                                     cu_seqlens, n_seq, initial_state, final_state,
-                                                    scale, blocks, workspace, (cudaStream_t)stream),
+                                                    (int)state_dt, scale, blocks, workspace,
+                                                    (cudaStream_t)stream),
                        "chunk_prefill (tensor-core) launch");
   }
   if (workspace != nullptr && workspace_bytes >= sizeof(int)) {   // no wait can fail here
@@ -203,8 +232,8 @@ gdn_status_t gdn_chunk_prefill_ex(const void* q, const void* k, const void* v, c
   }
   return cuda_status(gdn::launch_prefill_recurrent((int)dt, q, k, v, g, beta, o, T, Hk, Hv, dk,
                                                    qk_stride, v_stride, cu_seqlens, n_seq,
-                                                   initial_state, final_state, scale, qk_l2norm,
-                                                   blocks, (cudaStream_t)stream),
+                                                   initial_state, final_state, (int)state_dt, scale,
+                                                   qk_l2norm, blocks, (cudaStream_t)stream),
                      "chunk_prefill launch");
 }
 
@@ -228,8 +257,8 @@ gdn_status_t gdn_chunk_prefill(const void* q, const void* k, const void* v, cons
                                int32_t qk_l2norm, void* workspace, size_t workspace_bytes,
                                gdn_stream_t stream) {
   return gdn_chunk_prefill_ex(q, k, v, g, beta, o, dt, T, Hk, Hv, dk, dv, qk_stride, v_stride,
-                              cu_seqlens, n_seq, initial_state, final_state, scale, qk_l2norm, 0,
-                              nullptr, nullptr, 0, workspace, workspace_bytes, stream);
+                              cu_seqlens, n_seq, initial_state, final_state, GDN_F32, scale,
+                              qk_l2norm, 0, nullptr, nullptr, 0, workspace, workspace_bytes, stream);
 }
 
 gdn_status_t gdn_decode_step_ex(const void* x, const void* conv_w, void* conv_state, const float* g,

@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "gdn.h"
+
 namespace gdn {
 
 constexpr int kF32 = 0;   // GDN_F32
@@ -29,22 +31,24 @@ cudaError_t launch_decode_tokens(int dtype, const void* x, const void* conv_w, v
 
 // States at block boundaries (prefix caching): after every block_tokens tokens of a sequence
 // (block_tokens a positive multiple of 64; 0 = none), its state goes to row
-// block_rows[n] + m - 1 of block_states [n_block_rows, Hv, dv, dk] fp32 for the m-th
-// boundary; rows outside [0, n_block_rows) are skipped.
+// block_rows[n] + m - 1 of block_states [n_block_rows, Hv, dv, dk] (the state dtype of the
+// call) for the m-th boundary; rows outside [0, n_block_rows) are skipped.
 struct BlockStates {
   int32_t block_tokens = 0;
-  float* states = nullptr;
+  void* states = nullptr;
   const int32_t* rows = nullptr;
   int64_t n_rows = 0;
 };
 
-// Token-by-token fp32 recurrence (SIMT): the fp32-activation prefill path.
+// Token-by-token fp32 recurrence (SIMT): the fp32-activation prefill path. States (initial,
+// final, block) are stored as state_dtype (kF32, or kBF16 storage with fp32 math).
 cudaError_t launch_prefill_recurrent(int dtype, const void* q, const void* k, const void* v,
                                      const float* g, const float* beta, void* o, int64_t T,
                                      int32_t Hk, int32_t Hv, int32_t d, int64_t qk_stride,
                                      int64_t v_stride, const int32_t* cu, int32_t n_seq,
-                                     const float* init, float* final_state, float scale,
-                                     int32_t l2norm, BlockStates blocks, cudaStream_t stream);
+                                     const void* init, void* final_state, int state_dtype,
+                                     float scale, int32_t l2norm, BlockStates blocks,
+                                     cudaStream_t stream);
 
 // Chunked WY/UT prefill on tcgen05 (bf16 activations, dk = dv = 128, at most
 // kPrefillTcMaxG value heads per key head). Needs
@@ -56,7 +60,16 @@ const char* prefill_chunk_tc_error_string(int code);
 cudaError_t launch_prefill_chunk_tc(const void* q, const void* k, const void* v, const float* g,
                                     const float* beta, void* o, int64_t T, int32_t Hk, int32_t Hv,
                                     int64_t qk_stride, int64_t v_stride, const int32_t* cu,
-                                    int32_t n_seq, const float* init, float* fin, float scale,
-                                    BlockStates blocks, void* workspace, cudaStream_t stream);
+                                    int32_t n_seq, const void* init, void* fin, int state_dtype,
+                                    float scale, BlockStates blocks, void* workspace,
+                                    cudaStream_t stream);
+
+// Workspace bytes the prefill path chosen for these arguments needs (0 for the
+// token-recurrent path, which takes no workspace); SIZE_MAX for unsupported shapes.
+size_t prefill_workspace_need(gdn_dtype_t dt, int64_t T, int32_t n_seq, int32_t Hk, int32_t Hv,
+                              int32_t dk, int32_t dv, int32_t qk_l2norm);
+
+// Records the calling thread's gdn_last_error() text and returns s.
+gdn_status_t set_error(gdn_status_t s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
 
 }  // namespace gdn

@@ -53,13 +53,16 @@ constexpr int kErrIntraTma = 11, kErrIntraMma = 12, kErrChainTma = 21, kErrChain
 // ------------------------------------------------------------------ workspace layout
 
 struct Ws {
-  size_t err, prefix, wu, mq, vecs, total;
+  size_t err, prefix, wu, ul, mq, vecs, total;
 };
 
 // Per (chunk, value head): wu = [-W (64 x 128) ; U~ (64 x 128)] bf16 rows of 128 elements,
-// mq = Mqk (64 x 64) bf16, vecs = row scales: [0, 64) e^{G_r}/|q_r|, [64, 128)
-// e^{G_L - G_r}/|k_r|, [128] e^{G_L}; 132 floats = 528 bytes (a multiple of 16).
+// ul = U~ - bf16(U~) (64 x 128 bf16: U~ is carried as a hi + lo pair, because a chunk that
+// rewrites one key many times turns U~ into differences of values whose bf16 roundings would
+// add up in the state), mq = Mqk (64 x 64) bf16, vecs = row scales: [0, 64) e^{G_r}/|q_r|,
+// [64, 128) e^{G_L - G_r}/|k_r|, [128] e^{G_L}; 132 floats = 528 bytes (a multiple of 16).
 constexpr int kWuBytes = 2 * C * D * 2;
+constexpr int kUlBytes = C * D * 2;   // U~ - bf16(U~): the low half of a hi + lo bf16 pair
 constexpr int kVecFloats = 132;
 constexpr int kVecBytes = kVecFloats * 4;
 
@@ -73,7 +76,8 @@ __host__ __device__ inline Ws ws_layout(int64_t T, int32_t n_seq, int32_t Hv) {
   w.err = 0;
   w.prefix = 256;
   w.wu = align256(w.prefix + (size_t)(n_seq + 1) * 4);
-  w.mq = align256(w.wu + slots * Hv * kWuBytes);
+  w.ul = align256(w.wu + slots * Hv * kWuBytes);
+  w.mq = align256(w.ul + slots * Hv * kUlBytes);
   w.vecs = align256(w.mq + slots * Hv * kMatBytes);
   w.total = align256(w.vecs + slots * Hv * kVecBytes);
   return w;
@@ -144,7 +148,11 @@ __device__ __forceinline__ uint32_t tmem_quadrant(uint32_t tmem, int warp) {
 
 // ------------------------------------------------------------------------ intra
 
-// Warp-level tf32 MMA (m16n8k8) for the 16x16 block products of the triangular inverse.
+// Warp-level MMAs (m16n8k8, tf32 inputs, fp32 accumulate) for the 16 x 16 block products of the
+// triangular inverse off its diagonal. The inverse is rounded to bf16 right after (as the
+// factors P, Pk of the tcgen05 products), which dominates tf32's 10-bit operand rounding: a
+// split hi + lo tf32 form (fp32-accurate) changes the errors of the whole prefill by under 1 %
+// on the near-collinear, repeated-key and no-decay inputs, so the plain form is used.
 __device__ __forceinline__ uint32_t to_tf32(float x) {
   uint32_t r;
   asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
@@ -156,27 +164,8 @@ __device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
-// c (a 16x16 block as two m16n8 fragments) += X[xr.., xc..] * Y[yr.., yc..], fp32 matrices with
-// row pitch px / py. X is read transposed (X(i, k) = Xs[k][i]) when x_t is set.
-template <bool x_t>
-__device__ __forceinline__ void block_mma16(float (&c)[2][4], const float* Xs, int px, int xr, int xc,
-                                            const float* Ys, int py, int yr, int yc, int lane) {
-  const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-  for (int ks = 0; ks < 2; ++ks) {
-    const int k0 = 8 * ks + t;
-    auto X = [&](int i, int k) { return x_t ? Xs[(xc + k) * px + xr + i] : Xs[(xr + i) * px + xc + k]; };
-    const uint32_t a[4] = {to_tf32(X(g, k0)), to_tf32(X(g + 8, k0)), to_tf32(X(g, k0 + 4)), to_tf32(X(g + 8, k0 + 4))};
-#pragma unroll
-    for (int nh = 0; nh < 2; ++nh) {
-      const uint32_t bb[2] = {to_tf32(Ys[(yr + k0) * py + yc + 8 * nh + g]),
-                              to_tf32(Ys[(yr + k0 + 4) * py + yc + 8 * nh + g])};
-      mma_tf32_16x8x8(c[nh], a, bb);
-    }
-  }
-}
-
-// The same for one 16x8 half (columns 8 nh .. 8 nh + 7) of the result.
+// c (one 16x8 half, columns 8 nh .. 8 nh + 7, of a 16x16 block) += X[xr.., xc..] Y[yr.., yc..]
+// for fp32 matrices with row pitches px, py.
 __device__ __forceinline__ void block_mma16h(float (&c)[4], const float* Xs, int px, int xr, int xc,
                                              const float* Ys, int py, int yr, int yc, int nh, int lane) {
   const int g = lane >> 2, t = lane & 3;
@@ -189,6 +178,12 @@ __device__ __forceinline__ void block_mma16h(float (&c)[4], const float* Xs, int
                             to_tf32(Ys[(yr + k0 + 4) * py + yc + 8 * nh + g])};
     mma_tf32_16x8x8(c, a, bb);
   }
+}
+// Both halves of a 16 x 16 block product.
+__device__ __forceinline__ void block_mma16(float (&c)[2][4], const float* Xs, int px, int xr, int xc,
+                                            const float* Ys, int py, int yr, int yc, int lane) {
+  block_mma16h(c[0], Xs, px, xr, xc, Ys, py, yr, yc, 0, lane);
+  block_mma16h(c[1], Xs, px, xr, xc, Ys, py, yr, yc, 1, lane);
 }
 
 // shared memory of the intra kernel (offsets from a 1024-aligned base)
@@ -211,24 +206,20 @@ constexpr int kIBar = kIGB + 2 * kMaxG * 64 * 4;    // 4 mbarriers + tmem addres
 constexpr int kIntraSmem = kIBar + 64 + 1024;   // + alignment slack
 constexpr uint32_t kTKQ = 0, kTUW = 128;        // TMEM columns: [KK^T; QK^T], [P;Pk] V or K
 
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(128, 2)   // two CTAs per SM (shared and tensor memory allow two)
 chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                    const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_wu,
+                   const __grid_constant__ CUtensorMap map_mq, const __grid_constant__ CUtensorMap map_ul,
                    const float* __restrict__ g,
                    const float* __restrict__ beta, const int32_t* __restrict__ cu, int32_t n_seq,
                    int64_t T, int32_t Hk, int32_t Hv, uint8_t* __restrict__ ws) {
   const Ws L = ws_layout(T, n_seq, Hv);
   int* err = reinterpret_cast<int*>(ws + L.err);
   const int32_t* prefix = reinterpret_cast<const int32_t*>(ws + L.prefix);
-  const int32_t slot = blockIdx.x, hk = blockIdx.y;
-  if (slot >= prefix[n_seq]) return;
-  const int32_t n = slot_to_seq(prefix, n_seq, slot);
-  int64_t bos, eos;
-  seq_bounds(cu, n, T, bos, eos);
-  const int64_t t0 = bos + (int64_t)(slot - prefix[n]) * C;
-  const int len = (int)(eos - t0 < C ? eos - t0 : C);
+  const int32_t n_items = prefix[n_seq] * Hk;   // item = slot * Hk + key head
   const int G = Hv / Hk;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if ((int32_t)blockIdx.x >= n_items) return;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -245,48 +236,94 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
   uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + kIBar);   // K and Q landed
   uint64_t* bar_mma = bar_tma + 1;
   uint64_t* bar_v = bar_tma + 2;   // [2] V tile of a value head landed in buffer j % 2
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_tma + 4);
+  uint64_t* bar_drain = bar_tma + 4;   // on an early exit: every MMA of this CTA has completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_tma + 5);
+  // loads issued into each barrier (thread 0 only): an early exit waits for the last of each
+  uint32_t n_kq = 0, n_v0 = 0, n_v1 = 0;
+
+  // The CTA is persistent: it takes items blockIdx.x, + gridDim.x, ... Each item's K, Q, the
+  // first V tile and its g, beta are fetched while the previous item finishes.
+  struct Item { int32_t slot, hk; int64_t t0; int len; };
+  auto item_at = [&](int32_t it, Item& x) {
+    if (it >= n_items) return false;
+    x.slot = it / Hk;
+    x.hk = it - x.slot * Hk;
+    const int32_t n = slot_to_seq(prefix, n_seq, x.slot);
+    int64_t bos, eos;
+    seq_bounds(cu, n, T, bos, eos);
+    x.t0 = bos + (int64_t)(x.slot - prefix[n]) * C;
+    x.len = (int)(eos - x.t0 < C ? eos - x.t0 : C);
+    return true;
+  };
+  // V tiles are double-buffered: buffer 0 at kIV, buffer 1 in the Q atoms (free once the
+  // [K; Q] K^T MMA has read them); head j + 2 loads while head j + 1 is computed
+  auto v_tile = [&](int b) { return sm + (b == 0 ? kIV : kIKQ + 8192); };
+  auto load_v = [&](const Item& x, int j) {   // value head hk * G + j into buffer j % 2
+    uint8_t* dst = v_tile(j & 1);
+    const uint32_t atom = (j & 1) ? 16384u : 8192u;
+    if (j & 1) ++n_v1; else ++n_v0;
+    mbar_arrive_expect_tx(&bar_v[j & 1], 16384);
+    for (int hh = 0; hh < 2; ++hh)
+      tma_load_2d(dst + hh * atom, &map_v, (x.hk * G + j) * D + hh * 64, (int32_t)x.t0, &bar_v[j & 1]);
+  };
+  auto load_kqv = [&](const Item& x) {   // thread 0: K, Q and the first V tile of item x
+    ++n_kq;
+    mbar_arrive_expect_tx(bar_tma, 32768);
+    for (int hh = 0; hh < 2; ++hh) {
+      tma_load_2d(sm + kIKQ + hh * 16384, &map_k, x.hk * D + hh * 64, (int32_t)x.t0, bar_tma);
+      tma_load_2d(sm + kIKQ + hh * 16384 + 8192, &map_q, x.hk * D + hh * 64, (int32_t)x.t0, bar_tma);
+    }
+    load_v(x, 0);
+  };
+  // g, beta of the G value heads of item x, this thread's share (rows past the sequence: 0)
+  constexpr int kGB = kMaxG * 64 / 128;
+  float gr[kGB], br[kGB];
+  auto fetch_gb = [&](const Item& x) {
+#pragma unroll
+    for (int i = 0; i < kGB; ++i) {
+      const int e = tid + i * 128, j = e >> 6, r = e & 63;
+      const bool v = j < G && r < x.len;
+      gr[i] = v ? g[(x.t0 + r) * Hv + x.hk * G + j] : 0.f;
+      br[i] = v ? beta[(x.t0 + r) * Hv + x.hk * G + j] : 0.f;
+    }
+  };
+  auto store_gb = [&]() {
+#pragma unroll
+    for (int i = 0; i < kGB; ++i) {
+      const int e = tid + i * 128;
+      if ((e >> 6) < G) { gAll[e] = gr[i]; bAll[e] = br[i]; }
+    }
+  };
 
   if (tid == 0) {
     mbar_init(bar_tma, 1);
     mbar_init(bar_mma, 1);
     mbar_init(&bar_v[0], 1);
     mbar_init(&bar_v[1], 1);
+    mbar_init(bar_drain, 1);
     fence_mbar_init();
   }
   if (warp == 0) { tmem_alloc(tmem_slot, 256); tmem_relinquish(); }
-  // g, beta of all G value heads for the chunk (rows past the sequence end: 0)
-  for (int e = tid; e < G * 64; e += 128) {
-    const int j = e >> 6, r = e & 63;
-    const bool v = r < len;
-    gAll[e] = v ? g[(t0 + r) * Hv + hk * G + j] : 0.f;
-    bAll[e] = v ? beta[(t0 + r) * Hv + hk * G + j] : 0.f;
-  }
+  Item cur;
+  item_at((int32_t)blockIdx.x, cur);
+  fetch_gb(cur);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (tid == 0) load_kqv(cur);
+  store_gb();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tq = tmem_quadrant(tmem, warp);   // lanes 32 w .. 32 w + 31: rows of M = 128 results
-  uint32_t ph_mma = 0u;
+  uint32_t ph_mma = 0u, ph_kq = 0u;
+  uint32_t vbase0 = 0u, vbase1 = 0u;   // completed loads of V buffers 0 and 1 before this item
+  bool ok = true;
+  __syncthreads();
 
-  // V tiles are double-buffered: buffer 0 at kIV, buffer 1 in the Q atoms (free once the
-  // [K; Q] K^T MMA has read them); head j + 2 loads while head j + 1 is computed
-  auto v_tile = [&](int b) { return sm + (b == 0 ? kIV : kIKQ + 8192); };
-  auto load_v = [&](int j) {   // value head hk * G + j into buffer j % 2
-    uint8_t* dst = v_tile(j & 1);
-    const uint32_t atom = (j & 1) ? 16384u : 8192u;
-    mbar_arrive_expect_tx(&bar_v[j & 1], 16384);
-    for (int hh = 0; hh < 2; ++hh)
-      tma_load_2d(dst + hh * atom, &map_v, (hk * G + j) * D + hh * 64, (int32_t)t0, &bar_v[j & 1]);
-  };
-  if (tid == 0) {
-    mbar_arrive_expect_tx(bar_tma, 32768);
-    for (int hh = 0; hh < 2; ++hh) {
-      tma_load_2d(sm + kIKQ + hh * 16384, &map_k, hk * D + hh * 64, (int32_t)t0, bar_tma);
-      tma_load_2d(sm + kIKQ + hh * 16384 + 8192, &map_q, hk * D + hh * 64, (int32_t)t0, bar_tma);
-    }
-    load_v(0);
-  }
+  for (int32_t item = blockIdx.x; item < n_items; item += gridDim.x) {
+  const int32_t slot = cur.slot, hk = cur.hk;
+  const int len = cur.len;
+  Item nxt;
+  const bool has_next = item_at(item + (int32_t)gridDim.x, nxt);
   if (warp < G) {   // inclusive cumulative log-decay of every value head, in place (2 values per lane)
     for (int j = warp; j < G; j += 4) {
       const float a0 = gAll[j * 64 + 2 * lane], a1 = gAll[j * 64 + 2 * lane + 1];
@@ -301,8 +338,9 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
       gAll[j * 64 + 2 * lane + 1] = excl + a0 + a1;
     }
   }
-  bool ok = mbar_wait(bar_tma, 0u, err, kErrIntraTma);
-  if (__syncthreads_or(!ok)) goto teardown;
+  ok = mbar_wait(bar_tma, ph_kq, err, kErrIntraTma);
+  ph_kq ^= 1u;
+  if (__syncthreads_or(!ok)) { ok = false; goto teardown; }
 
   {  // inverse L2 norms of the chunk's q and k rows (0 for rows past the sequence end)
     const int r = tid & 63;
@@ -334,9 +372,9 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
   }
   ok = mbar_wait(bar_mma, ph_mma, err, kErrIntraMma);
   ph_mma ^= 1u;
-  if (__syncthreads_or(!ok)) goto teardown;
+  if (__syncthreads_or(!ok)) { ok = false; goto teardown; }
   tc_fence_after();
-  if (tid == 0 && G > 1) load_v(1);   // into the Q atoms, which the MMA has finished reading
+  if (tid == 0 && G > 1) load_v(cur, 1);   // into the Q atoms, which the MMA has finished reading
 
   for (int j = 0; j < G; ++j) {
     const int h = hk * G + j;
@@ -347,18 +385,19 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
       colPk[tid] = sb[tid] * __expf(sG[tid]) * rk[tid];
       colInv[tid] = -sG[C - 1] < 60.f ? __expf(-sG[tid]) * rk[tid] : 0.f;
     }
-    if (tid == 0) tma_store_wait_read();   // the previous head's staged tiles (A, Tm regions)
+    if (tid == 0) tma_store_wait_read();   // the previous head's staged tiles (A, Tm, [P | Pk])
     __syncthreads();
 
-    // thread t < 64: row t of A from K K^T; t >= 64: row t-64 of Mqk.
+    // thread t < 64: row t of A from K K^T; t >= 64: row t-64 of Mqk, staged (swizzled) in
+    // the [P | Pk] region, which is free until the solve is done, and stored by TMA.
     // e^{G_r - G_i} = e^{G_r} e^{-G_i} with the column factors e^{-G_i}/|k_i| in shared
     // memory; when the chunk's cumulative decay could leave the fp32 range the difference
     // form is used instead (one exp per element).
+    uint8_t* mq_stage = sm + kIPP;
     {
       const int r = tid & 63;
       const float Gr = sG[r];
       const bool factored = -sG[C - 1] < 60.f;     // G is non-increasing: G_63 is the minimum
-      uint8_t* mq = ws + L.mq + (size_t)(slot * Hv + h) * kMatBytes;
       const float f = tid < 64 ? sb[r] * rk[r] : rq[r];
       const float fr = factored ? f * __expf(Gr) : f;
       uint32_t raw[2][32];
@@ -389,41 +428,53 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
           for (int e = 0; e < 32; e += 4)
             *reinterpret_cast<float4*>(Am + r * kLdA + cb * 32 + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
         } else {
-          VecIO<bf16, 32>::store(reinterpret_cast<bf16*>(mq) + r * C + cb * 32, v);
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8) {
+            float v8[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) v8[q] = v[c8 * 8 + q];
+            VecIO<bf16, 8>::store(reinterpret_cast<bf16*>(mq_stage + sw128_off(r, cb * 32 + c8 * 8)), v8);
+          }
         }
       }
+      if (tid >= 64) fence_async_smem();
     }
     __syncthreads();
+    if (tid == 0) {
+      tma_store_2d(&map_mq, 0, (int32_t)(((int64_t)slot * Hv + h) * C), mq_stage);
+      tma_store_commit();
+    }
 
     // Tm = (I + A)^{-1}. Diagonal 16x16 blocks, one warp each, by fp32 forward substitution:
     // lane j < 16 solves column j of (I + L) X = I (L the block of A, strictly lower):
     // x_i = delta_ij - sum_{k<i} L_ik x_k, accumulating each x_k into every later row as soon
-    // as it is known (a 15-step dependent chain; the L loads are warp broadcasts). Blocks
-    // above the diagonal are not stored.
+    // as it is known (a 15-step dependent chain; the L loads are warp broadcasts). The column
+    // stays in registers until it is complete, so no store to Tm sits between the loads of L.
     if (lane < 16) {
       const int b0 = warp * 16, j = lane;
-      float acc[16];
+      float acc[16], x[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) acc[i] = 0.f;
 #pragma unroll
       for (int k = 0; k < 16; ++k) {
-        const float xk = k == j ? 1.f : (k < j ? 0.f : -acc[k]);
-        Tm[(b0 + k) * kLd + b0 + j] = xk;
+        x[k] = k == j ? 1.f : (k < j ? 0.f : -acc[k]);
 #pragma unroll
-        for (int i = k + 1; i < 16; ++i) acc[i] = fmaf(Am[(b0 + i) * kLdA + b0 + k], xk, acc[i]);   // L(i, k)
+        for (int i = k + 1; i < 16; ++i) acc[i] = fmaf(Am[(b0 + i) * kLdA + b0 + k], x[k], acc[i]);   // L(i, k)
       }
+#pragma unroll
+      for (int k = 0; k < 16; ++k) Tm[(b0 + k) * kLd + b0 + j] = x[k];
     }
     __syncthreads();
-    // off-diagonal blocks by block distance: Tm_ba = -Tm_bb sum_c A_bc Tm_ca. Distance 1:
-    // one warp per block; distances 2 and 3: two warps per block, one 8-column half each
-    // (a half of the result needs only the same half of the inner sum).
+    // off-diagonal blocks by block distance: Tm_ba = -Tm_bb sum_c A_bc Tm_ca (tf32 warp MMAs).
+    // Distance 1: one warp per block; distances 2 and 3: two warps per block, one 8-column
+    // half each (a half of the result needs only the same half of the inner sum).
     for (int dist = 1; dist < 4; ++dist) {
       const int gq = lane >> 2, tq4 = lane & 3;
       if (dist == 1) {
         if (warp < 3) {
           const int aa = warp, bb = warp + 1;
           float c[2][4] = {};
-          block_mma16<false>(c, Am, kLdA, 16 * bb, 16 * aa, Tm, kLd, 16 * aa, 16 * aa, lane);
+          block_mma16(c, Am, kLdA, 16 * bb, 16 * aa, Tm, kLd, 16 * aa, 16 * aa, lane);
 #pragma unroll
           for (int nh = 0; nh < 2; ++nh) {
             scratch[gq * kLd16 + 8 * nh + 2 * tq4] = c[nh][0];
@@ -433,7 +484,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
           }
           __syncwarp();
           float d[2][4] = {};
-          block_mma16<false>(d, Tm, kLd, 16 * bb, 16 * bb, scratch, kLd16, 0, 0, lane);
+          block_mma16(d, Tm, kLd, 16 * bb, 16 * bb, scratch, kLd16, 0, 0, lane);
 #pragma unroll
           for (int nh = 0; nh < 2; ++nh) {
             float* row0 = Tm + (16 * bb + gq) * kLd + 16 * aa + 8 * nh + 2 * tq4;
@@ -459,14 +510,16 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
         row0[0] = -d[0]; row0[1] = -d[1];
         row8[0] = -d[2]; row8[1] = -d[3];
       }
+      if (dist == 3 && tid == 0) tma_store_wait_read();   // Mqk left its staging tile ([P | Pk])
       __syncthreads();
     }
 
     // [P | Pk] as bf16 K-major operands: warps 0, 1 form P, warps 2, 3 Pk. A lane takes 4
-    // columns (chunk c) of a row per step, a warp 8 rows x 4 chunks: the 16-byte Tm loads
-    // (pitch 72 floats) and the 8-byte swizzled stores are free of bank conflicts. Row scales out.
+    // columns (chunk c) of a row per step, a warp 8 rows x 4 chunks with the 8 rows on
+    // consecutive lanes; the 8-byte swizzled stores of a half warp hit 16 different words.
+    // Row scales out.
     {
-      const int m = warp >> 1, wm = warp & 1, rl = lane >> 2, cl = lane & 3;
+      const int m = warp >> 1, wm = warp & 1, rl = lane & 7, cl = lane >> 3;
       const float* fv = m == 0 ? colP : colPk;
       float4 f[4];   // column factors of this lane's chunks cg * 4 + cl
 #pragma unroll
@@ -503,7 +556,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
 
     const uint64_t dpp = smem_desc(smem_u32(sm + kIPP), 16u, 1024u);
     if (tid == 0) {   // [P; Pk] V: rows 0..63 = U~ (M = 128, N = 128, K = 64)
-      if (mbar_wait(&bar_v[j & 1], (uint32_t)(j >> 1) & 1u, err, kErrIntraTma)) {
+      if (mbar_wait(&bar_v[j & 1], ((j & 1 ? vbase1 : vbase0) + (uint32_t)(j >> 1)) & 1u, err, kErrIntraTma)) {
         tc_fence_after();
         const uint64_t dv = smem_desc(smem_u32(v_tile(j & 1)), (j & 1) ? 16384u : 8192u, 1024u);
 #pragma unroll
@@ -514,11 +567,13 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     }
     ok = mbar_wait(bar_mma, ph_mma, err, kErrIntraMma);
     ph_mma ^= 1u;
-    if (__syncthreads_or(!ok)) goto teardown;
+    if (__syncthreads_or(!ok)) { ok = false; goto teardown; }
     tc_fence_after();
-    if (tid == 0 && j + 2 < G) load_v(j + 2);   // this V buffer is free
+    if (tid == 0 && j + 2 < G) load_v(cur, j + 2);   // this V buffer is free
     // U~ (rows 0..63 of the result) -> bf16 tile [64][128] in the free A region -> TMA store
-    uint8_t* stage_u = sm + kIA;   // 2 swizzled atoms of [64][64]
+    uint8_t* stage_u = sm + kIA;   // U~: 2 swizzled atoms of [64][64]
+    uint8_t* stage_ul = sm + kIT;  // U~ - bf16(U~), in the Tm region (read for the last time
+                                   // by the [P | Pk] build)
     if (warp < 2) {
 #pragma unroll
       for (int cp = 0; cp < 4; cp += 2) {
@@ -530,12 +585,17 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
         for (int hb = 0; hb < 2; ++hb) {
           const int cb = cp + hb;
           uint8_t* atom = stage_u + (cb >> 1) * 8192;
+          uint8_t* atom_l = stage_ul + (cb >> 1) * 8192;
 #pragma unroll
           for (int c8 = 0; c8 < 4; ++c8) {
-            float v8[8];
+            uint32_t hi[4], lo[4];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) v8[q] = __uint_as_float(raw[hb][c8 * 8 + q]);
-            VecIO<bf16, 8>::store(reinterpret_cast<bf16*>(atom + sw128_off(tid, (cb & 1) * 32 + c8 * 8)), v8);
+            for (int q = 0; q < 4; ++q)
+              split_bf16x2(__uint_as_float(raw[hb][c8 * 8 + 2 * q]), __uint_as_float(raw[hb][c8 * 8 + 2 * q + 1]),
+                           hi[q], lo[q]);
+            const uint32_t off = sw128_off(tid, (cb & 1) * 32 + c8 * 8);
+            *reinterpret_cast<uint4*>(atom + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4*>(atom_l + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
           }
         }
       }
@@ -547,6 +607,9 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     if (tid == 0) {
       tma_store_2d(&map_wu, 0, wrow + C, stage_u);
       tma_store_2d(&map_wu, 64, wrow + C, stage_u + 8192);
+      const int32_t lrow = (int32_t)(((int64_t)slot * Hv + h) * C);
+      tma_store_2d(&map_ul, 0, lrow, stage_ul);
+      tma_store_2d(&map_ul, 64, lrow, stage_ul + 8192);
       tma_store_commit();
     }
     if (tid == 0) {   // [P; Pk] K: rows 64..127 = W (N = 128, K read MN-major across its atoms)
@@ -559,9 +622,16 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     }
     ok = mbar_wait(bar_mma, ph_mma, err, kErrIntraMma);
     ph_mma ^= 1u;
-    if (__syncthreads_or(!ok)) goto teardown;
+    if (__syncthreads_or(!ok)) { ok = false; goto teardown; }
     tc_fence_after();
-    uint8_t* stage_w = sm + kIT;   // -W (rows 64..127 of the result) staged in the free Tm region
+    if (j == G - 1 && has_next) {
+      // every MMA of this item has read K, Q and the V tiles: fetch the next item's inputs
+      // (its g, beta into registers, stored to shared memory once this head is done)
+      if (tid == 0) load_kqv(nxt);
+      fetch_gb(nxt);
+    }
+    uint8_t* stage_w = sm + kIPP;  // -W (rows 64..127 of the result) staged in [P | Pk], which
+                                   // the MMA that produced it has finished reading
     if (warp >= 2) {
 #pragma unroll
       for (int cp = 0; cp < 4; cp += 2) {
@@ -586,16 +656,32 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (tid == 0) {   // read out before the next head rewrites A / Tm (waited there)
+    if (tid == 0) {   // read out before the next head rewrites [P | Pk] (waited there)
       tma_store_2d(&map_wu, 0, wrow, stage_w);
       tma_store_2d(&map_wu, 64, wrow, stage_w + 8192);
       tma_store_commit();
     }
     tc_fence_before();
   }
+  vbase0 += (uint32_t)(G + 1) / 2;
+  vbase1 += (uint32_t)G / 2;
+  if (!has_next) break;
+  store_gb();   // this item's last reader of g, beta was its last head's row scales
+  cur = nxt;
+  __syncthreads();
+  }
 
 teardown:
-  if (tid == 0) tma_store_wait_all();
+  if (tid == 0) {
+    if (!ok) {   // a wait gave up: let this CTA's loads and MMAs in flight finish (bounded)
+      if (n_kq) mbar_wait(bar_tma, (n_kq - 1) & 1u, nullptr, 0);
+      if (n_v0) mbar_wait(&bar_v[0], (n_v0 - 1) & 1u, nullptr, 0);
+      if (n_v1) mbar_wait(&bar_v[1], (n_v1 - 1) & 1u, nullptr, 0);
+      mma_commit(bar_drain);
+      mbar_wait(bar_drain, 0u, nullptr, 0);
+    }
+    tma_store_wait_all();
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 256);
@@ -605,40 +691,71 @@ teardown:
 
 // shared memory of the chain kernel (offsets from a 1024-aligned base). Per stage:
 //   WQ : [-W atom0 | Q atom0 | -W atom1 | Q atom1]: [-W; Q] is one K-major 128-row operand
-//   K  : 2 atoms;  U~ (this slice) then Mqk: [U~; Mqk] is a 128-row operand whose top half
-//        only lands in rows nobody reads
-constexpr int kSWQ = 0, kSK = 32768, kSU = 49152, kSM = 57344;
-constexpr int kSVec = 65536;                  // the chunk's row scales (kVecBytes)
-constexpr int kStage = 66560;                 // one chunk (1024-aligned)
-constexpr int kStageTx = 32768 + 16384 + 8192 + 8192 + kVecBytes;   // bytes its loads deliver
+//   K  : 2 atoms
+//   U~ (this slice) then Mqk: [U~; Mqk] is a 128-row operand whose top half only lands in
+//        rows nobody reads; then the low half of U~ (this slice)
+constexpr int kSWQ = 0, kSK = 32768, kSU = 49152, kSM = 57344, kSUl = 65536;
+constexpr int kSVec = 73728;                  // the chunk's row scales (kVecBytes)
+constexpr int kStage = 74752;                 // one chunk (1024-aligned)
+constexpr int kStageTx = 32768 + 16384 + 8192 + 8192 + 8192 + kVecBytes;   // bytes its loads deliver
 constexpr int kCS = 2 * kStage;               // S0^T bf16, MN-major [128][64]: 16 KB
-constexpr int kCU = kCS + 16384;              // U   bf16 [64][64]: 8 KB
-constexpr int kCU2 = kCU + 8192;              // U'  bf16 [64][64]: 8 KB
-constexpr int kCBar = kCU2 + 8192;            // mbarriers + tmem address
-constexpr int kChainSmem = kCBar + 128 + 1024;
+constexpr int kCU = kCS + 16384;              // U   bf16 [64][64]: 8 KB (for O2)
+constexpr int kCUp = kCU + 8192;              // U' = diag(e^{G_L - G_r}/|k_r|) U as a bf16 hi + lo
+constexpr int kCUpl = kCUp + 8192;            //   pair [64][64] each (for dS): 16 KB
+constexpr int kCI = kCUpl + 8192;             // [I; 0] bf16 K-major [128][64]: 16 KB (seeds A with U~)
+constexpr int kCO = kCI + 16384;              // o staging, 2 x [64 tokens][64] bf16: 16 KB
+constexpr int kCBar = kCO + 16384;            // mbarriers + tmem address
+constexpr int kChainSmem = kCBar + 256 + 1024;
 // warps 0..7 compute, 8 and 9 issue MMAs, 10 issues the TMA loads
 constexpr int kComputeWarps = 8;
 constexpr int kChainThreads = (kComputeWarps + 3) * 32;
+constexpr int kOBarrier = 1;                  // named barrier of the four output warps
 
 // TMEM columns (M = 128 accumulators, lane = row). A = [-W; Q] S0^T is accumulated in two
-// K halves (lo: dk 0..63, hi: dk 64..127) by the two issuers, each double-buffered; dS^T in
-// two K halves (tokens 0..31, 32..63); O2 = [U~; Mqk] U.
+// K halves (lo: dk 0..63, hi: dk 64..127) by the two issuers, each double-buffered; the lo
+// half starts from [I; 0] U~, so its rows 0..63 plus the hi half's are U itself. dS^T in two
+// K halves (tokens 0..31, 32..63); O2 = [U~; Mqk] U.
 constexpr uint32_t kTAlo = 0, kTAhi = 128, kTdSlo = 256, kTdShi = 320, kTO2 = 384;
 
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+// Barrier over `threads` threads that also returns whether any of them passed `pred`.
+__device__ __forceinline__ bool named_bar_or(int id, int threads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n"
+      " bar.red.or.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r) : "r"((uint32_t)pred), "r"(id), "r"(threads) : "memory");
+  return r != 0;
+}
+// Wait until at most one committed bulk store group of this thread still reads shared memory.
+__device__ __forceinline__ void tma_store_wait_read_le1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
 // One chain CTA: sequence n, value head h, dv rows [tile*64, tile*64 + 64). Per chunk c:
-//   issuers : rA(c) = [-W; Q] S0^T (after "S ready"), rB(c) = K^T U', rO(c) = [U~; Mqk] U
-//             (after "U ready")
-//   compute : U = U~ + rows 0..63 of rA -> U, U' (warps of quadrants 0, 1)      -> "U ready"
+//   issuers : rA(c) = [-W; Q] S0^T in two K halves (dk rows 0..63 after the state warps of
+//             quadrants 0, 1 are done, 64..127 after quadrants 2, 3), the lo half on top of
+//             [I; 0] U~ (issued as soon as the stage lands, off the serial path);
+//             dS^T = K^T U' in two token halves (each after the U warps of its quadrant; U'
+//             is carried as a bf16 hi + lo pair on the state path, where a chunk that
+//             rewrites one key telescopes U's rows); O2 = [U~; Mqk] U after both (issued by
+//             the second issuer behind its dS half)
+//   compute : U = rows 0..63 of rA -> U (bf16), U' (hi + lo) (quadrants 0, 1)   -> "U ready"
 //             S^T <- e^{G_L} S^T + dS^T, bf16 copy (all 8 warps)               -> "S ready"
-//             o = scale (e^{G_r}/|q_r| rows 64..127 of rA + O2) (quadrants 2, 3) -> "stage free"
-//   producer: chunk c+2's loads into stage c % 2 once it is free.
-// The serial path is rA -> U -> rB -> S -> rA(c+1); no thread on it issues anything else.
+//             o = scale (e^{G_r}/|q_r| rows 64..127 of rA + O2) (quadrants 2, 3): a full
+//             chunk is staged in shared memory and leaves by one TMA store     -> "stage free"
+//   producer: chunk c+2's loads into stage c % 2 once it is free; chunk c+1's seed of A-lo
+//             once its stage has landed
+// The serial path is rA -> U -> dS -> S -> rA(c+1); no thread on it issues anything else.
 __global__ void __launch_bounds__(kChainThreads, 1)
 chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                    const __grid_constant__ CUtensorMap map_wu, const __grid_constant__ CUtensorMap map_mq,
+                   const __grid_constant__ CUtensorMap map_ul, const __grid_constant__ CUtensorMap map_o,
                    const int32_t* __restrict__ cu, int32_t n_seq, int64_t T, int32_t Hk, int32_t Hv,
-                   const uint8_t* __restrict__ ws_ro, int* err_word, const float* init, float* fin,
-                   bf16* __restrict__ o, float scale, BlockStates blocks) {
+                   const uint8_t* __restrict__ ws_ro, int* err_word, const void* init, void* fin,
+                   int state_bf16, bf16* __restrict__ o, float scale, BlockStates blocks) {
   const Ws L = ws_layout(T, n_seq, Hv);
   const int32_t* prefix = reinterpret_cast<const int32_t*>(ws_ro + L.prefix);
   const int tile = blockIdx.x % NT;
@@ -646,6 +763,7 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
   const int32_t n = blockIdx.x / (NT * Hv);
   const int hk = h / (Hv / Hk);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const bool sbf = state_bf16 != 0;
   int64_t bos, eos;
   seq_bounds(cu, n, T, bos, eos);
   const int nc = (int)((eos - bos + C - 1) / C);
@@ -661,17 +779,38 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
   uint64_t* bar_B0 = bars + 6;
   uint64_t* bar_B1 = bars + 7;
   uint64_t* bar_O = bars + 8;
-  uint64_t* bar_U = bars + 9;      // U, U' written (8 compute warps)
-  uint64_t* bar_S = bars + 10;     // state bf16 written (8 compute warps)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+  uint64_t* bar_U0 = bars + 9;     // U, U' rows 0..31 written (the 2 warps of quadrant 0)
+  uint64_t* bar_U1 = bars + 10;    // rows 32..63 (quadrant 1)
+  uint64_t* bar_S0 = bars + 11;    // state bf16 rows 0..63 written (quadrants 0, 1: 4 warps)
+  uint64_t* bar_S1 = bars + 12;    // rows 64..127 (quadrants 2, 3)
+  uint64_t* bar_drain = bars + 15; // [3] on an early exit: each issuing thread's MMAs have completed
+  uint64_t* bar_seed = bars + 18;  // [2] A-lo buffer b holds [I; 0] (U~ + U~lo) of its next chunk
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
 
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) { mbar_init(&bar_tma[i], 1); mbar_init(&bar_free[i], kComputeWarps); }
     for (int i = 4; i < 9; ++i) mbar_init(&bars[i], 1);
-    mbar_init(bar_U, kComputeWarps);
-    mbar_init(bar_S, kComputeWarps);
+    mbar_init(bar_U0, 2);
+    mbar_init(bar_U1, 2);
+    mbar_init(bar_S0, 4);
+    mbar_init(bar_S1, 4);
+    for (int i = 0; i < 3; ++i) mbar_init(&bar_drain[i], 1);
+    mbar_init(&bar_seed[0], 1);
+    mbar_init(&bar_seed[1], 1);
     fence_mbar_init();
   }
+  // [I; 0]: rows 0..63 the identity, rows 64..127 zero (K-major, 128-byte swizzle)
+  for (int e = tid; e < 128 * 8; e += kChainThreads) {
+    const int r = e >> 3, c8 = e & 7;
+    uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    if (r < 64 && (r >> 3) == c8) {
+      const uint32_t one = 0x3F80u << (16 * (r & 1));   // bf16 1.0 in the low or high half
+      const int w = (r & 7) >> 1;
+      if (w == 0) z.x = one; else if (w == 1) z.y = one; else if (w == 2) z.z = one; else z.w = one;
+    }
+    *reinterpret_cast<uint4*>(sm + kCI + sw128_off(r, c8 * 8)) = z;
+  }
+  fence_async_smem();
   if (warp == 0) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
@@ -686,11 +825,18 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     auto soff = [](int b) { return (uint64_t)(b * (kStage >> 4)); };
     const uint64_t dS = smem_desc(smem_u32(sm + kCS), 8192u, 1024u);
     const uint64_t dU = smem_desc(smem_u32(sm + kCU), 8192u, 1024u);
-    const uint64_t dU2 = smem_desc(smem_u32(sm + kCU2), 8192u, 1024u);
+    const uint64_t dUp = smem_desc(smem_u32(sm + kCUp), 8192u, 1024u);
+    const uint64_t dUpl = smem_desc(smem_u32(sm + kCUpl), 8192u, 1024u);
+    const uint64_t dI = smem_desc(smem_u32(sm + kCI), 16u, 1024u);
     constexpr uint32_t kIA = idesc_bf16(128, DT, 0, 1);     // K-major A, MN-major B
     constexpr uint32_t kIB = idesc_bf16(128, DT, 1, 1);     // MN-major A and B
-    if (warp == kComputeWarps + 2) {   // TMA producer
-      if (nc > 0) tma_prefetch_desc(&map_q);
+    const uint64_t dUt = smem_desc(st0 + kSU, 8192u, 1024u);    // U~ as an MN-major B operand
+    const uint64_t dUtl = smem_desc(st0 + kSUl, 8192u, 1024u);  // and its low half
+    if (warp == kComputeWarps + 2) {
+      // TMA producer. Once a chunk's stage has landed and its A-lo buffer's previous chunk is
+      // done, it also seeds that buffer with [I; 0] (U~ + U~lo) (rows 0..63 = U~, rows
+      // 64..127 = 0), off the issuers' serial path.
+      tma_prefetch_desc(&map_q);
       auto issue_loads = [&](int c, int b) {
         const int64_t t0 = bos + (int64_t)c * C;
         const int32_t slot = slot0 + c;
@@ -704,17 +850,49 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
         }
         tma_load_2d(stg + kSU, &map_wu, tile * DT, wrow + C, &bar_tma[b]);
         tma_load_2d(stg + kSM, &map_mq, 0, (int32_t)(((int64_t)slot * Hv + h) * C), &bar_tma[b]);
+        tma_load_2d(stg + kSUl, &map_ul, tile * DT, (int32_t)(((int64_t)slot * Hv + h) * C), &bar_tma[b]);
         bulk_load(stg + kSVec, ws_ro + L.vecs + ((size_t)slot * Hv + h) * kVecBytes, kVecBytes, &bar_tma[b]);
+      };
+      auto seed = [&](int c) {   // chunk c's stage has landed and its A-lo buffer is free
+        const int b = c & 1;
+        const uint32_t ta = tmem + kTAlo + 64 * b;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) mma_bf16(ta, dI + 2 * kk, dUt + soff(b) + 128 * kk, kIA, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) mma_bf16(ta, dI + 2 * kk, dUtl + soff(b) + 128 * kk, kIA, true);
+        mma_commit(&bar_seed[b]);
       };
       issue_loads(0, 0);
       if (nc > 1) issue_loads(1, 1);
-      for (int c = 0; c + 2 < nc; ++c) {
-        if (!mbar_wait(&bar_free[c & 1], (uint32_t)(c >> 1) & 1u, err_word, kErrChainTma)) break;
-        issue_loads(c + 2, c & 1);
+      int c = 0, issued = nc > 1 ? 2 : 1;
+      bool good = mbar_wait(&bar_tma[0], 0u, err_word, kErrChainTma);
+      if (good) seed(0);
+      for (; good && c < nc; ++c) {
+        // chunk c + 1's seed: its stage; its buffer was last used by chunk c - 1, whose stage
+        // release was awaited before chunk c + 1's loads were issued
+        if (c + 1 < nc) {
+          if (!(good = mbar_wait(&bar_tma[(c + 1) & 1], (uint32_t)((c + 1) >> 1) & 1u, err_word, kErrChainTma))) break;
+          seed(c + 1);
+        }
+        if (c + 2 < nc) {
+          if (!(good = mbar_wait(&bar_free[c & 1], (uint32_t)(c >> 1) & 1u, err_word, kErrChainTma))) break;
+          issue_loads(c + 2, c & 1);
+          issued = c + 3;
+        }
       }
+      if (!good) {   // gave up: let the loads in flight land (bounded) before exiting
+        for (int b = 0; b < 2 && b < issued; ++b) {   // the last chunk loaded into stage b
+          const int last = (issued - 1) - (((issued - 1) - b) & 1);
+          mbar_wait(&bar_tma[b], (uint32_t)(last >> 1) & 1u, nullptr, 0);
+        }
+      }
+      mma_commit(&bar_drain[2]);   // every seed MMA has completed before TMEM is released
+      mbar_wait(&bar_drain[2], 0u, nullptr, 0);
       goto done;
     }
-    const int part = warp - kComputeWarps;   // 0: lo halves and O2, 1: hi halves
+    const int part = warp - kComputeWarps;   // 0: lo halves, 1: hi halves and O2
+    uint64_t* bar_Sp = part ? bar_S1 : bar_S0;
     const uint64_t dWQ = smem_desc(st0 + kSWQ, 16u, 1024u) + (uint64_t)(part * (16384 >> 4));
     const uint64_t dK = smem_desc(st0 + kSK, 8192u, 1024u);
     const uint64_t dUM = smem_desc(st0 + kSU, 16u, 1024u);
@@ -722,38 +900,46 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
       const uint32_t ta = tmem + (part ? kTAhi : kTAlo) + 64 * b;
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(ta, dWQ + soff(b) + 2 * kk, dS + 128 * (4 * part + kk), kIA, kk > 0);
+        mma_bf16(ta, dWQ + soff(b) + 2 * kk, dS + 128 * (4 * part + kk), kIA, part == 0 || kk > 0);
       mma_commit(part ? bar_A1 : bar_A0);
     };
-    uint32_t phT[2] = {0u, 0u};
-    // rA(0): chunk 0 landed and the initial state is in shared memory
-    if (!mbar_wait(&bar_tma[0], phT[0], err_word, kErrChainTma) ||
-        !mbar_wait(bar_S, 0u, err_word, kErrChainMma)) goto done;
-    phT[0] ^= 1u;
+    // rA(0): chunk 0 landed (and, for the lo half, was seeded) and this half of the initial
+    // state is in shared memory
+    if (!mbar_spin(&bar_tma[0], 0u, err_word, kErrChainTma) ||
+        (part == 0 && !mbar_spin(&bar_seed[0], 0u, err_word, kErrChainMma)) ||
+        !mbar_spin(bar_Sp, 0u, err_word, kErrChainMma)) goto done;
     tc_fence_after();
     issue_rA(0);
     for (int c = 0; c < nc; ++c) {
       const int b = c & 1;
-      if (!mbar_wait(bar_U, (uint32_t)c & 1u, err_word, kErrChainMma)) break;
+      if (!mbar_spin(part ? bar_U1 : bar_U0, (uint32_t)c & 1u, err_word, kErrChainMma)) break;
       tc_fence_after();
 #pragma unroll
-      for (int kk = 0; kk < 2; ++kk)   // dS^T = K^T U' over tokens [32 part, 32 part + 32)
+      for (int kk = 0; kk < 2; ++kk) {   // dS^T = K^T (U' + U'lo) over tokens [32 part, 32 part + 32)
         mma_bf16(tmem + (part ? kTdShi : kTdSlo), dK + soff(b) + 128 * (2 * part + kk),
-                 dU2 + 128 * (2 * part + kk), kIB, kk > 0);
+                 dUp + 128 * (2 * part + kk), kIB, kk > 0);
+        mma_bf16(tmem + (part ? kTdShi : kTdSlo), dK + soff(b) + 128 * (2 * part + kk),
+                 dUpl + 128 * (2 * part + kk), kIB, true);
+      }
       mma_commit(part ? bar_B1 : bar_B0);
-      if (part == 0) {   // rows 64..127 of [U~; Mqk] U
+      if (part == 1) {   // rows 64..127 of [U~; Mqk] U, once all of U is written
+        if (!mbar_spin(bar_U0, (uint32_t)c & 1u, err_word, kErrChainMma)) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) mma_bf16(tmem + kTO2, dUM + soff(b) + 2 * kk, dU + 128 * kk, kIA, kk > 0);
         mma_commit(bar_O);
       }
       if (c + 1 < nc) {
-        if (!mbar_wait(&bar_tma[b ^ 1], phT[b ^ 1], err_word, kErrChainTma) ||
-            !mbar_wait(bar_S, (uint32_t)(c + 1) & 1u, err_word, kErrChainMma)) break;
-        phT[b ^ 1] ^= 1u;
+        if (!mbar_spin(&bar_tma[b ^ 1], (uint32_t)((c + 1) >> 1) & 1u, err_word, kErrChainTma) ||
+            (part == 0 && !mbar_spin(&bar_seed[b ^ 1], (uint32_t)((c + 1) >> 1) & 1u, err_word, kErrChainMma)) ||
+            !mbar_spin(bar_Sp, (uint32_t)(c + 1) & 1u, err_word, kErrChainMma)) break;
         tc_fence_after();
         issue_rA(b ^ 1);
       }
     }
+    // every MMA this thread issued has completed before the tensor memory is released
+    mma_commit(&bar_drain[part]);
+    mbar_wait(&bar_drain[part], 0u, nullptr, 0);
     goto done;
   }
 
@@ -762,13 +948,14 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     const int quad = warp & 3, half = warp >> 2;     // TMEM lanes 32 quad.., column half
     const int lrow = quad * 32 + lane;               // this thread's accumulator row (lane)
     const uint32_t tq = tmem_quadrant(tmem, quad);
+    uint64_t* bar_Sq = quad < 2 ? bar_S0 : bar_S1;
 
     // state slice: thread (lrow, half) holds S[tile*64 + half*32 + j][lrow], j < 32
     constexpr int SJ = DT / 2;
     float s[SJ];
     const int64_t sbase = ((int64_t)n * Hv + h) * D * D + (int64_t)(tile * DT + half * SJ) * D + lrow;
 #pragma unroll
-    for (int j = 0; j < SJ; ++j) s[j] = init ? init[sbase + (int64_t)j * D] : 0.f;
+    for (int j = 0; j < SJ; ++j) s[j] = init ? state_load(init, sbase + (int64_t)j * D, sbf) : 0.f;
     auto store_state_bf16 = [&]() {
 #pragma unroll
       for (int c8 = 0; c8 < SJ / 8; ++c8) {
@@ -784,7 +971,7 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     };
     store_state_bf16();
     fence_async_smem();
-    warp_arrive(bar_S);
+    warp_arrive(bar_Sq);
 
     uint32_t phA = 0u, phB = 0u;
     for (int c = 0; c < nc; ++c) {
@@ -799,41 +986,36 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
       tc_fence_after();
       float os = 0.f;
       if (quad < 2) {
-        // U is free: its last reader, O2 of chunk c - 1, was issued before rA_lo(c) by the
-        // same thread, and that thread's commit of rA_lo(c) tracks every MMA it issued before
+        // U is free: its last reader, O2 of chunk c - 1, was issued before rA_hi(c) by the
+        // same thread, and that thread's commit of rA_hi(c) tracks every MMA it issued before
         const int r = lrow;
         const float us = vec[64 + r];
         uint32_t a0[32], a1[32];
         tmem_ld32_async(tq + kTAlo + 64 * b + half * 32, a0);
         tmem_ld32_async(tq + kTAhi + 64 * b + half * 32, a1);
-        const uint8_t* ut = sm + b * kStage + kSU;
-        float ub[32];
-#pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8) {
-          float v8[8];
-          VecIO<bf16, 8>::load(reinterpret_cast<const bf16*>(ut + sw128_off(r, half * 32 + c8 * 8)), v8);
-#pragma unroll
-          for (int q = 0; q < 8; ++q) ub[c8 * 8 + q] = v8[q];
-        }
         tmem_wait_ld(a0, a1);
 #pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8) {
-          float v8[8], w8[8];
+        for (int c8 = 0; c8 < 4; ++c8) {   // U in bf16; U' as a hi + lo bf16 pair
+          uint32_t u[4], hi[4], lo[4];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            v8[q] = ub[c8 * 8 + q] + __uint_as_float(a0[c8 * 8 + q]) + __uint_as_float(a1[c8 * 8 + q]);
-            w8[q] = us * v8[q];
+          for (int q = 0; q < 4; ++q) {
+            const float x0 = __uint_as_float(a0[c8 * 8 + 2 * q]) + __uint_as_float(a1[c8 * 8 + 2 * q]);
+            const float x1 = __uint_as_float(a0[c8 * 8 + 2 * q + 1]) + __uint_as_float(a1[c8 * 8 + 2 * q + 1]);
+            __nv_bfloat162 ub = __floats2bfloat162_rn(x0, x1);
+            u[q] = *reinterpret_cast<uint32_t*>(&ub);
+            split_bf16x2(us * x0, us * x1, hi[q], lo[q]);
           }
           const uint32_t off = sw128_off(r, half * 32 + c8 * 8);
-          VecIO<bf16, 8>::store(reinterpret_cast<bf16*>(sm + kCU + off), v8);
-          VecIO<bf16, 8>::store(reinterpret_cast<bf16*>(sm + kCU2 + off), w8);
+          *reinterpret_cast<uint4*>(sm + kCU + off) = make_uint4(u[0], u[1], u[2], u[3]);
+          *reinterpret_cast<uint4*>(sm + kCUp + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4*>(sm + kCUpl + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
         fence_async_smem();
+        tc_fence_before();
+        warp_arrive(quad == 0 ? bar_U0 : bar_U1);
       } else {
         os = vec[lrow - 64];
       }
-      tc_fence_before();
-      warp_arrive(bar_U);
 
       // state update: S^T <- e^{G_L} S^T + dS^T (both K halves)
       if (!(ok = mbar_wait(bar_B0, phB, err_word, kErrChainMma) && mbar_wait(bar_B1, phB, err_word, kErrChainMma))) break;
@@ -850,22 +1032,25 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
           s[e] = fmaf(decay_last, s[e], __uint_as_float(d0[e]) + __uint_as_float(d1[e]));
         store_state_bf16();
       }
+      fence_async_smem();
+      tc_fence_before();
+      warp_arrive(bar_Sq);
       // the state after a full chunk that ends a block of the sequence (prefix caching)
       if (blocks.block_tokens > 0 && len == C && ((int64_t)(c + 1) * C) % blocks.block_tokens == 0) {
         const int64_t brow = (int64_t)blocks.rows[n] + (int64_t)(c + 1) * C / blocks.block_tokens - 1;
         if (brow >= 0 && brow < blocks.n_rows) {
-          float* dst = blocks.states + ((brow * Hv + h) * D + tile * DT + half * SJ) * (int64_t)D + lrow;
+          const int64_t dst = ((brow * Hv + h) * D + tile * DT + half * SJ) * (int64_t)D + lrow;
 #pragma unroll
-          for (int j = 0; j < SJ; ++j) dst[(int64_t)j * D] = s[j];
+          for (int j = 0; j < SJ; ++j) state_store(blocks.states, dst + (int64_t)j * D, s[j], sbf);
         }
       }
-      fence_async_smem();
-      tc_fence_before();
-      warp_arrive(bar_S);
 
       // chunk c's output (quadrants 2, 3): o_r = scale (e^{G_r}/|q_r| O1_r + O2_r)
       if (quad >= 2) {
-        if (!(ok = mbar_wait(bar_O, (uint32_t)c & 1u, err_word, kErrChainMma))) break;
+        const bool got = mbar_wait(bar_O, (uint32_t)c & 1u, err_word, kErrChainMma);
+        // all four output warps leave together if any wait gave up; this barrier also
+        // orders this chunk's staging writes after the read of the store from two chunks ago
+        if (named_bar_or(kOBarrier, 128, !got)) { ok = false; break; }
         tc_fence_after();
         const int r = lrow - 64;
         uint32_t a0[32], a1[32];
@@ -878,7 +1063,23 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
         uint32_t o2[32];
         tmem_ld32_async(tq + kTO2 + half * 32, o2);
         tmem_wait_ld(o2);
-        if (r < len) {
+        if (len == C) {   // a full chunk: stage the 64 x 64 tile, one TMA store
+          uint8_t* ost = sm + kCO + b * 8192;
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8) {
+            float v8[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) v8[q] = scale * (o1[c8 * 8 + q] + __uint_as_float(o2[c8 * 8 + q]));
+            VecIO<bf16, 8>::store(reinterpret_cast<bf16*>(ost + sw128_off(r, half * 32 + c8 * 8)), v8);
+          }
+          fence_async_smem();
+          named_bar_sync(kOBarrier, 128);
+          if (warp == 2 && lane == 0) {
+            tma_store_2d(&map_o, h * D + tile * DT, (int32_t)t0, ost);
+            tma_store_commit();
+            tma_store_wait_read_le1();   // the other staging buffer may be written next chunk
+          }
+        } else if (r < len) {   // the ragged end of a sequence: rows past it belong to the next
           bf16* dst = o + ((t0 + r) * Hv + h) * (int64_t)D + tile * DT + half * 32;
 #pragma unroll
           for (int c8 = 0; c8 < 4; ++c8) {
@@ -892,9 +1093,10 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
       }
       warp_arrive(&bar_free[b]);
     }
+    if (warp == 2 && lane == 0) tma_store_wait_all();
     if (ok && fin != nullptr) {
 #pragma unroll
-      for (int j = 0; j < SJ; ++j) fin[sbase + (int64_t)j * D] = s[j];
+      for (int j = 0; j < SJ; ++j) state_store(fin, sbase + (int64_t)j * D, s[j], sbf);
     }
   }
 
@@ -955,12 +1157,20 @@ size_t prefill_chunk_tc_workspace(int64_t T, int32_t n_seq, int32_t Hv) {
 cudaError_t launch_prefill_chunk_tc(const void* q, const void* k, const void* v, const float* g,
                                     const float* beta, void* o, int64_t T, int32_t Hk, int32_t Hv,
                                     int64_t qk_stride, int64_t v_stride, const int32_t* cu,
-                                    int32_t n_seq, const float* init, float* fin, float scale,
-                                    BlockStates blocks, void* workspace, cudaStream_t stream) {
+                                    int32_t n_seq, const void* init, void* fin, int state_dtype,
+                                    float scale, BlockStates blocks, void* workspace,
+                                    cudaStream_t stream) {
   static uint64_t attrs_set = 0;   // one bit per device that has the smem attributes
+  static int sm_count[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  int num_sms = dev < 64 ? sm_count[dev] : 0;
+  if (num_sms == 0) {
+    e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 64) sm_count[dev] = num_sms;
+  }
   if (dev >= 64 || !(attrs_set >> dev & 1)) {
     e = cudaFuncSetAttribute(chunk_intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kIntraSmem);
     if (e != cudaSuccess) return e;
@@ -973,23 +1183,27 @@ cudaError_t launch_prefill_chunk_tc(const void* q, const void* k, const void* v,
   const int64_t slots = max_slots(T, n_seq);
   // with no tokens every sequence is empty: the chain kernel only copies the states and
   // never touches the maps, which are left zeroed
-  CUtensorMap mq{}, mk{}, mv{}, mwu{}, mmq{};
+  CUtensorMap mq{}, mk{}, mv{}, mwu{}, mmq{}, mul{}, mo{};
   if (T > 0 && (!make_map(&mq, q, (uint64_t)Hk * D, (uint64_t)T, (uint64_t)qk_stride) ||
                 !make_map(&mk, k, (uint64_t)Hk * D, (uint64_t)T, (uint64_t)qk_stride) ||
                 !make_map(&mv, v, (uint64_t)Hv * D, (uint64_t)T, (uint64_t)v_stride) ||
                 !make_map(&mwu, ws + L.wu, D, (uint64_t)slots * Hv * 2 * C, D) ||
-                !make_map(&mmq, ws + L.mq, C, (uint64_t)slots * Hv * C, C)))
+                !make_map(&mmq, ws + L.mq, C, (uint64_t)slots * Hv * C, C) ||
+                !make_map(&mul, ws + L.ul, D, (uint64_t)slots * Hv * C, D) ||
+                !make_map(&mo, o, (uint64_t)Hv * D, (uint64_t)T, (uint64_t)Hv * D)))
     return cudaErrorInvalidValue;
   chunk_plan_kernel<<<1, 1024, 0, stream>>>(cu, n_seq, T, reinterpret_cast<int32_t*>(ws + L.prefix),
                                             reinterpret_cast<int*>(ws + L.err));
-  if (T > 0) {
-    dim3 gi((unsigned)slots, (unsigned)Hk);
-    chunk_intra_kernel<<<gi, 128, kIntraSmem, stream>>>(mq, mk, mv, mwu, g, beta, cu, n_seq, T, Hk, Hv, ws);
+  if (T > 0) {   // persistent: two CTAs per SM (shared memory and tensor memory allow two)
+    const int64_t items = slots * Hk;
+    const int64_t grid = items < 2 * (int64_t)num_sms ? items : 2 * (int64_t)num_sms;
+    chunk_intra_kernel<<<(unsigned)grid, 128, kIntraSmem, stream>>>(mq, mk, mv, mwu, mmq, mul, g, beta,
+                                                                    cu, n_seq, T, Hk, Hv, ws);
   }
   dim3 gc((unsigned)((int64_t)n_seq * Hv * NT));
-  chunk_chain_kernel<<<gc, kChainThreads, kChainSmem, stream>>>(mq, mk, mwu, mmq, cu, n_seq, T, Hk, Hv, ws,
-                                                              reinterpret_cast<int*>(ws + L.err), init, fin,
-                                                              static_cast<bf16*>(o), scale, blocks);
+  chunk_chain_kernel<<<gc, kChainThreads, kChainSmem, stream>>>(
+      mq, mk, mwu, mmq, mul, mo, cu, n_seq, T, Hk, Hv, ws, reinterpret_cast<int*>(ws + L.err), init, fin,
+      state_dtype == kBF16 ? 1 : 0, static_cast<bf16*>(o), scale, blocks);
   return cudaGetLastError();
 }
 

@@ -13,7 +13,7 @@
 // device with cudaGetSymbolAddress (with that device current) and cached.
 #include <mutex>
 
-#include "../../include/gdn.h"
+#include "gdn.h"
 #include "launch.h"
 
 namespace {
@@ -50,24 +50,20 @@ extern "C" gdn_status_t gdn_chunk_prefill_noalloc(
     gdn_dtype_t dt, int64_t T, int32_t Hk, int32_t Hv, int32_t dk, int32_t dv, int64_t qk_stride,
     int64_t v_stride, const int32_t* cu_seqlens, int32_t n_seq, const float* initial_state,
     float* final_state, float scale, int32_t qk_l2norm, gdn_stream_t stream) {
-  const size_t need = gdn_chunk_prefill_workspace_size(T, cu_seqlens ? n_seq : 1, Hk, Hv, dk, dv, dt);
-  if (need == SIZE_MAX || need == 0) {
-    // unsupported shapes get the regular validation and status; shapes that need no
-    // scratch run the regular path directly
-    return gdn_chunk_prefill(q, k, v, g, beta, o, dt, T, Hk, Hv, dk, dv, qk_stride, v_stride,
-                             cu_seqlens, n_seq, initial_state, final_state, scale, qk_l2norm,
-                             nullptr, 0, stream);
-  }
-  if (need > kNoallocScratchBytes) {
-    // the regular entry point reports the size in gdn_last_error(); call it with no
-    // workspace so that it fails validation without launching anything
-    gdn_status_t s = gdn_chunk_prefill(q, k, v, g, beta, o, dt, T, Hk, Hv, dk, dv, qk_stride,
-                                       v_stride, cu_seqlens, n_seq, initial_state, final_state,
-                                       scale, qk_l2norm, nullptr, kNoallocScratchBytes, stream);
-    return s == GDN_OK ? GDN_ERR_WORKSPACE : s;
-  }
+  // the scratch the path taken by these arguments needs (0 for the token-recurrent path;
+  // SIZE_MAX for unsupported arguments, which the regular validation below reports)
+  const size_t need = gdn::prefill_workspace_need(dt, T, cu_seqlens ? n_seq : 1, Hk, Hv, dk, dv,
+                                                  qk_l2norm);
+  if (need != SIZE_MAX && need > kNoallocScratchBytes)
+    return gdn::set_error(GDN_ERR_WORKSPACE,
+                          "chunk_prefill_noalloc: these sizes need %zu bytes of scratch, more than "
+                          "the %zu-byte static array; nothing was launched (split the batch, or "
+                          "use gdn_chunk_prefill with a workspace)", need, kNoallocScratchBytes);
   void* scratch = nullptr;
-  if (scratch_for_current_device(&scratch) != cudaSuccess) return GDN_ERR_CUDA;
+  const cudaError_t e = scratch_for_current_device(&scratch);
+  if (e != cudaSuccess)
+    return gdn::set_error(GDN_ERR_CUDA, "chunk_prefill_noalloc: scratch address: %s", cudaGetErrorString(e));
+  // always hand over the scratch, so that every path clears its status word
   return gdn_chunk_prefill(q, k, v, g, beta, o, dt, T, Hk, Hv, dk, dv, qk_stride, v_stride,
                            cu_seqlens, n_seq, initial_state, final_state, scale, qk_l2norm,
                            scratch, kNoallocScratchBytes, stream);
@@ -75,6 +71,8 @@ extern "C" gdn_status_t gdn_chunk_prefill_noalloc(
 
 extern "C" gdn_status_t gdn_prefill_noalloc_status(gdn_stream_t stream) {
   void* scratch = nullptr;
-  if (scratch_for_current_device(&scratch) != cudaSuccess) return GDN_ERR_CUDA;
+  const cudaError_t e = scratch_for_current_device(&scratch);
+  if (e != cudaSuccess)
+    return gdn::set_error(GDN_ERR_CUDA, "prefill_noalloc_status: scratch address: %s", cudaGetErrorString(e));
   return gdn_prefill_status(scratch, stream);
 }

@@ -11,7 +11,8 @@
 // beta_t, and performs one warp reduction of 3 + 2 kRows values:
 //   |q|^2, |k|^2, k.q and, per row, s.k and s.q (un-normalised; scaled after),
 // then u = beta (v_i - alpha s.k^), s <- alpha s + u k^, o_i = scale (alpha s.q^ + u k^.q^).
-// Optionally the rows are also stored after every block_tokens tokens (block states).
+// Optionally the rows are also stored after every block_tokens tokens (block states). States
+// in HBM are fp32 or bf16 storage (the arithmetic is fp32 either way).
 #include "common.cuh"
 #include "launch.h"
 
@@ -28,8 +29,8 @@ prefill_recurrent_kernel(const T* __restrict__ q, const T* __restrict__ k,
                          const T* __restrict__ v, const float* __restrict__ g,
                          const float* __restrict__ beta, T* __restrict__ o, int64_t T_tok,
                          int32_t Hk, int32_t Hv, int64_t qk_stride, int64_t v_stride,
-                         const int32_t* __restrict__ cu, const float* init, float* fin,
-                         float scale, int32_t l2norm, BlockStates blocks) {
+                         const int32_t* __restrict__ cu, const void* init, void* fin,
+                         int32_t state_bf16, float scale, int32_t l2norm, BlockStates blocks) {
   constexpr int VEC = D >= 32 ? D / 32 : 1;
   constexpr int kRowsPerCta = kWarps * kRows;
   constexpr int kRowBlocks = (D + kRowsPerCta - 1) / kRowsPerCta;
@@ -40,6 +41,7 @@ prefill_recurrent_kernel(const T* __restrict__ q, const T* __restrict__ k,
   const int hk = h / (Hv / Hk);
   const int row0 = rb * kRowsPerCta + warp * kRows;
   const bool active = lane * VEC < D;
+  const bool sbf = state_bf16 != 0;
 
   int64_t bos, eos;
   seq_bounds(cu, n, T_tok, bos, eos);
@@ -51,7 +53,7 @@ prefill_recurrent_kernel(const T* __restrict__ q, const T* __restrict__ k,
 #pragma unroll
     for (int j = 0; j < VEC; ++j) {
       const int row = row0 + r, col = lane * VEC + j;
-      s[r][j] = (init != nullptr && row < D && active) ? init[sbase + (int64_t)row * D + col] : 0.f;
+      s[r][j] = (init != nullptr && row < D && active) ? state_load(init, sbase + (int64_t)row * D + col, sbf) : 0.f;
     }
 
   for (int64_t t = bos; t < eos; ++t) {
@@ -112,13 +114,13 @@ prefill_recurrent_kernel(const T* __restrict__ q, const T* __restrict__ k,
     if (blocks.block_tokens > 0 && done % blocks.block_tokens == 0) {
       const int64_t brow = (int64_t)blocks.rows[n] + done / blocks.block_tokens - 1;
       if (brow >= 0 && brow < blocks.n_rows) {
-        float* dst = blocks.states + (brow * Hv + h) * D * D;
+        const int64_t dst = (brow * Hv + h) * D * D;
 #pragma unroll
         for (int r = 0; r < kRows; ++r)
 #pragma unroll
           for (int j = 0; j < VEC; ++j) {
             const int row = row0 + r, col = lane * VEC + j;
-            if (row < D && active) dst[(int64_t)row * D + col] = s[r][j];
+            if (row < D && active) state_store(blocks.states, dst + (int64_t)row * D + col, s[r][j], sbf);
           }
       }
     }
@@ -130,7 +132,7 @@ prefill_recurrent_kernel(const T* __restrict__ q, const T* __restrict__ k,
 #pragma unroll
       for (int j = 0; j < VEC; ++j) {
         const int row = row0 + r, col = lane * VEC + j;
-        if (row < D && active) fin[sbase + (int64_t)row * D + col] = s[r][j];
+        if (row < D && active) state_store(fin, sbase + (int64_t)row * D + col, s[r][j], sbf);
       }
   }
 }
@@ -139,26 +141,26 @@ template <typename T, int D>
 cudaError_t launch_typed(const void* q, const void* k, const void* v, const float* g,
                          const float* beta, void* o, int64_t n_tok, int32_t Hk, int32_t Hv,
                          int64_t qks, int64_t vs, const int32_t* cu, int32_t n_seq,
-                         const float* init, float* fin, float scale, int32_t l2, BlockStates bl,
-                         cudaStream_t st) {
+                         const void* init, void* fin, int32_t sbf, float scale, int32_t l2,
+                         BlockStates bl, cudaStream_t st) {
   constexpr int kRowBlocks = (D + kWarps * kRows - 1) / (kWarps * kRows);
   dim3 grid((unsigned)((int64_t)n_seq * Hv * kRowBlocks));
   prefill_recurrent_kernel<T, D><<<grid, kWarps * 32, 0, st>>>(
       (const T*)q, (const T*)k, (const T*)v, g, beta, (T*)o, n_tok, Hk, Hv, qks, vs, cu, init, fin,
-      scale, l2, bl);
+      sbf, scale, l2, bl);
   return cudaGetLastError();
 }
 
 template <typename T>
 cudaError_t launch_d(const void* q, const void* k, const void* v, const float* g,
                      const float* beta, void* o, int64_t n_tok, int32_t Hk, int32_t Hv, int32_t d,
-                     int64_t qks, int64_t vs, const int32_t* cu, int32_t n_seq, const float* init,
-                     float* fin, float scale, int32_t l2, BlockStates bl, cudaStream_t st) {
+                     int64_t qks, int64_t vs, const int32_t* cu, int32_t n_seq, const void* init,
+                     void* fin, int32_t sbf, float scale, int32_t l2, BlockStates bl, cudaStream_t st) {
   switch (d) {
-    case 16: return launch_typed<T, 16>(q, k, v, g, beta, o, n_tok, Hk, Hv, qks, vs, cu, n_seq, init, fin, scale, l2, bl, st);
-    case 32: return launch_typed<T, 32>(q, k, v, g, beta, o, n_tok, Hk, Hv, qks, vs, cu, n_seq, init, fin, scale, l2, bl, st);
-    case 64: return launch_typed<T, 64>(q, k, v, g, beta, o, n_tok, Hk, Hv, qks, vs, cu, n_seq, init, fin, scale, l2, bl, st);
-    default: return launch_typed<T, 128>(q, k, v, g, beta, o, n_tok, Hk, Hv, qks, vs, cu, n_seq, init, fin, scale, l2, bl, st);
+    case 16: return launch_typed<T, 16>(q, k, v, g, beta, o, n_tok, Hk, Hv, qks, vs, cu, n_seq, init, fin, sbf, scale, l2, bl, st);
+    case 32: return launch_typed<T, 32>(q, k, v, g, beta, o, n_tok, Hk, Hv, qks, vs, cu, n_seq, init, fin, sbf, scale, l2, bl, st);
+    case 64: return launch_typed<T, 64>(q, k, v, g, beta, o, n_tok, Hk, Hv, qks, vs, cu, n_seq, init, fin, sbf, scale, l2, bl, st);
+    default: return launch_typed<T, 128>(q, k, v, g, beta, o, n_tok, Hk, Hv, qks, vs, cu, n_seq, init, fin, sbf, scale, l2, bl, st);
   }
 }
 
@@ -168,13 +170,14 @@ cudaError_t launch_prefill_recurrent(int dtype, const void* q, const void* k, co
                                      const float* g, const float* beta, void* o, int64_t T,
                                      int32_t Hk, int32_t Hv, int32_t d, int64_t qk_stride,
                                      int64_t v_stride, const int32_t* cu, int32_t n_seq,
-                                     const float* init, float* fin, float scale, int32_t l2norm,
-                                     BlockStates blocks, cudaStream_t stream) {
+                                     const void* init, void* fin, int state_dtype, float scale,
+                                     int32_t l2norm, BlockStates blocks, cudaStream_t stream) {
+  const int32_t sbf = state_dtype == kBF16 ? 1 : 0;
   if (dtype == kF32)
     return launch_d<float>(q, k, v, g, beta, o, T, Hk, Hv, d, qk_stride, v_stride, cu, n_seq,
-                           init, fin, scale, l2norm, blocks, stream);
+                           init, fin, sbf, scale, l2norm, blocks, stream);
   return launch_d<bf16>(q, k, v, g, beta, o, T, Hk, Hv, d, qk_stride, v_stride, cu, n_seq, init,
-                        fin, scale, l2norm, blocks, stream);
+                        fin, sbf, scale, l2norm, blocks, stream);
 }
 
 }  // namespace gdn

@@ -144,6 +144,70 @@ def make_recurrence(shape: LayerShape, T: int, seed: int, dtype=torch.float32,
                             _as(g, torch.float32), _as(beta, torch.float32), cu, init)
 
 
+# The method's defining edge cases, as inputs (see make_edge_recurrence).
+EDGE_CASES = ("beta0", "g0_beta1", "orthonormal", "repeated_key", "collinear", "strong_decay")
+
+
+def make_edge_recurrence(kind: str, shape: LayerShape, T: int, seed: int, dtype=torch.bfloat16,
+                         init_std: float = 0.02, lengths: Optional[List[int]] = None) -> RecurrenceInputs:
+    """Inputs for the edge cases of the gated delta rule. q, k, v ~ N(0, 1) and
+    S0 ~ N(0, init_std) are drawn first (in that order, then g and beta as below):
+
+    beta0        beta = 0 (pure decay); g ~ U[-0.02, 0]
+    g0_beta1     g = 0 (alpha = 1), beta = 1
+    orthonormal  g = 0, beta = 1, S0 = 0; the key of token t is column (t mod dk) of a random
+                 orthogonal matrix (QR of an N(0, 1) matrix, one per key head), so keys are
+                 mutually orthogonal and each repeats every dk tokens
+    repeated_key g ~ U[-0.3, 0], beta = sigmoid(N(0, 1)); tokens 64..127 share one key and
+                 have beta = 1 (a whole chunk rewriting the same association)
+    collinear    k_t = k0 + 0.05 n_t with n_t ~ N(0, 1) (one k0 per key head);
+                 beta ~ U[0.9, 1], g ~ U[-0.1, 0]
+    strong_decay g ~ U[-8, 0], beta = sigmoid(N(0, 1))
+    """
+    assert kind in EDGE_CASES, kind
+    rng = _rng(seed)
+    cu = None
+    if lengths is not None:
+        T = int(sum(lengths))
+        cu = torch.tensor(np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32))
+    Hk, Hv, dk, dv = shape.Hk, shape.Hv, shape.dk, shape.dv
+    q = _normal(rng, (T, Hk, dk))
+    k = _normal(rng, (T, Hk, dk))
+    v = _normal(rng, (T, Hv, dv))
+    n_seq = 1 if lengths is None else len(lengths)
+    init = _normal(rng, (n_seq, Hv, dv, dk), std=init_std)
+    if kind == "beta0":
+        g = rng.uniform(-0.02, 0.0, size=(T, Hv)).astype(np.float32)
+        beta = np.zeros((T, Hv), np.float32)
+    elif kind == "g0_beta1":
+        g = np.zeros((T, Hv), np.float32)
+        beta = np.ones((T, Hv), np.float32)
+    elif kind == "orthonormal":
+        g = np.zeros((T, Hv), np.float32)
+        beta = np.ones((T, Hv), np.float32)
+        init[:] = 0.0
+        for j in range(Hk):
+            basis, _ = np.linalg.qr(rng.standard_normal((dk, dk)))
+            k[:, j] = basis[:, np.arange(T) % dk].T.astype(np.float32)
+    elif kind == "repeated_key":
+        g = rng.uniform(-0.3, 0.0, size=(T, Hv)).astype(np.float32)
+        beta = _sigmoid(rng.standard_normal((T, Hv)))
+        a, b = min(64, T), min(128, T)
+        k[a:b] = k[a]
+        beta[a:b] = 1.0
+    elif kind == "collinear":
+        k0 = rng.standard_normal((1, Hk, dk)).astype(np.float32)
+        k = k0 + np.float32(0.05) * _normal(rng, (T, Hk, dk))
+        beta = rng.uniform(0.9, 1.0, size=(T, Hv)).astype(np.float32)
+        g = rng.uniform(-0.1, 0.0, size=(T, Hv)).astype(np.float32)
+    else:   # strong_decay
+        g = rng.uniform(-8.0, 0.0, size=(T, Hv)).astype(np.float32)
+        beta = _sigmoid(rng.standard_normal((T, Hv)))
+    return RecurrenceInputs(shape, _as(q, dtype), _as(k, dtype), _as(v, dtype),
+                            _as(g, torch.float32), _as(beta, torch.float32), cu,
+                            _as(init, torch.float32))
+
+
 @dataclasses.dataclass
 class DecodeInputs:
     shape: LayerShape

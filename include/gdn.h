@@ -110,6 +110,22 @@ size_t gdn_chunk_prefill_workspace_size(int64_t T, int32_t n_seq, int32_t Hk, in
                                         int32_t dk, int32_t dv, gdn_dtype_t dt);
 
 /*
+ * gdn_chunk_prefill_path -- which kernels gdn_chunk_prefill (and _ex, _noalloc) runs for
+ * these arguments, so that a caller can see a slow path before taking it:
+ *   GDN_PATH_CHUNKED_TC (1)  the chunked WY/UT form on tcgen05 tensor cores: bf16
+ *                            activations, dk = dv = 128, Hv / Hk <= 8, qk_l2norm = 1;
+ *   GDN_PATH_RECURRENT  (0)  the token-by-token fp32 SIMT kernel: every other supported
+ *                            shape (fp32 activations, heads of 16/32/64, qk_l2norm = 0).
+ *                            It is exact to fp32 rounding but about 25x slower on long
+ *                            bf16 sequences of 128-wide heads;
+ *   -1                       unsupported arguments (the prefill returns an error).
+ * The same path serves every length, sequence count and state dtype.
+ */
+enum { GDN_PATH_RECURRENT = 0, GDN_PATH_CHUNKED_TC = 1 };
+int32_t gdn_chunk_prefill_path(gdn_dtype_t dt, int32_t Hk, int32_t Hv, int32_t dk, int32_t dv,
+                               int32_t qk_l2norm);
+
+/*
  * gdn_chunk_prefill -- the gated delta rule over packed sequences (prefill).
  *
  * Defined by the Qwen3.5 page, section 5: S <- alpha S + beta (v - S k) k^T read as
@@ -161,32 +177,38 @@ gdn_status_t gdn_prefill_status(const void* workspace, gdn_stream_t stream);
 gdn_status_t gdn_prefill_noalloc_status(gdn_stream_t stream);
 
 /*
- * gdn_chunk_prefill_ex -- gdn_chunk_prefill that also stores each sequence's state at block
- * boundaries, for prefix caching (a block's cached state lets a later request that shares
- * the prefix resume from it; the state after token t is the S_t of the Qwen3.5 page,
- * section 5).
+ * gdn_chunk_prefill_ex -- gdn_chunk_prefill with a selectable state storage dtype, that can
+ * also store each sequence's state at block boundaries for prefix caching (a block's cached
+ * state lets a later request that shares the prefix resume from it; the state after token t
+ * is the S_t of the Qwen3.5 page, section 5).
  *
+ * initial_state, final_state  [n_seq, Hv, dv, dk] of state_dt (as in gdn_chunk_prefill).
+ * state_dt      GDN_F32, or GDN_BF16: states stored in bf16 (the storage a server that keeps
+ *               bf16 decode states uses, see gdn_decode_step_ex). Each element is widened to
+ *               fp32 on load; the recurrence runs in fp32 as for GDN_F32; the final and block
+ *               states are rounded to bf16 (nearest, ties to even) once, when stored.
  * block_tokens  0: no block states (the other three block arguments are ignored); else a
  *               positive multiple of 64 (the chunk length, so boundaries fall on chunk ends).
- * block_states  fp32 [n_block_rows, Hv, dv, dk], 16-byte aligned: after the first
+ * block_states  [n_block_rows, Hv, dv, dk] of state_dt, 16-byte aligned: after the first
  *               m * block_tokens tokens of sequence n (m >= 1, m * block_tokens <= its
  *               length) its state is written to row block_rows[n] + m - 1. A sequence whose
  *               length is a multiple of block_tokens also gets its final state there.
  * block_rows    int32 [n_seq] device array: the first row of each sequence. Rows outside
  *               [0, n_block_rows) are skipped, not an error.
- * Other arguments and return codes as gdn_chunk_prefill; GDN_ERR_INVALID_ARG also for a
- * bad block_tokens, missing block buffers or block_states overlapping another buffer.
+ * Other arguments and return codes as gdn_chunk_prefill; GDN_ERR_UNSUPPORTED also for an
+ * unknown state_dt; GDN_ERR_INVALID_ARG also for a bad block_tokens, missing block buffers
+ * or block_states overlapping another buffer.
  */
 gdn_status_t gdn_chunk_prefill_ex(const void* q, const void* k, const void* v,
                                   const float* g, const float* beta, void* o,
                                   gdn_dtype_t dt, int64_t T, int32_t Hk, int32_t Hv,
                                   int32_t dk, int32_t dv, int64_t qk_stride, int64_t v_stride,
                                   const int32_t* cu_seqlens, int32_t n_seq,
-                                  const float* initial_state, float* final_state,
-                                  float scale, int32_t qk_l2norm, int32_t block_tokens,
-                                  float* block_states, const int32_t* block_rows,
-                                  int64_t n_block_rows, void* workspace, size_t workspace_bytes,
-                                  gdn_stream_t stream);
+                                  const void* initial_state, void* final_state,
+                                  gdn_dtype_t state_dt, float scale, int32_t qk_l2norm,
+                                  int32_t block_tokens, void* block_states,
+                                  const int32_t* block_rows, int64_t n_block_rows,
+                                  void* workspace, size_t workspace_bytes, gdn_stream_t stream);
 
 /*
  * gdn_chunk_prefill_noalloc -- gdn_chunk_prefill for callers that cannot allocate.
@@ -200,16 +222,19 @@ gdn_status_t gdn_chunk_prefill_ex(const void* q, const void* k, const void* v,
  * that loads it (64 MiB, held until the process exits). It allocates nothing and calls
  * no allocating routine.
  *
- * Limit: the call is refused with GDN_ERR_WORKSPACE, launching nothing, when
- * gdn_chunk_prefill_workspace_size(...) for these sizes exceeds 64 MiB (with 48 value
- * heads of 128 that is about 3,300 tokens per call; use gdn_chunk_prefill with a caller
- * workspace beyond that). Shapes that need no workspace run exactly as gdn_chunk_prefill.
+ * Limit: the call is refused with GDN_ERR_WORKSPACE, launching nothing, when the path it
+ * takes (gdn_chunk_prefill_path) needs more than 64 MiB of scratch for these sizes. The
+ * tensor-core path needs gdn_chunk_prefill_workspace_size(...) bytes: with 48 value heads
+ * of 128 in one sequence that allows 1,472 tokens per call (2,240 with 32 value heads); use
+ * gdn_chunk_prefill with a caller workspace beyond that. The token-recurrent path needs
+ * no scratch and is never refused.
  * Set-up: the first call on each device looks up the scratch array's device address
  * (cudaGetSymbolAddress, with that device current); make that first call before any
- * stream capture. The array is shared by every call: the kernels rewrite everything they
- * read from it, so no clearing is needed, but calls whose execution overlaps on the GPU
- * (different streams, or different host threads on one device) race on it -- order them
- * on one stream or synchronise between them.
+ * stream capture. The array is shared by every call: its first word (the status word of
+ * gdn_prefill_noalloc_status) is cleared by every call, the kernels rewrite everything
+ * else they read from it, but calls whose execution overlaps on the GPU (different
+ * streams, or different host threads on one device) race on it -- order them on one
+ * stream or synchronise between them.
  * Returns the same codes as gdn_chunk_prefill.
  */
 gdn_status_t gdn_chunk_prefill_noalloc(const void* q, const void* k, const void* v,

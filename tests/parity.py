@@ -13,6 +13,17 @@ import oracle
 FP32_TOL = 1e-4
 BF16_TOL = 2e-2
 
+# (test case, quantity, worst error, tolerance) of every checked comparison; the terminal
+# summary prints them so that each parity test's margin is on record.
+MARGINS = []
+
+
+def check(case: str, what: str, err: float, tol: float) -> float:
+    """Record a worst error against its tolerance, then assert it is within."""
+    MARGINS.append((case, what, float(err), float(tol)))
+    assert err <= tol, f"{case}: {what} error {err:.3e} > {tol:.1e}"
+    return err
+
 
 def np64(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy().astype(np.float64)

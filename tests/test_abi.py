@@ -175,8 +175,9 @@ def test_prefill_block_state_validation(L):
                  o=FAKE + (4 << 30), fin=FAKE + (5 << 30))
         a.update(kw)
         return L.gdn_chunk_prefill_ex(a["q"], a["k"], a["v"], a["g"], a["b"], a["o"], 0, 128, 2,
-                                      4, 32, 32, 128, 128, None, 1, None, a["fin"], 1.0, 1, bt, bs,
-                                      br, nr, None, 0, None)
+                                      4, 32, 32, 128, 128, None, 1, None, a["fin"],
+                                      kw.get("state_dt", _lib.GDN_F32), 1.0, 1, bt, bs, br, nr,
+                                      None, 0, None)
     rows = FAKE + (7 << 30)
     assert call(-64, FAKE + (6 << 30), rows, 4) == _lib.GDN_ERR_INVALID_ARG
     assert call(96, FAKE + (6 << 30), rows, 4) == _lib.GDN_ERR_INVALID_ARG      # not a multiple of 64
@@ -185,6 +186,12 @@ def test_prefill_block_state_validation(L):
     assert call(64, FAKE + (6 << 30), rows, 0) == _lib.GDN_ERR_INVALID_ARG
     assert call(64, FAKE + (6 << 30) + 8, rows, 4) == _lib.GDN_ERR_INVALID_ARG  # misaligned
     assert call(64, FAKE + (5 << 30) + 4096, rows, 4) == _lib.GDN_ERR_INVALID_ARG  # inside final_state
+    # the state dtype: unknown codes are unsupported; with bf16 states the buffers are half
+    # the size, so a block buffer starting 64 KB after a bf16 final state no longer overlaps it
+    assert call(64, FAKE + (6 << 30), rows, 4, state_dt=7) == _lib.GDN_ERR_UNSUPPORTED
+    fin_f32_bytes = 1 * 4 * 32 * 32 * 4
+    assert call(64, FAKE + (5 << 30) + fin_f32_bytes // 2, rows, 4, state_dt=_lib.GDN_F32) == \
+        _lib.GDN_ERR_INVALID_ARG
 
 
 def test_prefill_beyond_32bit_coordinates_is_refused(L):
@@ -211,3 +218,35 @@ def test_python_binding_refuses_cpu_tensors():
     w = torch.zeros(64, 4, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         gdn.gdn_conv1d_silu(x, w)
+
+
+def test_prefill_path_query(L):
+    """The path each shape takes is visible before the call: the tensor-core chunked form
+    for bf16 heads of 128 with the L2 norm, the token-recurrent kernel otherwise."""
+    B, F = _lib.GDN_BF16, _lib.GDN_F32
+    assert L.gdn_chunk_prefill_path(B, 16, 48, 128, 128, 1) == 1
+    assert L.gdn_chunk_prefill_path(B, 16, 48, 128, 128, 0) == 0
+    assert L.gdn_chunk_prefill_path(F, 2, 2, 16, 16, 1) == 0
+    assert L.gdn_chunk_prefill_path(B, 2, 4, 64, 64, 1) == 0
+    assert L.gdn_chunk_prefill_path(B, 1, 16, 128, 128, 1) == 0      # 16 value heads per key head
+    assert L.gdn_chunk_prefill_path(B, 3, 4, 128, 128, 1) == -1      # Hv % Hk != 0
+    assert L.gdn_chunk_prefill_path(B, 2, 4, 96, 96, 1) == -1        # head size not built
+
+
+def test_noalloc_refusal_follows_the_path(L):
+    """The no-allocation prefill refuses a size only when the path it takes needs more
+    scratch than its static array: with the L2 norm on (tensor-core path) the call returns
+    GDN_ERR_WORKSPACE before any CUDA call; with it off (token-recurrent path, no scratch) it
+    is not refused and goes on to the device (which a machine without a GPU reports as a
+    CUDA error)."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("passes fake device addresses; the second call would launch on a GPU")
+    T, Hk, Hv, d = 3000, 16, 48, 128
+    args = (FAKE, FAKE + (1 << 34), FAKE + (2 << 34), FAKE + (3 << 34), FAKE + (4 << 34),
+            FAKE + (5 << 34), _lib.GDN_BF16, T, Hk, Hv, d, d, 0, 0, None, 1, None, None, 1.0)
+    st = L.gdn_chunk_prefill_noalloc(*args, 1, None)
+    assert st == _lib.GDN_ERR_WORKSPACE
+    assert "nothing was launched" in L.gdn_last_error().decode()
+    st = L.gdn_chunk_prefill_noalloc(*args, 0, None)
+    assert st == _lib.GDN_ERR_CUDA

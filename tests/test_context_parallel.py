@@ -1,6 +1,7 @@
 """Context-parallel prefill of one sequence split across ranks: the exchange and the fold
 run as gloo ranks on the CPU with the oracle as the per-segment prefill (exact in fp64); on
-one GPU the same pieces run with the library's prefill, segment by segment."""
+one GPU the same pieces run with the library's prefill, segment by segment, and are compared
+with the oracle."""
 import os
 import socket
 import sys
@@ -70,11 +71,14 @@ def test_cp_prefill_gloo_equals_one_run(oracle_mod, lengths, with_state):
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-def test_cp_pieces_on_gpu(cuda_device, dtype):
-    """Two segments on one GPU (summaries, fold, second pass) against one prefill of the
-    whole sequence: fp32 (token-recurrent path) at 1e-4, bf16 heads of 128 (tensor-core
-    path) at the bf16 tolerance."""
-    from parity import BF16_TOL, FP32_TOL, frob_rel, max_rel, np64
+def test_cp_pieces_on_gpu_against_oracle(cuda_device, dtype):
+    """Two segments on one GPU with the library's prefill: each segment's transition P (the
+    v = 0 run from the identity) and zero-start state S_loc, the fold, and the second pass,
+    against the fp64 oracle run over the whole sequence (and over each segment for P and
+    S_loc). fp32 (token-recurrent path) at 1e-4; bf16 heads of 128 (tensor-core path) at the
+    bf16 per-head gate."""
+    import oracle
+    from parity import BF16_TOL, FP32_TOL, check, frob_rel, max_rel, np64
     r = W.make_recurrence(W.LayerShape(2, 4, 128, 128), 700, seed=53, dtype=dtype, init_std=0.02)
     dev = cuda_device
     q, k, v, g, b = (t.to(dev) for t in (r.q, r.k, r.v, r.g, r.beta))
@@ -85,12 +89,29 @@ def test_cp_pieces_on_gpu(cuda_device, dtype):
     states = cp.fold(sums, s0)
     o_cp = torch.cat([prefill(q[a:e], k[a:e], v[a:e], g[a:e], b[a:e], states[i].contiguous())[0]
                       for i, (a, e) in enumerate(cuts)])
-    o_one, fin_one = prefill(q, k, v, g, b, s0)
     torch.cuda.synchronize()
+    qn, kn, vn = (t.double().numpy() for t in (r.q, r.k, r.v))
+    gn, bn = r.g.double().numpy(), r.beta.double().numpy()
+    o_ref, fin_ref = oracle.recurrence(qn, kn, vn, gn, bn, initial_state=r.initial_state.numpy())
+    case = f"test_cp_pieces_on_gpu_against_oracle[{'f32' if dtype == torch.float32 else 'bf16'}]"
+    eye = np.broadcast_to(np.eye(128), (1, 4, 128, 128))
+    for i, (a, e) in enumerate(cuts):
+        _, p_ref = oracle.recurrence(qn[a:e], kn[a:e], np.zeros_like(vn[a:e]), gn[a:e], bn[a:e],
+                                     initial_state=eye)
+        _, l_ref = oracle.recurrence(qn[a:e], kn[a:e], vn[a:e], gn[a:e], bn[a:e])
+        s_loc, P = np64(sums[i][0]), np64(sums[i][1])
+        if dtype == torch.float32:
+            check(case, f"P seg {i}", max_rel(P, p_ref), FP32_TOL)
+            check(case, f"S_loc seg {i}", max_rel(s_loc, l_ref), FP32_TOL)
+        else:
+            check(case, f"P seg {i}", max(frob_rel(P[0, h], p_ref[0, h]) for h in range(4)), BF16_TOL)
+            check(case, f"S_loc seg {i}", max(frob_rel(s_loc[0, h], l_ref[0, h]) for h in range(4)),
+                  BF16_TOL)
+    o, fin = np64(o_cp), np64(states[-1])
     if dtype == torch.float32:
-        assert max_rel(np64(o_cp), np64(o_one)) <= FP32_TOL
-        assert max_rel(np64(states[-1]), np64(fin_one)) <= FP32_TOL
+        check(case, "max rel o", max_rel(o, o_ref), FP32_TOL)
+        check(case, "max rel state", max_rel(fin, fin_ref), FP32_TOL)
     else:
-        for h in range(4):
-            assert frob_rel(np64(o_cp)[:, h], np64(o_one)[:, h]) <= BF16_TOL, h
-            assert frob_rel(np64(states[-1])[0, h], np64(fin_one)[0, h]) <= BF16_TOL, h
+        check(case, "o per head", max(frob_rel(o[:, h], o_ref[:, h]) for h in range(4)), BF16_TOL)
+        check(case, "state per head", max(frob_rel(fin[0, h], fin_ref[0, h]) for h in range(4)),
+              BF16_TOL)

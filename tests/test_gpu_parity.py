@@ -12,8 +12,8 @@ import torch
 import gated_deltanet_mixer_causal_b200 as gdn
 from gated_deltanet_mixer_causal_b200 import workloads as W
 import oracle
-from parity import (BF16_TOL, FP32_TOL, frob_rel, max_rel, np64, oracle_layer_heads, worst_head_o,
-                    worst_head_state)
+from parity import (BF16_TOL, FP32_TOL, check, frob_rel, max_rel, np64, oracle_layer_heads,
+                    worst_head_o, worst_head_state)
 
 pytestmark = pytest.mark.gpu
 
@@ -54,8 +54,8 @@ def test_tiny_recurrence_fp32(cuda_device):
     fin = torch.empty((1, 2, 16, 16), device=cuda_device)
     o = gdn.gdn_chunk_prefill(r.q.to(cuda_device), r.k.to(cuda_device), r.v.to(cuda_device),
                               r.g.to(cuda_device), r.beta.to(cuda_device), final_state=fin)
-    assert max_rel(np64(o), o_ref) <= FP32_TOL
-    assert max_rel(np64(fin), f_ref) <= FP32_TOL
+    check("test_tiny_recurrence_fp32", "max rel o", max_rel(np64(o), o_ref), FP32_TOL)
+    check("test_tiny_recurrence_fp32", "max rel state", max_rel(np64(fin), f_ref), FP32_TOL)
 
 
 def test_tiny_layer_fp32(cuda_device):
@@ -64,8 +64,8 @@ def test_tiny_layer_fp32(cuda_device):
     o_ref, f_ref, cs_ref = oracle.layer_prefill(p.x.numpy(), p.conv_w.numpy(), p.g.numpy(),
                                                 p.beta.numpy(), sh.Hk, sh.Hv, sh.dk, sh.dv)
     o, fin, cs = run_layer(p, cuda_device, want_conv_state=True)
-    assert max_rel(np64(o), o_ref) <= FP32_TOL
-    assert max_rel(np64(fin), f_ref) <= FP32_TOL
+    check("test_tiny_layer_fp32", "max rel o", max_rel(np64(o), o_ref), FP32_TOL)
+    check("test_tiny_layer_fp32", "max rel state", max_rel(np64(fin), f_ref), FP32_TOL)
     np.testing.assert_array_equal(np64(cs), cs_ref)
 
 
@@ -118,8 +118,8 @@ def test_prefill_bf16_ragged_9b_shape(cuda_device):
     o_ref, f_ref, _ = oracle.layer_prefill(p.x.float().numpy(), p.conv_w.float().numpy(),
                                            p.g.numpy(), p.beta.numpy(), sh.Hk, sh.Hv, sh.dk, sh.dv)
     o, fin, _ = run_layer(p, cuda_device)
-    assert worst_head_o(np64(o), o_ref, None) <= BF16_TOL
-    assert worst_head_state(np64(fin), f_ref) <= BF16_TOL
+    check("test_prefill_bf16_ragged_9b_shape", "o per head", worst_head_o(np64(o), o_ref, None), BF16_TOL)
+    check("test_prefill_bf16_ragged_9b_shape", "state per head", worst_head_state(np64(fin), f_ref), BF16_TOL)
 
 
 def test_prefill_bf16_varlen_with_state(cuda_device):
@@ -137,8 +137,8 @@ def test_prefill_bf16_varlen_with_state(cuda_device):
                                                 sh.dk, sh.dv, cu, p.initial_state.numpy(),
                                                 cs_in.float().numpy())
     o, fin, cs = run_layer(p, cuda_device, conv_state_in=cs_in, want_conv_state=True)
-    assert worst_head_o(np64(o), o_ref, cu) <= BF16_TOL
-    assert worst_head_state(np64(fin), f_ref) <= BF16_TOL
+    check("test_prefill_bf16_varlen_with_state", "o per head", worst_head_o(np64(o), o_ref, cu), BF16_TOL)
+    check("test_prefill_bf16_varlen_with_state", "state per head", worst_head_state(np64(fin), f_ref), BF16_TOL)
     np.testing.assert_array_equal(np64(fin)[5], p.initial_state.numpy()[5])   # empty sequence
     np.testing.assert_array_equal(np64(cs), cs_ref)
 
@@ -160,8 +160,8 @@ def test_prefill_bf16_d128_without_l2norm(cuda_device):
     o_r, fin_r = oracle.recurrence(q.float().numpy(), k.float().numpy(), v.float().numpy(),
                                    r.g.numpy(), r.beta.numpy(), initial_state=r.initial_state.numpy(),
                                    l2norm=False)
-    assert worst_head_o(np64(o), o_r, [0, 200]) <= BF16_TOL
-    assert worst_head_state(np64(fin), fin_r) <= BF16_TOL
+    check("test_prefill_bf16_d128_without_l2norm", "o per head", worst_head_o(np64(o), o_r, [0, 200]), BF16_TOL)
+    check("test_prefill_bf16_d128_without_l2norm", "state per head", worst_head_state(np64(fin), fin_r), BF16_TOL)
 
 
 def test_prefill_status_after_a_call(cuda_device):
@@ -190,8 +190,8 @@ def test_prefill_final_state_in_place(cuda_device):
                           p.beta.to(cuda_device), sh.Hk, sh.Hv, sh.dk, initial_state=st,
                           final_state=st)
     torch.cuda.synchronize()
-    assert worst_head_o(np64(o), o_ref, None) <= BF16_TOL
-    assert worst_head_state(np64(st), f_ref) <= BF16_TOL
+    check("test_prefill_final_state_in_place", "o per head", worst_head_o(np64(o), o_ref, None), BF16_TOL)
+    check("test_prefill_final_state_in_place", "state per head", worst_head_state(np64(st), f_ref), BF16_TOL)
 
 
 def test_prefill_empty_batch_passes_state(cuda_device):
@@ -213,8 +213,8 @@ def test_prefill_9b_full(cuda_device):
     o, fin, _ = run_layer(p, cuda_device)
     o_ref, f_ref, _ = oracle.layer_prefill(p.x.float().numpy(), p.conv_w.float().numpy(),
                                            p.g.numpy(), p.beta.numpy(), sh.Hk, sh.Hv, sh.dk, sh.dv)
-    assert worst_head_o(np64(o), o_ref, None) <= BF16_TOL
-    assert worst_head_state(np64(fin), f_ref) <= BF16_TOL
+    check("test_prefill_9b_full", "o per head", worst_head_o(np64(o), o_ref, None), BF16_TOL)
+    check("test_prefill_9b_full", "state per head", worst_head_state(np64(fin), f_ref), BF16_TOL)
 
 
 def test_prefill_27b_64k_sampled_heads(cuda_device):
@@ -225,10 +225,10 @@ def test_prefill_27b_64k_sampled_heads(cuda_device):
     heads = [0, 25, 47]
     ref = oracle_layer_heads(p, heads)
     o_np, f_np = np64(o), np64(fin)
-    for h in heads:
-        o_r, f_r = ref[(0, h)]
-        assert frob_rel(o_np[:, h], o_r) <= BF16_TOL, h
-        assert frob_rel(f_np[0, h], f_r) <= BF16_TOL, h
+    check("test_prefill_27b_64k_sampled_heads", "o per head",
+          max(frob_rel(o_np[:, h], ref[(0, h)][0]) for h in heads), BF16_TOL)
+    check("test_prefill_27b_64k_sampled_heads", "state per head",
+          max(frob_rel(f_np[0, h], ref[(0, h)][1]) for h in heads), BF16_TOL)
 
 
 def test_prefill_27b_varlen_sampled(cuda_device):
@@ -241,13 +241,16 @@ def test_prefill_27b_varlen_sampled(cuda_device):
     short, long_ = int(np.argmin(lens)), int(np.argmax(lens))
     o_np, f_np = np64(o), np64(fin)
     checks = [(short, list(range(p.shape.Hv))), (long_, [7, 40])]
+    eo, es = 0.0, 0.0
     for n, heads in checks:
         ref = oracle_layer_heads(p, heads, seqs=[n])
         a, b = int(cu[n]), int(cu[n + 1])
         for h in heads:
             o_r, f_r = ref[(n, h)]
-            assert frob_rel(o_np[a:b, h], o_r) <= BF16_TOL, (n, h)
-            assert frob_rel(f_np[n, h], f_r) <= BF16_TOL, (n, h)
+            eo = max(eo, frob_rel(o_np[a:b, h], o_r))
+            es = max(es, frob_rel(f_np[n, h], f_r))
+    check("test_prefill_27b_varlen_sampled", "o per head", eo, BF16_TOL)
+    check("test_prefill_27b_varlen_sampled", "state per head", es, BF16_TOL)
 
 
 # --------------------------------------------------------------------------- decode
@@ -266,8 +269,8 @@ def test_decode_fp32_small(cuda_device):
                                              d.gs[t].numpy(), d.betas[t].numpy(), st_r, sh.Hk,
                                              sh.Hv, sh.dk, sh.dv)
         torch.cuda.synchronize()
-        assert max_rel(np64(o), o_r) <= FP32_TOL
-        assert max_rel(np64(st), st_r) <= FP32_TOL
+        check("test_decode_fp32_small", "max rel o", max_rel(np64(o), o_r), FP32_TOL)
+        check("test_decode_fp32_small", "max rel state", max_rel(np64(st), st_r), FP32_TOL)
         np.testing.assert_array_equal(np64(cs), cs_r)
 
 
@@ -293,16 +296,18 @@ def test_decode_27b_batch256_100_steps(cuda_device):
             torch.cuda.synchronize()
             o_g = np64(o)[sample]
             st_g = np64(st[sample])
-            for j in range(len(sample)):
-                for h in range(sh.Hv):
-                    assert frob_rel(o_g[j, h], o_r[j, h]) <= BF16_TOL, (t, j, h)
-                    assert frob_rel(st_g[j, h], st_r[j, h]) <= BF16_TOL, (t, j, h)
+            check(f"test_decode_27b_batch256_100_steps (step {t + 1})", "o per head",
+                  max(frob_rel(o_g[j, h], o_r[j, h]) for j in range(len(sample)) for h in range(sh.Hv)),
+                  BF16_TOL)
+            check(f"test_decode_27b_batch256_100_steps (step {t + 1})", "state per head",
+                  max(frob_rel(st_g[j, h], st_r[j, h]) for j in range(len(sample)) for h in range(sh.Hv)),
+                  BF16_TOL)
             np.testing.assert_array_equal(np64(cs[sample]), cs_r)
 
 
 def test_decode_matches_prefill_on_gpu(cuda_device):
-    """Eight decode steps equal a prefill of the same eight tokens from the same states
-    (both on the GPU; bf16 tolerance)."""
+    """Eight decode steps and a prefill of the same eight tokens from the same states, each
+    against the oracle's eight steps (bf16 tolerance)."""
     sh = W.LayerShape(2, 6, 64, 64)
     d = W.make_decode(sh, B=2, steps=8, seed=42)
     cs = d.conv_state.to(cuda_device).clone()
@@ -321,8 +326,16 @@ def test_decode_matches_prefill_on_gpu(cuda_device):
                             d.conv_state.to(cuda_device), fin)
     torch.cuda.synchronize()
     o_d = torch.stack(outs, 1).reshape(16, sh.Hv, sh.dv)
-    assert worst_head_o(np64(o_d), np64(o_p), [0, 8, 16]) <= BF16_TOL
-    assert worst_head_state(np64(st), np64(fin)) <= BF16_TOL
+    o_r, st_r, _ = oracle.decode_tokens(torch.stack(d.xs, 1).float().numpy(), d.conv_w.float().numpy(),
+                                        d.conv_state.float().numpy(), torch.stack(d.gs, 1).numpy(),
+                                        torch.stack(d.betas, 1).numpy(), d.state.numpy(), sh.Hk, sh.Hv,
+                                        sh.dk, sh.dv)
+    o_r = o_r.reshape(16, sh.Hv, sh.dv)
+    for name, o, s in (("8 decode steps", o_d, st), ("prefill of the 8 tokens", o_p, fin)):
+        check(f"test_decode_matches_prefill_on_gpu ({name})", "o per head",
+              worst_head_o(np64(o), o_r, [0, 8, 16]), BF16_TOL)
+        check(f"test_decode_matches_prefill_on_gpu ({name})", "state per head",
+              worst_head_state(np64(s), st_r), BF16_TOL)
 
 
 # ------------------------------------------------------------ multi-token decode
@@ -343,8 +356,8 @@ def test_decode_tokens_fp32_small(cuda_device, n_tok):
                                            g.numpy(), b.numpy(), d.state.numpy(), sh.Hk, sh.Hv,
                                            sh.dk, sh.dv)
     assert o.shape == (3, n_tok, sh.Hv, sh.dv)
-    assert max_rel(np64(o), o_r) <= FP32_TOL
-    assert max_rel(np64(st), st_r) <= FP32_TOL
+    check("test_decode_tokens_fp32_small", "max rel o", max_rel(np64(o), o_r), FP32_TOL)
+    check("test_decode_tokens_fp32_small", "max rel state", max_rel(np64(st), st_r), FP32_TOL)
     np.testing.assert_array_equal(np64(cs), cs_r)
 
 
@@ -364,16 +377,16 @@ def test_decode_tokens_27b_bf16(cuda_device, n_tok):
                                            d.conv_state.float().numpy(), g.numpy(), b.numpy(),
                                            d.state.numpy(), sh.Hk, sh.Hv, sh.dk, sh.dv)
     o_g, st_g = np64(o), np64(st)
-    for j in range(16):
-        for h in range(sh.Hv):
-            assert frob_rel(o_g[j, :, h], o_r[j, :, h]) <= BF16_TOL, (j, h)
-            assert frob_rel(st_g[j, h], st_r[j, h]) <= BF16_TOL, (j, h)
+    check(f"test_decode_tokens_27b_bf16[{n_tok}]", "o per head",
+          max(frob_rel(o_g[j, :, h], o_r[j, :, h]) for j in range(16) for h in range(sh.Hv)), BF16_TOL)
+    check(f"test_decode_tokens_27b_bf16[{n_tok}]", "state per head",
+          max(frob_rel(st_g[j, h], st_r[j, h]) for j in range(16) for h in range(sh.Hv)), BF16_TOL)
     np.testing.assert_array_equal(np64(cs), cs_r)
 
 
-def test_decode_tokens_equals_single_steps_on_gpu(cuda_device):
-    """Four tokens in one call agree with four gdn_decode_step calls (both on the GPU, the
-    same per-row arithmetic)."""
+def test_decode_tokens_and_single_steps_against_oracle(cuda_device):
+    """Four tokens in one call and four gdn_decode_step calls from the same states, each
+    against the oracle's four steps (27B-shaped heads, 8 sequences)."""
     d = W.make_decode(W.QWEN35_27B, B=8, steps=4, seed=45)
     sh = d.shape
     w = d.conv_w.to(cuda_device)
@@ -381,13 +394,20 @@ def test_decode_tokens_equals_single_steps_on_gpu(cuda_device):
     outs = [gdn.gdn_decode_step(d.xs[t].to(cuda_device), w, cs1, d.gs[t].to(cuda_device),
                                 d.betas[t].to(cuda_device), st1, sh.Hk) for t in range(4)]
     cs4 = d.conv_state.to(cuda_device).clone(); st4 = d.state.to(cuda_device).clone()
-    o4 = gdn.gdn_decode_tokens(torch.stack(d.xs, 1).to(cuda_device), w, cs4,
-                               torch.stack(d.gs, 1).to(cuda_device),
-                               torch.stack(d.betas, 1).to(cuda_device), st4, sh.Hk)
+    x = torch.stack(d.xs, 1); g = torch.stack(d.gs, 1); b = torch.stack(d.betas, 1)
+    o4 = gdn.gdn_decode_tokens(x.to(cuda_device), w, cs4, g.to(cuda_device), b.to(cuda_device),
+                               st4, sh.Hk)
     torch.cuda.synchronize()
-    np.testing.assert_allclose(np64(o4), np64(torch.stack(outs, 1)), rtol=1e-2, atol=1e-3)
-    assert max_rel(np64(st4), np64(st1)) <= 1e-5
-    assert torch.equal(cs4, cs1)
+    o_r, st_r, cs_r = oracle.decode_tokens(x.float().numpy(), d.conv_w.float().numpy(),
+                                           d.conv_state.float().numpy(), g.numpy(), b.numpy(),
+                                           d.state.numpy(), sh.Hk, sh.Hv, sh.dk, sh.dv)
+    o1 = np64(torch.stack(outs, 1))
+    for name, o, st, cs in (("single steps", o1, np64(st1), cs1), ("one 4-token call", np64(o4), np64(st4), cs4)):
+        check(f"test_decode_tokens_and_single_steps_against_oracle ({name})", "o per head",
+              max(frob_rel(o[j, :, h], o_r[j, :, h]) for j in range(8) for h in range(sh.Hv)), BF16_TOL)
+        check(f"test_decode_tokens_and_single_steps_against_oracle ({name})", "state per head",
+              max(frob_rel(st[j, h], st_r[j, h]) for j in range(8) for h in range(sh.Hv)), BF16_TOL)
+        np.testing.assert_array_equal(np64(cs), cs_r)
 
 
 # ---------------------------------------------------------------- bf16 states
@@ -411,10 +431,10 @@ def test_decode_bf16_state_27b(cuda_device):
         if (t + 1) % 5 == 0:
             torch.cuda.synchronize()
             o_g, st_g = np64(o), np64(st)
-            for j in range(16):
-                for h in range(sh.Hv):
-                    assert frob_rel(o_g[j, h], o_r[j, h]) <= BF16_TOL, (t, j, h)
-                    assert frob_rel(st_g[j, h], st_r[j, h]) <= BF16_TOL, (t, j, h)
+            check(f"test_decode_bf16_state_27b (step {t + 1})", "o per head",
+                  max(frob_rel(o_g[j, h], o_r[j, h]) for j in range(16) for h in range(sh.Hv)), BF16_TOL)
+            check(f"test_decode_bf16_state_27b (step {t + 1})", "state per head",
+                  max(frob_rel(st_g[j, h], st_r[j, h]) for j in range(16) for h in range(sh.Hv)), BF16_TOL)
             np.testing.assert_array_equal(np64(cs), cs_r)
     assert st.dtype == torch.bfloat16
 
@@ -435,10 +455,10 @@ def test_decode_tokens_bf16_state_27b(cuda_device, n_tok):
                                            d.conv_state.float().numpy(), g.numpy(), b.numpy(), s0,
                                            sh.Hk, sh.Hv, sh.dk, sh.dv, state_dtype="bf16")
     o_g, st_g = np64(o), np64(st)
-    for j in range(16):
-        for h in range(sh.Hv):
-            assert frob_rel(o_g[j, :, h], o_r[j, :, h]) <= BF16_TOL, (j, h)
-            assert frob_rel(st_g[j, h], st_r[j, h]) <= BF16_TOL, (j, h)
+    check(f"test_decode_tokens_bf16_state_27b[{n_tok}]", "o per head",
+          max(frob_rel(o_g[j, :, h], o_r[j, :, h]) for j in range(16) for h in range(sh.Hv)), BF16_TOL)
+    check(f"test_decode_tokens_bf16_state_27b[{n_tok}]", "state per head",
+          max(frob_rel(st_g[j, h], st_r[j, h]) for j in range(16) for h in range(sh.Hv)), BF16_TOL)
     np.testing.assert_array_equal(np64(cs), cs_r)
 
 
@@ -487,9 +507,8 @@ def test_prefill_block_states_bf16(cuda_device):
     got = _run_with_blocks(r, cuda_device, block, rows, 10)
     ref = _block_state_reference(r, lengths, block, rows, 10)
     assert sorted(ref) == list(range(10))
-    for row, s_ref in ref.items():
-        for h in range(4):
-            assert frob_rel(got[row, h], s_ref[h]) <= BF16_TOL, (row, h)
+    check("test_prefill_block_states_bf16", "state per head",
+          max(frob_rel(got[row, h], s_ref[h]) for row, s_ref in ref.items() for h in range(4)), BF16_TOL)
 
 
 def test_prefill_block_states_fp32_rows_out_of_range(cuda_device):
@@ -502,6 +521,57 @@ def test_prefill_block_states_fp32_rows_out_of_range(cuda_device):
     got = _run_with_blocks(r, cuda_device, block, rows, n_rows)   # row 2 is never written
     ref = _block_state_reference(r, lengths, block, rows, n_rows)
     assert sorted(ref) == [0, 1, 3, 4, 5]
-    for row, s_ref in ref.items():
-        assert max_rel(got[row], s_ref) <= FP32_TOL, row
+    check("test_prefill_block_states_fp32_rows_out_of_range", "max rel state",
+          max(max_rel(got[row], s_ref) for row, s_ref in ref.items()), FP32_TOL)
     assert np.isnan(got[2]).all()
+
+
+# ------------------------------------------------------- bf16 states in the prefill
+
+@pytest.mark.parametrize("path", ["chunked_tc", "recurrent"])
+def test_prefill_bf16_states(cuda_device, path):
+    """Initial, final and block states stored in bf16 (fp32 math): 27B-shaped heads on the
+    tensor-core path, and fp32 activations with heads of 32 on the token-recurrent path. The
+    oracle starts from the same bf16 initial states and rounds its fp64 final and block states
+    to bf16 once, as the kernels do; per-head bf16 gate."""
+    dev = cuda_device
+    if path == "chunked_tc":
+        sh, dt, lengths = W.QWEN35_27B, torch.bfloat16, [300, 129, 64]
+    else:
+        sh, dt, lengths = W.LayerShape(2, 4, 32, 32), torch.float32, [150, 64, 70]
+    r = W.make_recurrence(sh, 0, seed=57, dtype=dt, init_std=0.02, lengths=lengths)
+    assert gdn.gdn_chunk_prefill_path(dt, sh.Hk, sh.Hv, sh.dk, sh.dv) == path
+    s0 = oracle.round_bf16(r.initial_state.numpy())
+    init = torch.from_numpy(s0).to(torch.bfloat16).to(dev)
+    n = len(lengths)
+    fin = torch.empty((n, sh.Hv, sh.dv, sh.dk), dtype=torch.bfloat16, device=dev)
+    bs = torch.full((8, sh.Hv, sh.dv, sh.dk), float("nan"), dtype=torch.bfloat16, device=dev)
+    rows = torch.tensor([0, 4, 6], dtype=torch.int32, device=dev)
+    o = gdn.gdn_chunk_prefill(r.q.to(dev), r.k.to(dev), r.v.to(dev), r.g.to(dev), r.beta.to(dev),
+                              r.cu_seqlens.to(dev), init, fin, block_tokens=64, block_states=bs,
+                              block_rows=rows)
+    torch.cuda.synchronize()
+    cu = r.cu_seqlens.numpy()
+    o_r, f_r = oracle.recurrence(r.q.float().numpy(), r.k.float().numpy(), r.v.float().numpy(),
+                                 r.g.numpy(), r.beta.numpy(), cu, s0)
+    case = f"test_prefill_bf16_states[{path}]"
+    tol = BF16_TOL if dt == torch.bfloat16 else FP32_TOL
+    if dt == torch.bfloat16:
+        check(case, "o per head", worst_head_o(np64(o), o_r, cu), tol)
+    else:
+        check(case, "max rel o", max_rel(np64(o), o_r), tol)
+    check(case, "state per head", worst_head_state(np64(fin), oracle.round_bf16(f_r)), BF16_TOL)
+    assert fin.dtype == torch.bfloat16
+    # block states: rows 0..3 = sequence 0 after 64, 128, 192, 256 tokens; rows 4, 5 =
+    # sequence 1 after 64, 128; row 6 = sequence 2 after 64 (its final state); row 7 unused
+    want = {0: (0, 64), 1: (0, 128), 2: (0, 192), 3: (0, 256), 4: (1, 64), 5: (1, 128), 6: (2, 64)}
+    got = np64(bs)
+    worst = 0.0
+    for row, (nq, m) in want.items():
+        a = cu[nq]
+        _, fr = oracle.recurrence(r.q[a:a + m].float().numpy(), r.k[a:a + m].float().numpy(),
+                                  r.v[a:a + m].float().numpy(), r.g[a:a + m].numpy(),
+                                  r.beta[a:a + m].numpy(), initial_state=s0[nq:nq + 1])
+        worst = max(worst, worst_head_state(got[row:row + 1], oracle.round_bf16(fr)))
+    check(case, "block states", worst, BF16_TOL)
+    assert np.isnan(got[7]).all()
