@@ -97,7 +97,7 @@ template <typename S, int D> struct RowShape {
 };
 
 template <typename T, int D, typename S>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 3)   // three CTAs per SM: 24 warps of loads in flight
 decode_step_kernel(const T* __restrict__ x, const T* __restrict__ conv_w, T* __restrict__ conv_state,
                    const float* __restrict__ g, const float* __restrict__ beta,
                    S* __restrict__ state, T* __restrict__ o, int32_t Hk, int32_t Hv,
@@ -178,13 +178,12 @@ decode_step_kernel(const T* __restrict__ x, const T* __restrict__ conv_w, T* __r
   const int sub = lane / LPR;
   for (int r0 = warp * kRowUnroll * RPW; r0 < rows; r0 += kWarps * kRowUnroll * RPW) {
     float s[kRowUnroll][VEC];
-    S* ptr[kRowUnroll];
+    // the CTA's G value heads are consecutive, so its rows are one contiguous block
+    S* rows_base = state + (b * Hv + (int64_t)hk * G) * D * D + col;
 #pragma unroll
     for (int u = 0; u < kRowUnroll; ++u) {
       const int r = r0 + u * RPW + sub;
-      const int h = hk * G + r / D, i = r % D;
-      ptr[u] = state + ((b * Hv + h) * (int64_t)D + i) * D + col;
-      if (r < rows && active) RowIO<S, VEC>::load(ptr[u], s[u]);
+      if (r < rows && active) RowIO<S, VEC>::load(rows_base + (int64_t)r * D, s[u]);
       else {
 #pragma unroll
         for (int j = 0; j < VEC; ++j) s[u][j] = 0.f;
@@ -215,7 +214,7 @@ decode_step_kernel(const T* __restrict__ x, const T* __restrict__ conv_w, T* __r
       const float uu = bt * (ys[2 * D + r] - alpha * sk[u]);
 #pragma unroll
       for (int j = 0; j < VEC; ++j) s[u][j] = fmaf(alpha, s[u][j], uu * kh[j]);
-      if (active) RowIO<S, VEC>::store(ptr[u], s[u]);
+      if (active) RowIO<S, VEC>::store(rows_base + (int64_t)r * D, s[u]);
       if (lane % LPR == 0) os[r] = scale * fmaf(alpha, sq[u], uu * kqh);
     }
   }

@@ -689,15 +689,21 @@ teardown:
 
 // ------------------------------------------------------------------------ chain
 
-// shared memory of the chain kernel (offsets from a 1024-aligned base). Per stage:
-//   WQ : [-W atom0 | Q atom0 | -W atom1 | Q atom1]: [-W; Q] is one K-major 128-row operand
-//   K  : 2 atoms
-//   U~ (this slice) then Mqk: [U~; Mqk] is a 128-row operand whose top half only lands in
-//        rows nobody reads; then the low half of U~ (this slice)
-constexpr int kSWQ = 0, kSK = 32768, kSU = 49152, kSM = 57344, kSUl = 65536;
-constexpr int kSVec = 73728;                  // the chunk's row scales (kVecBytes)
+// shared memory of the chain kernel (offsets from a 1024-aligned base). A stage holds one
+// chunk in two parts with their own loads and releases, so that the data the serial path
+// needs first is requested as early as possible:
+//   part A (read by the seed and rA; released as soon as rA has completed):
+//     WQ : [-W atom0 | Q atom0 | -W atom1 | Q atom1]: [-W; Q] is one K-major 128-row operand
+//     U~ and U~lo (this slice)
+//   part B (read by dS, O2 and the epilogues; released once the chunk's output is out):
+//     K : 2 atoms, then Mqk: [K atom1; Mqk] is O2's 128-row A operand, whose top half only
+//         lands in rows nobody reads; then the chunk's row scales
+constexpr int kSWQ = 0, kSU = 32768, kSUl = 40960;          // part A: 48 KB
+constexpr int kSB = 49152;                                  // part B
+constexpr int kSK = kSB, kSM = kSB + 16384, kSVec = kSB + 24576;
 constexpr int kStage = 74752;                 // one chunk (1024-aligned)
-constexpr int kStageTx = 32768 + 16384 + 8192 + 8192 + 8192 + kVecBytes;   // bytes its loads deliver
+constexpr int kStageTxA = 32768 + 8192 + 8192;              // bytes the part A loads deliver
+constexpr int kStageTxB = 16384 + 8192 + kVecBytes;         // and part B
 constexpr int kCS = 2 * kStage;               // S0^T bf16, MN-major [128][64]: 16 KB
 constexpr int kCU = kCS + 16384;              // U   bf16 [64][64]: 8 KB (for O2)
 constexpr int kCUp = kCU + 8192;              // U' = diag(e^{G_L - G_r}/|k_r|) U as a bf16 hi + lo
@@ -714,7 +720,7 @@ constexpr int kOBarrier = 1;                  // named barrier of the four outpu
 // TMEM columns (M = 128 accumulators, lane = row). A = [-W; Q] S0^T is accumulated in two
 // K halves (lo: dk 0..63, hi: dk 64..127) by the two issuers, each double-buffered; the lo
 // half starts from [I; 0] U~, so its rows 0..63 plus the hi half's are U itself. dS^T in two
-// K halves (tokens 0..31, 32..63); O2 = [U~; Mqk] U.
+// K halves (tokens 0..31, 32..63); O2 = [K atom1; Mqk] U (rows 64..127 used).
 constexpr uint32_t kTAlo = 0, kTAhi = 128, kTdSlo = 256, kTdShi = 320, kTO2 = 384;
 
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
@@ -772,24 +778,31 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kCBar);
-  uint64_t* bar_tma = bars;        // [2] stage landed
-  uint64_t* bar_free = bars + 2;   // [2] stage no longer read (8 compute warps)
-  uint64_t* bar_A0 = bars + 4;
-  uint64_t* bar_A1 = bars + 5;
-  uint64_t* bar_B0 = bars + 6;
-  uint64_t* bar_B1 = bars + 7;
-  uint64_t* bar_O = bars + 8;
-  uint64_t* bar_U0 = bars + 9;     // U, U' rows 0..31 written (the 2 warps of quadrant 0)
-  uint64_t* bar_U1 = bars + 10;    // rows 32..63 (quadrant 1)
-  uint64_t* bar_S0 = bars + 11;    // state bf16 rows 0..63 written (quadrants 0, 1: 4 warps)
-  uint64_t* bar_S1 = bars + 12;    // rows 64..127 (quadrants 2, 3)
-  uint64_t* bar_drain = bars + 15; // [3] on an early exit: each issuing thread's MMAs have completed
-  uint64_t* bar_seed = bars + 18;  // [2] A-lo buffer b holds [I; 0] (U~ + U~lo) of its next chunk
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
+  uint64_t* bar_tma = bars;        // [2] part A of stage b landed
+  uint64_t* bar_tmb = bars + 2;    // [2] part B landed
+  uint64_t* bar_free_a = bars + 4; // [2] part A no longer read (rA has completed)
+  uint64_t* bar_free = bars + 6;   // [2] part B no longer read (8 compute warps)
+  uint64_t* bar_A0 = bars + 8;
+  uint64_t* bar_A1 = bars + 9;
+  uint64_t* bar_B0 = bars + 10;
+  uint64_t* bar_B1 = bars + 11;
+  uint64_t* bar_O = bars + 12;
+  uint64_t* bar_U0 = bars + 13;    // U, U' rows 0..31 written (the 2 warps of quadrant 0)
+  uint64_t* bar_U1 = bars + 14;    // rows 32..63 (quadrant 1)
+  uint64_t* bar_S0 = bars + 15;    // state bf16 rows 0..63 written (quadrants 0, 1: 4 warps)
+  uint64_t* bar_S1 = bars + 16;    // rows 64..127 (quadrants 2, 3)
+  uint64_t* bar_drain = bars + 17; // [3] on an early exit: each issuing thread's MMAs have completed
+  uint64_t* bar_seed = bars + 20;  // [2] A-lo buffer b holds [I; 0] (U~ + U~lo) of its next chunk
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
 
   if (tid == 0) {
-    for (int i = 0; i < 2; ++i) { mbar_init(&bar_tma[i], 1); mbar_init(&bar_free[i], kComputeWarps); }
-    for (int i = 4; i < 9; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar_tma[i], 1);
+      mbar_init(&bar_tmb[i], 1);
+      mbar_init(&bar_free_a[i], 1);
+      mbar_init(&bar_free[i], kComputeWarps);
+    }
+    for (int i = 8; i < 13; ++i) mbar_init(&bars[i], 1);
     mbar_init(bar_U0, 2);
     mbar_init(bar_U1, 2);
     mbar_init(bar_S0, 4);
@@ -837,23 +850,30 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
       // done, it also seeds that buffer with [I; 0] (U~ + U~lo) (rows 0..63 = U~, rows
       // 64..127 = 0), off the issuers' serial path.
       tma_prefetch_desc(&map_q);
-      auto issue_loads = [&](int c, int b) {
-        const int64_t t0 = bos + (int64_t)c * C;
+      auto issue_a = [&](int c, int b) {   // part A of chunk c into stage b
         const int32_t slot = slot0 + c;
+        const int64_t t0 = bos + (int64_t)c * C;
         uint8_t* stg = sm + b * kStage;
         const int32_t wrow = (int32_t)(((int64_t)slot * Hv + h) * 2 * C);
-        mbar_arrive_expect_tx(&bar_tma[b], kStageTx);
+        mbar_arrive_expect_tx(&bar_tma[b], kStageTxA);
         for (int hh = 0; hh < 2; ++hh) {
           tma_load_2d(stg + kSWQ + hh * 16384, &map_wu, hh * 64, wrow, &bar_tma[b]);
           tma_load_2d(stg + kSWQ + hh * 16384 + 8192, &map_q, hk * D + hh * 64, (int32_t)t0, &bar_tma[b]);
-          tma_load_2d(stg + kSK + hh * 8192, &map_k, hk * D + hh * 64, (int32_t)t0, &bar_tma[b]);
         }
         tma_load_2d(stg + kSU, &map_wu, tile * DT, wrow + C, &bar_tma[b]);
-        tma_load_2d(stg + kSM, &map_mq, 0, (int32_t)(((int64_t)slot * Hv + h) * C), &bar_tma[b]);
         tma_load_2d(stg + kSUl, &map_ul, tile * DT, (int32_t)(((int64_t)slot * Hv + h) * C), &bar_tma[b]);
-        bulk_load(stg + kSVec, ws_ro + L.vecs + ((size_t)slot * Hv + h) * kVecBytes, kVecBytes, &bar_tma[b]);
       };
-      auto seed = [&](int c) {   // chunk c's stage has landed and its A-lo buffer is free
+      auto issue_b = [&](int c, int b) {   // part B of chunk c into stage b
+        const int32_t slot = slot0 + c;
+        const int64_t t0 = bos + (int64_t)c * C;
+        uint8_t* stg = sm + b * kStage;
+        mbar_arrive_expect_tx(&bar_tmb[b], kStageTxB);
+        for (int hh = 0; hh < 2; ++hh)
+          tma_load_2d(stg + kSK + hh * 8192, &map_k, hk * D + hh * 64, (int32_t)t0, &bar_tmb[b]);
+        tma_load_2d(stg + kSM, &map_mq, 0, (int32_t)(((int64_t)slot * Hv + h) * C), &bar_tmb[b]);
+        bulk_load(stg + kSVec, ws_ro + L.vecs + ((size_t)slot * Hv + h) * kVecBytes, kVecBytes, &bar_tmb[b]);
+      };
+      auto seed = [&](int c) {   // chunk c's part A has landed and its A-lo buffer is free
         const int b = c & 1;
         const uint32_t ta = tmem + kTAlo + 64 * b;
         tc_fence_after();
@@ -863,28 +883,38 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
         for (int kk = 0; kk < 4; ++kk) mma_bf16(ta, dI + 2 * kk, dUtl + soff(b) + 128 * kk, kIA, true);
         mma_commit(&bar_seed[b]);
       };
-      issue_loads(0, 0);
-      if (nc > 1) issue_loads(1, 1);
-      int c = 0, issued = nc > 1 ? 2 : 1;
+      int issued_a = nc > 1 ? 2 : 1, issued_b = issued_a;
+      for (int c = 0; c < issued_a; ++c) { issue_a(c, c); issue_b(c, c); }
       bool good = mbar_wait(&bar_tma[0], 0u, err_word, kErrChainTma);
       if (good) seed(0);
-      for (; good && c < nc; ++c) {
-        // chunk c + 1's seed: its stage; its buffer was last used by chunk c - 1, whose stage
-        // release was awaited before chunk c + 1's loads were issued
+      for (int c = 0; good && c < nc; ++c) {
+        const uint32_t ph = (uint32_t)(c >> 1) & 1u;
+        // chunk c + 1's seed: its part A; its A-lo buffer was last read by chunk c - 1
         if (c + 1 < nc) {
           if (!(good = mbar_wait(&bar_tma[(c + 1) & 1], (uint32_t)((c + 1) >> 1) & 1u, err_word, kErrChainTma))) break;
+          if (c >= 1 && !(good = mbar_wait(&bar_free[(c - 1) & 1], (uint32_t)((c - 1) >> 1) & 1u, err_word,
+                                           kErrChainTma))) break;
           seed(c + 1);
         }
-        if (c + 2 < nc) {
-          if (!(good = mbar_wait(&bar_free[c & 1], (uint32_t)(c >> 1) & 1u, err_word, kErrChainTma))) break;
-          issue_loads(c + 2, c & 1);
-          issued = c + 3;
+        if (c + 2 < nc) {   // chunk c + 2 into stage c % 2: part A once rA(c) is done, B after c
+          if (!(good = mbar_wait(&bar_free_a[c & 1], ph, err_word, kErrChainTma))) break;
+          issue_a(c + 2, c & 1);
+          issued_a = c + 3;
+          if (!(good = mbar_wait(&bar_free[c & 1], ph, err_word, kErrChainTma))) break;
+          issue_b(c + 2, c & 1);
+          issued_b = c + 3;
         }
       }
       if (!good) {   // gave up: let the loads in flight land (bounded) before exiting
-        for (int b = 0; b < 2 && b < issued; ++b) {   // the last chunk loaded into stage b
-          const int last = (issued - 1) - (((issued - 1) - b) & 1);
-          mbar_wait(&bar_tma[b], (uint32_t)(last >> 1) & 1u, nullptr, 0);
+        for (int b = 0; b < 2; ++b) {   // the last chunk loaded into each part of stage b
+          if (b < issued_a) {
+            const int last = (issued_a - 1) - (((issued_a - 1) - b) & 1);
+            mbar_wait(&bar_tma[b], (uint32_t)(last >> 1) & 1u, nullptr, 0);
+          }
+          if (b < issued_b) {
+            const int last = (issued_b - 1) - (((issued_b - 1) - b) & 1);
+            mbar_wait(&bar_tmb[b], (uint32_t)(last >> 1) & 1u, nullptr, 0);
+          }
         }
       }
       mma_commit(&bar_drain[2]);   // every seed MMA has completed before TMEM is released
@@ -895,7 +925,7 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     uint64_t* bar_Sp = part ? bar_S1 : bar_S0;
     const uint64_t dWQ = smem_desc(st0 + kSWQ, 16u, 1024u) + (uint64_t)(part * (16384 >> 4));
     const uint64_t dK = smem_desc(st0 + kSK, 8192u, 1024u);
-    const uint64_t dUM = smem_desc(st0 + kSU, 16u, 1024u);
+    const uint64_t dUM = smem_desc(st0 + kSK + 8192, 16u, 1024u);   // [K atom1; Mqk]
     auto issue_rA = [&](int b) {
       const uint32_t ta = tmem + (part ? kTAhi : kTAlo) + 64 * b;
 #pragma unroll
@@ -912,7 +942,8 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     issue_rA(0);
     for (int c = 0; c < nc; ++c) {
       const int b = c & 1;
-      if (!mbar_spin(part ? bar_U1 : bar_U0, (uint32_t)c & 1u, err_word, kErrChainMma)) break;
+      if (!mbar_spin(part ? bar_U1 : bar_U0, (uint32_t)c & 1u, err_word, kErrChainMma) ||
+          !mbar_spin(&bar_tmb[b], (uint32_t)(c >> 1) & 1u, err_word, kErrChainTma)) break;
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < 2; ++kk) {   // dS^T = K^T (U' + U'lo) over tokens [32 part, 32 part + 32)
@@ -979,10 +1010,12 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
       const int64_t t0 = bos + (int64_t)c * C;
       const int len = (int)(eos - t0 < C ? eos - t0 : C);
       const float* vec = reinterpret_cast<const float*>(sm + b * kStage + kSVec);
+      if (!(ok = mbar_wait(&bar_tmb[b], (uint32_t)(c >> 1) & 1u, err_word, kErrChainTma))) break;
 
       // U = U~ + (-W S0^T): rows 0..63 (quadrants 0, 1) -> U and U' in bf16
       if (!(ok = mbar_wait(bar_A0, phA, err_word, kErrChainMma) && mbar_wait(bar_A1, phA, err_word, kErrChainMma))) break;
       phA ^= 1u;
+      if (warp == 0 && lane == 0) mbar_arrive(&bar_free_a[b]);   // rA(c) and its seed are done
       tc_fence_after();
       float os = 0.f;
       if (quad < 2) {
