@@ -27,6 +27,17 @@ __device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uin
   lo = *reinterpret_cast<uint32_t*>(&l);
 }
 
+// The same split without the conversion unit (integer and fp32 ALU only): hi is x rounded
+// to the nearest bf16 by adding half a bf16 unit in the last place to the bit pattern (half-way
+// cases go away from zero), lo = x - hi (exact in fp32) truncated to bf16, so
+// |x - hi - lo| < 2^-15 |x|.
+__device__ __forceinline__ void split_bf16x2_alu(float a, float b, uint32_t& hi, uint32_t& lo) {
+  const uint32_t ha = (__float_as_uint(a) + 0x8000u) & 0xFFFF0000u;
+  const uint32_t hb = (__float_as_uint(b) + 0x8000u) & 0xFFFF0000u;
+  hi = __byte_perm(ha, hb, 0x7632);
+  lo = __byte_perm(__float_as_uint(a - __uint_as_float(ha)), __float_as_uint(b - __uint_as_float(hb)), 0x7632);
+}
+
 // Recurrent-state elements in HBM: fp32, or bf16 storage (widened to fp32 on load, rounded
 // to nearest-even once on store).
 __device__ __forceinline__ float state_load(const void* p, int64_t i, bool bf) {

@@ -720,7 +720,9 @@ constexpr int kOBarrier = 1;                  // named barrier of the four outpu
 // TMEM columns (M = 128 accumulators, lane = row). A = [-W; Q] S0^T is accumulated in two
 // K halves (lo: dk 0..63, hi: dk 64..127) by the two issuers, each double-buffered; the lo
 // half starts from [I; 0] U~, so its rows 0..63 plus the hi half's are U itself. dS^T in two
-// K halves (tokens 0..31, 32..63); O2 = [K atom1; Mqk] U (rows 64..127 used).
+// K halves (tokens 0..31, 32..63); O2 = [K atom1; Mqk] U (rows 64..127 used), double-buffered:
+// chunk c's O2 is issued once chunk c's loads have landed, and those were requested only after
+// chunk c - 2's output warps had read the same buffer.
 constexpr uint32_t kTAlo = 0, kTAhi = 128, kTdSlo = 256, kTdShi = 320, kTO2 = 384;
 
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
@@ -833,7 +835,8 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
 
   if (warp >= kComputeWarps) {
     // ---------------------------------------------------------------- issuers / producer
-    if (lane != 0 || nc == 0) goto done;
+    // the producer is one lane; each issuer is a whole warp, one elected lane of which issues
+    if (nc == 0 || (warp == kComputeWarps + 2 && lane != 0)) goto done;
     const uint32_t st0 = smem_u32(sm);
     auto soff = [](int b) { return (uint64_t)(b * (kStage >> 4)); };
     const uint64_t dS = smem_desc(smem_u32(sm + kCS), 8192u, 1024u);
@@ -930,46 +933,50 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
       const uint32_t ta = tmem + (part ? kTAhi : kTAlo) + 64 * b;
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(ta, dWQ + soff(b) + 2 * kk, dS + 128 * (4 * part + kk), kIA, part == 0 || kk > 0);
-      mma_commit(part ? bar_A1 : bar_A0);
+        mma_bf16_warp(ta, dWQ + soff(b) + 2 * kk, dS + 128 * (4 * part + kk), kIA, part == 0 || kk > 0);
+      mma_commit_warp(part ? bar_A1 : bar_A0);
     };
     // rA(0): chunk 0 landed (and, for the lo half, was seeded) and this half of the initial
     // state is in shared memory
-    if (!mbar_spin(&bar_tma[0], 0u, err_word, kErrChainTma) ||
-        (part == 0 && !mbar_spin(&bar_seed[0], 0u, err_word, kErrChainMma)) ||
-        !mbar_spin(bar_Sp, 0u, err_word, kErrChainMma)) goto done;
+    // (every wait's outcome is made warp-uniform: the warp issues together or leaves together)
+    if (__any_sync(0xffffffffu, !mbar_spin(&bar_tma[0], 0u, err_word, kErrChainTma) ||
+                                    (part == 0 && !mbar_spin(&bar_seed[0], 0u, err_word, kErrChainMma)) ||
+                                    !mbar_spin(bar_Sp, 0u, err_word, kErrChainMma))) goto done;
     tc_fence_after();
     issue_rA(0);
     for (int c = 0; c < nc; ++c) {
       const int b = c & 1;
-      if (!mbar_spin(part ? bar_U1 : bar_U0, (uint32_t)c & 1u, err_word, kErrChainMma) ||
-          !mbar_spin(&bar_tmb[b], (uint32_t)(c >> 1) & 1u, err_word, kErrChainTma)) break;
+      if (__any_sync(0xffffffffu, !mbar_spin(part ? bar_U1 : bar_U0, (uint32_t)c & 1u, err_word, kErrChainMma) ||
+                                      !mbar_spin(&bar_tmb[b], (uint32_t)(c >> 1) & 1u, err_word, kErrChainTma))) break;
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < 2; ++kk) {   // dS^T = K^T (U' + U'lo) over tokens [32 part, 32 part + 32)
-        mma_bf16(tmem + (part ? kTdShi : kTdSlo), dK + soff(b) + 128 * (2 * part + kk),
-                 dUp + 128 * (2 * part + kk), kIB, kk > 0);
-        mma_bf16(tmem + (part ? kTdShi : kTdSlo), dK + soff(b) + 128 * (2 * part + kk),
-                 dUpl + 128 * (2 * part + kk), kIB, true);
+        mma_bf16_warp(tmem + (part ? kTdShi : kTdSlo), dK + soff(b) + 128 * (2 * part + kk),
+                      dUp + 128 * (2 * part + kk), kIB, kk > 0);
+        mma_bf16_warp(tmem + (part ? kTdShi : kTdSlo), dK + soff(b) + 128 * (2 * part + kk),
+                      dUpl + 128 * (2 * part + kk), kIB, true);
       }
-      mma_commit(part ? bar_B1 : bar_B0);
+      mma_commit_warp(part ? bar_B1 : bar_B0);
       if (part == 1) {   // rows 64..127 of [U~; Mqk] U, once all of U is written
-        if (!mbar_spin(bar_U0, (uint32_t)c & 1u, err_word, kErrChainMma)) break;
+        if (__any_sync(0xffffffffu, !mbar_spin(bar_U0, (uint32_t)c & 1u, err_word, kErrChainMma))) break;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) mma_bf16(tmem + kTO2, dUM + soff(b) + 2 * kk, dU + 128 * kk, kIA, kk > 0);
-        mma_commit(bar_O);
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16_warp(tmem + kTO2 + 64 * b, dUM + soff(b) + 2 * kk, dU + 128 * kk, kIA, kk > 0);
+        mma_commit_warp(bar_O);
       }
       if (c + 1 < nc) {
-        if (!mbar_spin(&bar_tma[b ^ 1], (uint32_t)((c + 1) >> 1) & 1u, err_word, kErrChainTma) ||
-            (part == 0 && !mbar_spin(&bar_seed[b ^ 1], (uint32_t)((c + 1) >> 1) & 1u, err_word, kErrChainMma)) ||
-            !mbar_spin(bar_Sp, (uint32_t)(c + 1) & 1u, err_word, kErrChainMma)) break;
+        if (__any_sync(0xffffffffu,
+                       !mbar_spin(&bar_tma[b ^ 1], (uint32_t)((c + 1) >> 1) & 1u, err_word, kErrChainTma) ||
+                       (part == 0 && !mbar_spin(&bar_seed[b ^ 1], (uint32_t)((c + 1) >> 1) & 1u, err_word,
+                                                kErrChainMma)) ||
+                       !mbar_spin(bar_Sp, (uint32_t)(c + 1) & 1u, err_word, kErrChainMma))) break;
         tc_fence_after();
         issue_rA(b ^ 1);
       }
     }
-    // every MMA this thread issued has completed before the tensor memory is released
-    mma_commit(&bar_drain[part]);
+    // every MMA this warp issued has completed before the tensor memory is released
+    mma_commit_warp(&bar_drain[part]);
     mbar_wait(&bar_drain[part], 0u, nullptr, 0);
     goto done;
   }
@@ -1036,7 +1043,7 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
             const float x1 = __uint_as_float(a0[c8 * 8 + 2 * q + 1]) + __uint_as_float(a1[c8 * 8 + 2 * q + 1]);
             __nv_bfloat162 ub = __floats2bfloat162_rn(x0, x1);
             u[q] = *reinterpret_cast<uint32_t*>(&ub);
-            split_bf16x2(us * x0, us * x1, hi[q], lo[q]);
+            split_bf16x2_alu(us * x0, us * x1, hi[q], lo[q]);
           }
           const uint32_t off = sw128_off(r, half * 32 + c8 * 8);
           *reinterpret_cast<uint4*>(sm + kCU + off) = make_uint4(u[0], u[1], u[2], u[3]);
@@ -1094,7 +1101,7 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
 #pragma unroll
         for (int e = 0; e < 32; ++e) o1[e] = os * (__uint_as_float(a0[e]) + __uint_as_float(a1[e]));
         uint32_t o2[32];
-        tmem_ld32_async(tq + kTO2 + half * 32, o2);
+        tmem_ld32_async(tq + kTO2 + 64 * b + half * 32, o2);
         tmem_wait_ld(o2);
         if (len == C) {   // a full chunk: stage the 64 x 64 tile, one TMA store
           uint8_t* ost = sm + kCO + b * 8192;
