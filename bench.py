@@ -432,7 +432,7 @@ def main():
                 "frac_of_sustained_peak": pre_tflops / tc_sust,
                 "algorithmic_per_launch": prefill_flops_per_token() * T,
                 "traffic": traffic("prefill", T),
-                "traffic_before_block_state_store": TRAFFIC_BEFORE_CHANGE["prefill"] * T}
+                "kernels": prefill_kernel_split(T, pre_avg, tc_tflops)}
     elif dominant == "decode":
         roof = {"kernel": "gdn_decode_step", "bound": "hbm", "achieved": dec_gbs, "peak": hbm_gbs,
                 "unit": "GB/s", "frac": dec_gbs / hbm_gbs, "peak_kind": f"HBM copy ({peak_src})",
@@ -532,13 +532,41 @@ def gdn_prefill_launches() -> int:
 # DRAM traffic (bytes, dram__bytes_read.sum + dram__bytes_write.sum) from one ncu capture
 # of each kernel on the small case (T = 8192, decode batch 64), per unit processed (token
 # for the prefill kernels and the conv, sequence for the decode step), scaled to the
-# benchmark's launch; None when the kernel changed since the capture.
-TRAFFIC_PER_UNIT = {"prefill": None, "conv": 289.54e6 / 8192, "decode": 355.05e6 / 64}
+# benchmark's launch; None when the kernel changed since the capture. The prefill figure is
+# the intra-chunk kernel's 467.18 MB plus the chain kernel's 510.90 MB.
+TRAFFIC_PER_UNIT = {"prefill": (467.18e6 + 510.90e6) / 8192, "conv": 289.54e6 / 8192,
+                    "decode": 354.58e6 / 64}
 
-# The chain kernel gained the block-boundary state store (a branch the benchmark never
-# takes: no block states are requested) after its capture; the figure from that capture,
-# intra-chunk + chain kernels, is reported beside the roofline as context only.
-TRAFFIC_BEFORE_CHANGE = {"prefill": (375.06e6 + 405.27e6) / 8192}
+# The chunked prefill's two kernels: their share of its FLOPs (from the chunked form: the
+# intra-chunk kernel forms K K^T and Q K^T per key head, solves the triangular system and
+# builds U~ = P V, W = Pk K and Mqk; the chain applies [-W; Q] S0^T, K^T U' and Mqk U), their
+# share of its time (the ncu launch list of the 65536-token run: 1442.9 and 2058.6 us of
+# 3504.2 us) and their DRAM traffic per token from the same captures as above.
+PREFILL_KERNELS = {
+    "chunk_intra": {"time_share": 1442.9 / 3504.2, "traffic_per_token": 467.18e6 / 8192},
+    "chunk_chain": {"time_share": 2058.6 / 3504.2, "traffic_per_token": 510.90e6 / 8192},
+}
+
+
+def prefill_kernel_flops_per_token(kernel: str, sh=SHAPE, C=64):
+    d, G = sh.dk, sh.Hv // sh.Hk
+    if kernel == "chunk_chain":
+        return sh.Hv * (6 * d * d + 2 * C * d)
+    return sh.Hv * (4 * C * d / G + C * C / 3 + 4 * C * d)
+
+
+def prefill_kernel_split(T: int, prefill_ms: float, peak_tflops: float) -> dict:
+    """Per-kernel FLOPs and traffic of one prefill launch, with each kernel's time taken as
+    its launch-list share of the measured call time."""
+    out = {}
+    for k, v in PREFILL_KERNELS.items():
+        flops = prefill_kernel_flops_per_token(k) * T
+        ms = prefill_ms * v["time_share"]
+        out[k] = {"flops": flops, "time_share": v["time_share"], "ms": ms,
+                  "tflops": flops / (ms / 1e3) / 1e12,
+                  "frac": flops / (ms / 1e3) / 1e12 / peak_tflops,
+                  "traffic": v["traffic_per_token"] * T}
+    return out
 
 
 def traffic(kernel: str, units: int):

@@ -50,6 +50,30 @@ def test_prefill_flops_match_gemm_list(bench, shape, C):
     assert bench.prefill_flops_per_token(shape, C) == pytest.approx(expect, rel=1e-12)
 
 
+# which kernel applies each product of chunk_gemms (same order); the triangular inverse is
+# the intra-chunk kernel's
+KERNEL_OF = ["chunk_intra", "chunk_intra", "chunk_intra", "chunk_intra",
+             "chunk_chain", "chunk_chain", "chunk_chain", "chunk_chain"]
+
+
+@pytest.mark.parametrize("shape,C", [(W.QWEN35_27B, 64), (W.QWEN35_9B, 64), (W.TINY, 16)])
+def test_prefill_kernel_split_matches_gemm_list(bench, shape, C):
+    """The per-kernel FLOP attribution: each kernel's GEMMs from the list above, and the two
+    kernels together account for the whole call."""
+    G = shape.Hv // shape.Hk
+    for kernel in ("chunk_intra", "chunk_chain"):
+        per_chunk = sum(2 * m * n * k * w for (m, n, k, w), kk in zip(chunk_gemms(C, shape.dk, G), KERNEL_OF)
+                        if kk == kernel)
+        if kernel == "chunk_intra":
+            per_chunk += C ** 3 / 3
+        assert bench.prefill_kernel_flops_per_token(kernel, shape, C) == pytest.approx(
+            shape.Hv * per_chunk / C, rel=1e-12)
+    split = bench.prefill_kernel_split(65536, 3.5, 1590.0)
+    assert sum(v["flops"] for v in split.values()) == pytest.approx(
+        bench.prefill_flops_per_token() * 65536, rel=1e-12)
+    assert sum(v["time_share"] for v in split.values()) == pytest.approx(1.0, abs=2e-3)
+
+
 def test_prefill_roofline_time_27b_64k(bench):
     """7.67 MFLOP per token for the 27B layer; at 1,391.6 TFLOP/s (sustained bf16) the
     65,536-token prefill cannot take less than 0.361 ms."""
