@@ -23,7 +23,6 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kMaxTok = 8;
 constexpr float kEps = 1e-6f;
 
 // Four consecutive state values, streamed (evict-first): fp32 storage, or bf16 storage
@@ -46,12 +45,12 @@ template <> struct Quad<bf16> {
   }
 };
 
-template <typename T, int D, typename S>
+template <typename T, int D, typename S, int NT>
 __global__ void __launch_bounds__(kThreads, 3)
 decode_tokens_kernel(const T* __restrict__ x, const T* __restrict__ conv_w, T* __restrict__ conv_state,
                      const float* __restrict__ g, const float* __restrict__ beta,
-                     S* __restrict__ state, T* __restrict__ o, int32_t Hk, int32_t Hv,
-                     int32_t n_tok, float scale) {
+                     S* __restrict__ state, T* __restrict__ o, int32_t Hk, int32_t Hv, float scale) {
+  constexpr int n_tok = NT;
   constexpr int VEC = D >= 32 ? D / 32 : 1;
   const int G = Hv / Hk;
   const int32_t Cc = 2 * Hk * D + Hv * D;
@@ -62,7 +61,8 @@ decode_tokens_kernel(const T* __restrict__ x, const T* __restrict__ conv_w, T* _
 
   extern __shared__ float smem[];
   float* ys = smem;                       // [n_tok][n_local]
-  float* os = smem + n_tok * n_local;     // [n_tok][G * D], then k_t.q_t [n_tok]
+  float* os = smem + n_tok * n_local;     // [n_tok][G * D], then k_t.q_t [n_tok], then
+                                          // (alpha_t, beta_t) per value head [G][n_tok]
 
   // 1. conv + SiLU of every token over this CTA's channels; the taps advance by n_tok.
   for (int lv = threadIdx.x; lv < n_local / 4; lv += kThreads) {
@@ -71,23 +71,16 @@ decode_tokens_kernel(const T* __restrict__ x, const T* __restrict__ conv_w, T* _
     if (lc < D) gc = hk * D + lc;
     else if (lc < 2 * D) gc = Hk * D + hk * D + (lc - D);
     else gc = 2 * Hk * D + hk * G * D + (lc - 2 * D);
-    float win[3 + kMaxTok][4], wr[16];
+    float win[3 + NT][4], wr[16];
     T* cs = conv_state + b * 3 * Cc + gc;
 #pragma unroll
     for (int j = 0; j < 3; ++j) VecIO<T, 4>::load(cs + j * Cc, win[j]);
 #pragma unroll
-    for (int t = 0; t < kMaxTok; ++t) {
-      if (t < n_tok) {
-        VecIO<T, 4>::load(x + (b * n_tok + t) * Cc + gc, win[3 + t]);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) win[3 + t][i] = 0.f;
-      }
-    }
+    for (int t = 0; t < NT; ++t) VecIO<T, 4>::load(x + (b * n_tok + t) * Cc + gc, win[3 + t]);
     VecIO<T, 16>::load(conv_w + (int64_t)gc * 4, wr);
 #pragma unroll
-    for (int t = 0; t < kMaxTok; ++t) {
-      if (t < n_tok) {
+    for (int t = 0; t < NT; ++t) {
+      {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           float z = wr[i * 4 + 0] * win[t][i];
@@ -140,6 +133,13 @@ decode_tokens_kernel(const T* __restrict__ x, const T* __restrict__ conv_w, T* _
     }
     if (lane == 0) kqs[warp] = kq * iq * ik;
   }
+  // the decay and write strength of each (value head, token), once per CTA
+  float2* ab = reinterpret_cast<float2*>(kqs + ((n_tok + 1) & ~1));   // 8-byte aligned
+  for (int i = threadIdx.x; i < G * n_tok; i += kThreads) {
+    const int hh = i / n_tok, t = i % n_tok;
+    const int64_t gi = (b * n_tok + t) * Hv + hk * G + hh;
+    ab[i] = make_float2(expf(g[gi]), beta[gi]);
+  }
   __syncthreads();
 
   // 3. stream the G * D state rows of this CTA, each through every token. A row is split
@@ -171,15 +171,14 @@ decode_tokens_kernel(const T* __restrict__ x, const T* __restrict__ conv_w, T* _
   for (int r0 = warp * RPW; r0 < rows; r0 += kWarps * RPW) {
     const int r = r0 + lane / L;
     const bool live = r < rows;
-    const int h = hk * G + (live ? r : 0) / D;
+    const float2* abh = ab + ((live ? r : 0) / D) * n_tok;   // this row's value head
     S* ptr = row_ptr(r);
     float s[SEG];
 #pragma unroll
     for (int j = 0; j < SEG; ++j) s[j] = s_next[j];
     if (r0 + kWarps * RPW < rows) load_row(r + kWarps * RPW, s_next);
 #pragma unroll
-    for (int t = 0; t < kMaxTok; ++t) {
-      if (t >= n_tok) break;
+    for (int t = 0; t < NT; ++t) {
       const float* qt = ys + t * n_local + seg * 4;
       const float* kt = qt + D;
       float kv[SEG], a = 0.f, c = 0.f;
@@ -197,8 +196,8 @@ decode_tokens_kernel(const T* __restrict__ x, const T* __restrict__ conv_w, T* _
         c += __shfl_xor_sync(0xffffffffu, c, m);
       }
       if (live) {
-        const float alpha = expf(g[(b * n_tok + t) * Hv + h]);
-        const float bt = beta[(b * n_tok + t) * Hv + h];
+        const float2 sc = abh[t];
+        const float alpha = sc.x, bt = sc.y;
         const float uu = bt * (ys[t * n_local + 2 * D + r] - alpha * a);
 #pragma unroll
         for (int j = 0; j < SEG; ++j) s[j] = fmaf(alpha, s[j], uu * kv[j]);
@@ -220,21 +219,38 @@ decode_tokens_kernel(const T* __restrict__ x, const T* __restrict__ conv_w, T* _
   }
 }
 
-template <typename T, int D, typename S>
-cudaError_t launch_typed(const void* x, const void* w, void* cs, const float* g, const float* beta,
-                         void* state, void* o, int32_t B, int32_t n_tok, int32_t Hk, int32_t Hv,
-                         float scale, cudaStream_t st) {
+template <typename T, int D, typename S, int NT>
+cudaError_t launch_nt(const void* x, const void* w, void* cs, const float* g, const float* beta,
+                      void* state, void* o, int32_t B, int32_t Hk, int32_t Hv, float scale, cudaStream_t st) {
   const int G = Hv / Hk;
-  const size_t smem = sizeof(float) * (size_t)n_tok * ((2 + G) * D + G * D + 1);
+  // ys, os, k_t.q_t (padded to an even count), (alpha, beta) per value head and token
+  const size_t smem = sizeof(float) * ((size_t)NT * ((2 + G) * D + G * D) + ((NT + 1) & ~1) + 2 * (size_t)G * NT);
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(decode_tokens_kernel<T, D, S>,
+    cudaError_t e = cudaFuncSetAttribute(decode_tokens_kernel<T, D, S, NT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
   dim3 grid((unsigned)((int64_t)B * Hk));
-  decode_tokens_kernel<T, D, S><<<grid, kThreads, smem, st>>>(
-      (const T*)x, (const T*)w, (T*)cs, g, beta, (S*)state, (T*)o, Hk, Hv, n_tok, scale);
+  decode_tokens_kernel<T, D, S, NT><<<grid, kThreads, smem, st>>>(
+      (const T*)x, (const T*)w, (T*)cs, g, beta, (S*)state, (T*)o, Hk, Hv, scale);
   return cudaGetLastError();
+}
+
+// the token count is a template parameter, so the per-token loops are unrolled
+template <typename T, int D, typename S>
+cudaError_t launch_typed(const void* x, const void* w, void* cs, const float* g, const float* beta,
+                         void* state, void* o, int32_t B, int32_t n_tok, int32_t Hk, int32_t Hv,
+                         float scale, cudaStream_t st) {
+  switch (n_tok) {
+    case 1: return launch_nt<T, D, S, 1>(x, w, cs, g, beta, state, o, B, Hk, Hv, scale, st);
+    case 2: return launch_nt<T, D, S, 2>(x, w, cs, g, beta, state, o, B, Hk, Hv, scale, st);
+    case 3: return launch_nt<T, D, S, 3>(x, w, cs, g, beta, state, o, B, Hk, Hv, scale, st);
+    case 4: return launch_nt<T, D, S, 4>(x, w, cs, g, beta, state, o, B, Hk, Hv, scale, st);
+    case 5: return launch_nt<T, D, S, 5>(x, w, cs, g, beta, state, o, B, Hk, Hv, scale, st);
+    case 6: return launch_nt<T, D, S, 6>(x, w, cs, g, beta, state, o, B, Hk, Hv, scale, st);
+    case 7: return launch_nt<T, D, S, 7>(x, w, cs, g, beta, state, o, B, Hk, Hv, scale, st);
+    default: return launch_nt<T, D, S, 8>(x, w, cs, g, beta, state, o, B, Hk, Hv, scale, st);
+  }
 }
 
 template <typename T, typename S>
