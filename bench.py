@@ -535,7 +535,7 @@ def gdn_prefill_launches() -> int:
 # benchmark's launch; None when the kernel changed since the capture. The prefill figure is
 # the intra-chunk kernel's 467.18 MB plus the chain kernel's 510.90 MB.
 TRAFFIC_PER_UNIT = {"prefill": (467.18e6 + 510.90e6) / 8192, "conv": 289.54e6 / 8192,
-                    "decode": 354.58e6 / 64}
+                    "decode": None}
 
 # The chunked prefill's two kernels: their share of its FLOPs (from the chunked form: the
 # intra-chunk kernel forms K K^T and Q K^T per key head, solves the triangular system and

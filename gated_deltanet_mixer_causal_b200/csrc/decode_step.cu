@@ -114,6 +114,7 @@ decode_step_kernel(const T* __restrict__ x, const T* __restrict__ conv_w, T* __r
   extern __shared__ float smem[];
   float* ys = smem;                       // [(2 + G) * D]: q | k | v of the G heads
   float* os = smem + (2 + G) * D;         // [G * D] outputs
+  float2* ab = reinterpret_cast<float2*>(os + G * D);   // [G] (e^g, beta) of each value head
 
   // 1. conv + SiLU over this CTA's channels; shift the taps in place.
   const int n_local = (2 + G) * D;
@@ -144,6 +145,10 @@ decode_step_kernel(const T* __restrict__ x, const T* __restrict__ conv_w, T* __r
     VecIO<T, 8>::store(cs, t1);
     VecIO<T, 8>::store(cs + Cc, t2);
     VecIO<T, 8>::store(cs + 2 * Cc, xv);
+  }
+  if (threadIdx.x < G) {   // once per CTA rather than once per row lane
+    const int64_t gi = b * Hv + (int64_t)hk * G + threadIdx.x;
+    ab[threadIdx.x] = make_float2(expf(g[gi]), beta[gi]);
   }
   __syncthreads();
 
@@ -208,9 +213,8 @@ decode_step_kernel(const T* __restrict__ x, const T* __restrict__ conv_w, T* __r
     for (int u = 0; u < kRowUnroll; ++u) {
       const int r = r0 + u * RPW + sub;
       if (r >= rows) continue;
-      const int h = hk * G + r / D;
-      const float alpha = expf(g[b * Hv + h]);
-      const float bt = beta[b * Hv + h];
+      const float2 sc = ab[r / D];
+      const float alpha = sc.x, bt = sc.y;
       const float uu = bt * (ys[2 * D + r] - alpha * sk[u]);
 #pragma unroll
       for (int j = 0; j < VEC; ++j) s[u][j] = fmaf(alpha, s[u][j], uu * kh[j]);
@@ -230,7 +234,7 @@ cudaError_t launch_typed(const void* x, const void* w, void* cs, const float* g,
                          void* state, void* o, int32_t B, int32_t Hk, int32_t Hv, float scale,
                          cudaStream_t st) {
   const int G = Hv / Hk;
-  const size_t smem = sizeof(float) * (size_t)((2 + G) * D + G * D);
+  const size_t smem = sizeof(float) * (size_t)((2 + G) * D + G * D + 2 * G);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(decode_step_kernel<T, D, S>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
