@@ -719,11 +719,13 @@ constexpr int kOBarrier = 1;                  // named barrier of the four outpu
 
 // TMEM columns (M = 128 accumulators, lane = row). A = [-W; Q] S0^T is accumulated in two
 // K halves (lo: dk 0..63, hi: dk 64..127) by the two issuers, each double-buffered; the lo
-// half starts from [I; 0] U~, so its rows 0..63 plus the hi half's are U itself. dS^T in two
-// K halves (tokens 0..31, 32..63); O2 = [K atom1; Mqk] U (rows 64..127 used), double-buffered:
+// half starts from [I; 0] U~, so its rows 0..63 plus the hi half's are U itself. dS^T =
+// K^T [U' | U'lo] is one N = 128 accumulator whose column halves the state epilogue sums (an
+// N = 128 MMA takes about as long as an N = 64 one, so this halves the MMAs on the serial
+// path); O2 = [K atom1; Mqk] U (rows 64..127 used), double-buffered:
 // chunk c's O2 is issued once chunk c's loads have landed, and those were requested only after
 // chunk c - 2's output warps had read the same buffer.
-constexpr uint32_t kTAlo = 0, kTAhi = 128, kTdSlo = 256, kTdShi = 320, kTO2 = 384;
+constexpr uint32_t kTAlo = 0, kTAhi = 128, kTdS = 256, kTO2 = 384;
 
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
@@ -746,10 +748,9 @@ __device__ __forceinline__ void tma_store_wait_read_le1() {
 //   issuers : rA(c) = [-W; Q] S0^T in two K halves (dk rows 0..63 after the state warps of
 //             quadrants 0, 1 are done, 64..127 after quadrants 2, 3), the lo half on top of
 //             [I; 0] U~ (issued as soon as the stage lands, off the serial path);
-//             dS^T = K^T U' in two token halves (each after the U warps of its quadrant; U'
-//             is carried as a bf16 hi + lo pair on the state path, where a chunk that
-//             rewrites one key telescopes U's rows); O2 = [U~; Mqk] U after both (issued by
-//             the second issuer behind its dS half)
+//             dS^T = K^T [U' | U'lo] once all of U is written (U' is carried as a bf16
+//             hi + lo pair on the state path, where a chunk that rewrites one key
+//             telescopes U's rows), then O2 = [K atom1; Mqk] U behind it (second issuer)
 //   compute : U = rows 0..63 of rA -> U (bf16), U' (hi + lo) (quadrants 0, 1)   -> "U ready"
 //             S^T <- e^{G_L} S^T + dS^T, bf16 copy (all 8 warps)               -> "S ready"
 //             o = scale (e^{G_r}/|q_r| rows 64..127 of rA + O2) (quadrants 2, 3): a full
@@ -786,8 +787,7 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
   uint64_t* bar_free = bars + 6;   // [2] part B no longer read (8 compute warps)
   uint64_t* bar_A0 = bars + 8;
   uint64_t* bar_A1 = bars + 9;
-  uint64_t* bar_B0 = bars + 10;
-  uint64_t* bar_B1 = bars + 11;
+  uint64_t* bar_B = bars + 10;     // dS^T complete
   uint64_t* bar_O = bars + 12;
   uint64_t* bar_U0 = bars + 13;    // U, U' rows 0..31 written (the 2 warps of quadrant 0)
   uint64_t* bar_U1 = bars + 14;    // rows 32..63 (quadrant 1)
@@ -841,11 +841,11 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     auto soff = [](int b) { return (uint64_t)(b * (kStage >> 4)); };
     const uint64_t dS = smem_desc(smem_u32(sm + kCS), 8192u, 1024u);
     const uint64_t dU = smem_desc(smem_u32(sm + kCU), 8192u, 1024u);
+    // [U' | U'lo] as one MN-major B operand of N = 128 (its two 64-column atoms 8 KB apart)
     const uint64_t dUp = smem_desc(smem_u32(sm + kCUp), 8192u, 1024u);
-    const uint64_t dUpl = smem_desc(smem_u32(sm + kCUpl), 8192u, 1024u);
     const uint64_t dI = smem_desc(smem_u32(sm + kCI), 16u, 1024u);
     constexpr uint32_t kIA = idesc_bf16(128, DT, 0, 1);     // K-major A, MN-major B
-    constexpr uint32_t kIB = idesc_bf16(128, DT, 1, 1);     // MN-major A and B
+    constexpr uint32_t kIB = idesc_bf16(128, 2 * DT, 1, 1); // MN-major A and B, N = 128 (dS^T)
     const uint64_t dUt = smem_desc(st0 + kSU, 8192u, 1024u);    // U~ as an MN-major B operand
     const uint64_t dUtl = smem_desc(st0 + kSUl, 8192u, 1024u);  // and its low half
     if (warp == kComputeWarps + 2) {
@@ -946,22 +946,17 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     issue_rA(0);
     for (int c = 0; c < nc; ++c) {
       const int b = c & 1;
-      if (__any_sync(0xffffffffu, !mbar_spin(part ? bar_U1 : bar_U0, (uint32_t)c & 1u, err_word, kErrChainMma) ||
-                                      !mbar_spin(&bar_tmb[b], (uint32_t)(c >> 1) & 1u, err_word, kErrChainTma))) break;
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < 2; ++kk) {   // dS^T = K^T (U' + U'lo) over tokens [32 part, 32 part + 32)
-        mma_bf16_warp(tmem + (part ? kTdShi : kTdSlo), dK + soff(b) + 128 * (2 * part + kk),
-                      dUp + 128 * (2 * part + kk), kIB, kk > 0);
-        mma_bf16_warp(tmem + (part ? kTdShi : kTdSlo), dK + soff(b) + 128 * (2 * part + kk),
-                      dUpl + 128 * (2 * part + kk), kIB, true);
-      }
-      mma_commit_warp(part ? bar_B1 : bar_B0);
-      if (part == 1) {   // rows 64..127 of [U~; Mqk] U, once all of U is written
-        if (__any_sync(0xffffffffu, !mbar_spin(bar_U0, (uint32_t)c & 1u, err_word, kErrChainMma))) break;
+      if (part == 1) {   // once all of U is written: dS^T, then O2 behind it in the queue
+        if (__any_sync(0xffffffffu, !mbar_spin(bar_U1, (uint32_t)c & 1u, err_word, kErrChainMma) ||
+                                        !mbar_spin(bar_U0, (uint32_t)c & 1u, err_word, kErrChainMma) ||
+                                        !mbar_spin(&bar_tmb[b], (uint32_t)(c >> 1) & 1u, err_word, kErrChainTma))) break;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
+        for (int kk = 0; kk < 4; ++kk)   // dS^T = K^T [U' | U'lo]: N = 128, the two halves summed later
+          mma_bf16_warp(tmem + kTdS, dK + soff(b) + 128 * kk, dUp + 128 * kk, kIB, kk > 0);
+        mma_commit_warp(bar_B);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)   // rows 64..127 of [K atom1; Mqk] U
           mma_bf16_warp(tmem + kTO2 + 64 * b, dUM + soff(b) + 2 * kk, dU + 128 * kk, kIA, kk > 0);
         mma_commit_warp(bar_O);
       }
@@ -1058,14 +1053,14 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
       }
 
       // state update: S^T <- e^{G_L} S^T + dS^T (both K halves)
-      if (!(ok = mbar_wait(bar_B0, phB, err_word, kErrChainMma) && mbar_wait(bar_B1, phB, err_word, kErrChainMma))) break;
+      if (!(ok = mbar_wait(bar_B, phB, err_word, kErrChainMma))) break;
       phB ^= 1u;
       tc_fence_after();
       {
         const float decay_last = vec[128];
         uint32_t d0[32], d1[32];
-        tmem_ld32_async(tq + kTdSlo + half * 32, d0);
-        tmem_ld32_async(tq + kTdShi + half * 32, d1);
+        tmem_ld32_async(tq + kTdS + half * 32, d0);        // K^T U'
+        tmem_ld32_async(tq + kTdS + DT + half * 32, d1);   // K^T U'lo
         tmem_wait_ld(d0, d1);
 #pragma unroll
         for (int e = 0; e < SJ; ++e)
