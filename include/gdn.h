@@ -12,8 +12,8 @@
  *   o_t    = scale * S_t q_t
  *
  * One recurrent state S (dv x dk, fp32, row index = value dimension) exists per sequence
- * and value head; the _ex decode calls can store it in bf16 instead. Value head h reads key
- * head h / (Hv / Hk).
+ * and value head; the _ex calls (prefill and decode) can store it in bf16 instead. Value
+ * head h reads key head h / (Hv / Hk).
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -57,7 +57,7 @@ typedef enum {
 typedef enum {
   GDN_F32 = 0,               /* fp32 activations; fp32 state */
   GDN_BF16 = 1               /* bf16 activations, fp32 math and state (as a state_dt of
-                                the _ex decode calls: bf16 state storage, fp32 math) */
+                                the _ex calls: bf16 state storage, fp32 math) */
 } gdn_dtype_t;
 
 /* Static string naming a status code. Never NULL. */
