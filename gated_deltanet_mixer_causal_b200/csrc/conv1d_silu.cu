@@ -18,10 +18,16 @@
 namespace gdn {
 namespace {
 
+// Tiles of 32 tokens x 512 channels, 128 threads, five CTAs per SM (96 registers, 36 KB
+// of shared memory each): one CTA's loads overlap the others' compute and stores. Measured
+// on the 27B layer at T = 65536 against the alternatives (tokens x threads x CTAs per SM):
+// 64 x 256 x 2 0.561 ms, 64 x 256 x 3 0.526, 32 x 128 x 4 0.500, 16 x 64 x 8 0.490,
+// 32 x 128 x 5 0.467 (5.7 TB/s).
 constexpr int kVec = 8;            // channels per thread
-constexpr int kTileTokens = 64;
+constexpr int kTileTokens = 32;
 constexpr int kTileVecs = 64;      // 8-channel vectors per tile (512 channels)
-constexpr int kThreads = 256;
+constexpr int kThreads = 128;
+constexpr int kMinBlocks = 5;
 constexpr int kTokPerThread = kTileTokens * kTileVecs / kThreads;   // 16
 constexpr int kRows = kTileTokens + 3;
 
@@ -53,7 +59,7 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool va
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, kMinBlocks)
 conv1d_silu_kernel(const T* __restrict__ x, T* __restrict__ y, const T* __restrict__ w,
                    const int32_t* __restrict__ cu, int32_t n_seq, int64_t T_tok, int32_t Cc,
                    const T* __restrict__ state_in, T* __restrict__ state_out) {
