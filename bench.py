@@ -533,18 +533,19 @@ def gdn_prefill_launches() -> int:
 # of each kernel on the small case (T = 8192, decode batch 64), per unit processed (token
 # for the prefill kernels and the conv, sequence for the decode step), scaled to the
 # benchmark's launch; None when the kernel changed since the capture. The prefill figure is
-# the intra-chunk kernel's 467.18 MB plus the chain kernel's 510.90 MB.
-TRAFFIC_PER_UNIT = {"prefill": (467.18e6 + 510.90e6) / 8192, "conv": 289.54e6 / 8192,
-                    "decode": None}
+# the intra-chunk kernel's 467.18 MB plus the chain kernel's 511.14 MB.
+TRAFFIC_PER_UNIT = {"prefill": (467.18e6 + 511.14e6) / 8192, "conv": 291.25e6 / 8192,
+                    "decode": 357.64e6 / 64}
 
 # The chunked prefill's two kernels: their share of its FLOPs (from the chunked form: the
 # intra-chunk kernel forms K K^T and Q K^T per key head, solves the triangular system and
 # builds U~ = P V, W = Pk K and Mqk; the chain applies [-W; Q] S0^T, K^T U' and Mqk U), their
-# share of its time (the ncu launch list of the 65536-token run: 1442.9 and 2058.6 us of
-# 3504.2 us) and their DRAM traffic per token from the same captures as above.
+# share of its time (the ncu launch list of the 65536-token run: 1434.4 and 1977.6 us of
+# 3414.7 us, the plan kernel the rest) and their DRAM traffic per token from the same
+# captures as above.
 PREFILL_KERNELS = {
-    "chunk_intra": {"time_share": 1442.9 / 3504.2, "traffic_per_token": 467.18e6 / 8192},
-    "chunk_chain": {"time_share": 2058.6 / 3504.2, "traffic_per_token": 510.90e6 / 8192},
+    "chunk_intra": {"time_share": 1434.4 / 3414.7, "traffic_per_token": 467.18e6 / 8192},
+    "chunk_chain": {"time_share": 1977.6 / 3414.7, "traffic_per_token": 511.14e6 / 8192},
 }
 
 
