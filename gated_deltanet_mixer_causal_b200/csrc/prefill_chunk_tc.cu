@@ -31,6 +31,9 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <climits>
+#include <mutex>
+
 #include "common.cuh"
 #include "launch.h"
 #include "sm100.cuh"
@@ -53,7 +56,7 @@ constexpr int kErrIntraTma = 11, kErrIntraMma = 12, kErrChainTma = 21, kErrChain
 // ------------------------------------------------------------------ workspace layout
 
 struct Ws {
-  size_t err, prefix, wu, ul, mq, vecs, total;
+  size_t err, ctr, prefix, wu, ul, mq, vecs, carry, total;
 };
 
 // Per (chunk, value head): wu = [-W (64 x 128) ; U~ (64 x 128)] bf16 rows of 128 elements,
@@ -68,18 +71,30 @@ constexpr int kVecBytes = kVecFloats * 4;
 
 __host__ __device__ inline int64_t max_slots(int64_t T, int32_t n_seq) { return (T + C - 1) / C + n_seq; }
 
+// A long single sequence is prefilled in pieces of kPieceChunks chunks (at most kMaxPieces):
+// the intra-chunk kernel of the next pieces runs beside the chain kernel of the current one,
+// which occupies only 2 Hv of the SMs. The workspace then also holds the fp32 state handed
+// from one chain piece to the next.
+constexpr int64_t kPieceChunks = 128;
+constexpr int kMaxPieces = 64;
+__host__ __device__ inline bool piece_layout(int64_t T, int32_t n_seq) {
+  return n_seq == 1 && T >= 2 * kPieceChunks * C;
+}
+
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 __host__ __device__ inline Ws ws_layout(int64_t T, int32_t n_seq, int32_t Hv) {
   Ws w;
   const size_t slots = (size_t)max_slots(T, n_seq);
   w.err = 0;
-  w.prefix = 256;
+  w.ctr = 64;      // [kMaxPieces] item counters of the intra-chunk kernel, one per piece
+  w.prefix = 512;
   w.wu = align256(w.prefix + (size_t)(n_seq + 1) * 4);
   w.ul = align256(w.wu + slots * Hv * kWuBytes);
   w.mq = align256(w.ul + slots * Hv * kUlBytes);
   w.vecs = align256(w.mq + slots * Hv * kMatBytes);
-  w.total = align256(w.vecs + slots * Hv * kVecBytes);
+  w.carry = align256(w.vecs + slots * Hv * kVecBytes);
+  w.total = align256(w.carry + (piece_layout(T, n_seq) ? (size_t)Hv * D * D * 4 : 0));
   return w;
 }
 
@@ -88,10 +103,11 @@ __host__ __device__ inline Ws ws_layout(int64_t T, int32_t n_seq, int32_t Hv) {
 __global__ void __launch_bounds__(1024) chunk_plan_kernel(const int32_t* __restrict__ cu,
                                                           int32_t n_seq, int64_t T,
                                                           int32_t* __restrict__ prefix,
-                                                          int* __restrict__ err) {
+                                                          int* __restrict__ err, int* __restrict__ ctr) {
   __shared__ int32_t warp_tot[32];
   __shared__ int32_t carry;
   if (threadIdx.x == 0) { carry = 0; *err = 0; }
+  if (threadIdx.x < kMaxPieces) ctr[threadIdx.x] = 0;
   __syncthreads();
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
   for (int base = 0; base < n_seq; base += blockDim.x) {
@@ -212,14 +228,19 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
                    const __grid_constant__ CUtensorMap map_mq, const __grid_constant__ CUtensorMap map_ul,
                    const float* __restrict__ g,
                    const float* __restrict__ beta, const int32_t* __restrict__ cu, int32_t n_seq,
-                   int64_t T, int32_t Hk, int32_t Hv, uint8_t* __restrict__ ws) {
+                   int64_t T, int32_t Hk, int32_t Hv, uint8_t* __restrict__ ws, int32_t slot_lo,
+                   int32_t slot_hi, int piece) {
   const Ws L = ws_layout(T, n_seq, Hv);
   int* err = reinterpret_cast<int*>(ws + L.err);
+  int* ctr = reinterpret_cast<int*>(ws + L.ctr) + piece;
   const int32_t* prefix = reinterpret_cast<const int32_t*>(ws + L.prefix);
-  const int32_t n_items = prefix[n_seq] * Hk;   // item = slot * Hk + key head
+  // items = (slot, key head) pairs of the slots [slot_lo, slot_hi) (item = slot * Hk + key head)
+  const int32_t n_slots = prefix[n_seq];
+  const int32_t item_lo = (slot_lo < n_slots ? slot_lo : n_slots) * Hk;
+  const int32_t n_items = (slot_hi < n_slots ? slot_hi : n_slots) * Hk;
   const int G = Hv / Hk;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if ((int32_t)blockIdx.x >= n_items) return;
+  if (item_lo + (int32_t)blockIdx.x >= n_items) return;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -238,11 +259,14 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
   uint64_t* bar_v = bar_tma + 2;   // [2] V tile of a value head landed in buffer j % 2
   uint64_t* bar_drain = bar_tma + 4;   // on an early exit: every MMA of this CTA has completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_tma + 5);
+  int32_t* next_item = reinterpret_cast<int32_t*>(bar_tma + 6);   // taken by thread 0 per item
   // loads issued into each barrier (thread 0 only): an early exit waits for the last of each
   uint32_t n_kq = 0, n_v0 = 0, n_v1 = 0;
 
-  // The CTA is persistent: it takes items blockIdx.x, + gridDim.x, ... Each item's K, Q, the
-  // first V tile and its g, beta are fetched while the previous item finishes.
+  // The CTA is persistent: its first item is item_lo + blockIdx.x, and each further one is
+  // taken from the piece's counter while the current one starts (so CTAs that become
+  // resident late, beside another kernel, take fewer). Each item's K, Q, the first V tile and
+  // its g, beta are fetched while the previous item finishes.
   struct Item { int32_t slot, hk; int64_t t0; int len; };
   auto item_at = [&](int32_t it, Item& x) {
     if (it >= n_items) return false;
@@ -305,7 +329,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
   }
   if (warp == 0) { tmem_alloc(tmem_slot, 256); tmem_relinquish(); }
   Item cur;
-  item_at((int32_t)blockIdx.x, cur);
+  item_at(item_lo + (int32_t)blockIdx.x, cur);
   fetch_gb(cur);
   tc_fence_before();
   __syncthreads();
@@ -319,11 +343,12 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
   bool ok = true;
   __syncthreads();
 
-  for (int32_t item = blockIdx.x; item < n_items; item += gridDim.x) {
+  for (;;) {
   const int32_t slot = cur.slot, hk = cur.hk;
   const int len = cur.len;
+  if (tid == 0) *next_item = item_lo + (int32_t)gridDim.x + atomicAdd(ctr, 1);   // read after a barrier
   Item nxt;
-  const bool has_next = item_at(item + (int32_t)gridDim.x, nxt);
+  bool has_next = false;
   if (warp < G) {   // inclusive cumulative log-decay of every value head, in place (2 values per lane)
     for (int j = warp; j < G; j += 4) {
       const float a0 = gAll[j * 64 + 2 * lane], a1 = gAll[j * 64 + 2 * lane + 1];
@@ -341,6 +366,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
   ok = mbar_wait(bar_tma, ph_kq, err, kErrIntraTma);
   ph_kq ^= 1u;
   if (__syncthreads_or(!ok)) { ok = false; goto teardown; }
+  has_next = item_at(*next_item, nxt);   // thread 0 wrote it before the barrier above
 
   {  // inverse L2 norms of the chunk's q and k rows (0 for rows past the sequence end)
     const int r = tid & 63;
@@ -716,6 +742,7 @@ constexpr int kChainSmem = kCBar + 256 + 1024;
 constexpr int kComputeWarps = 8;
 constexpr int kChainThreads = (kComputeWarps + 3) * 32;
 constexpr int kOBarrier = 1;                  // named barrier of the four output warps
+constexpr int kStateInitBf16 = 1, kStateFinBf16 = 2, kStateBlocksBf16 = 4;   // chain state_flags
 
 // TMEM columns (M = 128 accumulators, lane = row). A = [-W; Q] S0^T is accumulated in two
 // K halves (lo: dk 0..63, hi: dk 64..127) by the two issuers, each double-buffered; the lo
@@ -764,7 +791,8 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
                    const __grid_constant__ CUtensorMap map_ul, const __grid_constant__ CUtensorMap map_o,
                    const int32_t* __restrict__ cu, int32_t n_seq, int64_t T, int32_t Hk, int32_t Hv,
                    const uint8_t* __restrict__ ws_ro, int* err_word, const void* init, void* fin,
-                   int state_bf16, bf16* __restrict__ o, float scale, BlockStates blocks) {
+                   int state_flags, bf16* __restrict__ o, float scale, BlockStates blocks,
+                   int32_t c_begin, int32_t c_end) {
   const Ws L = ws_layout(T, n_seq, Hv);
   const int32_t* prefix = reinterpret_cast<const int32_t*>(ws_ro + L.prefix);
   const int tile = blockIdx.x % NT;
@@ -772,11 +800,19 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
   const int32_t n = blockIdx.x / (NT * Hv);
   const int hk = h / (Hv / Hk);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const bool sbf = state_bf16 != 0;
+  // storage of the initial, final and block states: fp32, or bf16 (kStateInitBf16 ...)
+  const bool init_bf = (state_flags & kStateInitBf16) != 0, fin_bf = (state_flags & kStateFinBf16) != 0;
+  const bool sbf = (state_flags & kStateBlocksBf16) != 0;
   int64_t bos, eos;
   seq_bounds(cu, n, T, bos, eos);
-  const int nc = (int)((eos - bos + C - 1) / C);
-  const int32_t slot0 = prefix[n];
+  // this launch's chunks of the sequence: [c_begin, c_end) clamped to its length; bos and the
+  // first slot move to the first of them, cfirst keeps its index for the block states
+  const int nc_all = (int)((eos - bos + C - 1) / C);
+  const int cfirst = c_begin < nc_all ? c_begin : nc_all;
+  const int clast = c_end < nc_all ? c_end : nc_all;
+  const int nc = clast > cfirst ? clast - cfirst : 0;
+  bos += (int64_t)cfirst * C;
+  const int32_t slot0 = prefix[n] + cfirst;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -988,7 +1024,7 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     float s[SJ];
     const int64_t sbase = ((int64_t)n * Hv + h) * D * D + (int64_t)(tile * DT + half * SJ) * D + lrow;
 #pragma unroll
-    for (int j = 0; j < SJ; ++j) s[j] = init ? state_load(init, sbase + (int64_t)j * D, sbf) : 0.f;
+    for (int j = 0; j < SJ; ++j) s[j] = init ? state_load(init, sbase + (int64_t)j * D, init_bf) : 0.f;
     auto store_state_bf16 = [&]() {
 #pragma unroll
       for (int c8 = 0; c8 < SJ / 8; ++c8) {
@@ -1071,8 +1107,8 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
       tc_fence_before();
       warp_arrive(bar_Sq);
       // the state after a full chunk that ends a block of the sequence (prefix caching)
-      if (blocks.block_tokens > 0 && len == C && ((int64_t)(c + 1) * C) % blocks.block_tokens == 0) {
-        const int64_t brow = (int64_t)blocks.rows[n] + (int64_t)(c + 1) * C / blocks.block_tokens - 1;
+      if (blocks.block_tokens > 0 && len == C && ((int64_t)(cfirst + c + 1) * C) % blocks.block_tokens == 0) {
+        const int64_t brow = (int64_t)blocks.rows[n] + (int64_t)(cfirst + c + 1) * C / blocks.block_tokens - 1;
         if (brow >= 0 && brow < blocks.n_rows) {
           const int64_t dst = ((brow * Hv + h) * D + tile * DT + half * SJ) * (int64_t)D + lrow;
 #pragma unroll
@@ -1131,7 +1167,7 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     if (warp == 2 && lane == 0) tma_store_wait_all();
     if (ok && fin != nullptr) {
 #pragma unroll
-      for (int j = 0; j < SJ; ++j) state_store(fin, sbase + (int64_t)j * D, s[j], sbf);
+      for (int j = 0; j < SJ; ++j) state_store(fin, sbase + (int64_t)j * D, s[j], fin_bf);
     }
   }
 
@@ -1189,6 +1225,34 @@ size_t prefill_chunk_tc_workspace(int64_t T, int32_t n_seq, int32_t Hv) {
   return ws_layout(T, n_seq, Hv).total;
 }
 
+// Per device: the two streams a prefill in pieces forks onto (intra-chunk work at the lowest
+// priority, chains at the highest) and the events that order them, created on first use and
+// kept for the life of the process. Calls on one device take the mutex while they enqueue.
+struct PieceStreams {
+  std::mutex mu;
+  cudaStream_t side = nullptr, chain = nullptr;
+  cudaEvent_t ev[kMaxPieces + 2] = {};
+};
+
+PieceStreams* piece_streams(int dev) {
+  static PieceStreams slots[64];
+  static std::mutex init_mu;
+  if (dev < 0 || dev >= 64) return nullptr;
+  PieceStreams* p = &slots[dev];
+  std::lock_guard<std::mutex> lock(init_mu);
+  if (p->side != nullptr) return p;
+  int lo = 0, hi = 0;   // numerically lowest = highest priority
+  if (cudaDeviceGetStreamPriorityRange(&lo, &hi) != cudaSuccess) return nullptr;
+  cudaStream_t side = nullptr, chain = nullptr;
+  if (cudaStreamCreateWithPriority(&side, cudaStreamNonBlocking, lo) != cudaSuccess) return nullptr;
+  if (cudaStreamCreateWithPriority(&chain, cudaStreamNonBlocking, hi) != cudaSuccess) return nullptr;
+  for (int i = 0; i < kMaxPieces + 2; ++i)
+    if (cudaEventCreateWithFlags(&p->ev[i], cudaEventDisableTiming) != cudaSuccess) return nullptr;
+  p->chain = chain;
+  p->side = side;
+  return p;
+}
+
 cudaError_t launch_prefill_chunk_tc(const void* q, const void* k, const void* v, const float* g,
                                     const float* beta, void* o, int64_t T, int32_t Hk, int32_t Hv,
                                     int64_t qk_stride, int64_t v_stride, const int32_t* cu,
@@ -1228,17 +1292,65 @@ cudaError_t launch_prefill_chunk_tc(const void* q, const void* k, const void* v,
                 !make_map(&mo, o, (uint64_t)Hv * D, (uint64_t)T, (uint64_t)Hv * D)))
     return cudaErrorInvalidValue;
   chunk_plan_kernel<<<1, 1024, 0, stream>>>(cu, n_seq, T, reinterpret_cast<int32_t*>(ws + L.prefix),
-                                            reinterpret_cast<int*>(ws + L.err));
-  if (T > 0) {   // persistent: two CTAs per SM (shared memory and tensor memory allow two)
-    const int64_t items = slots * Hk;
-    const int64_t grid = items < 2 * (int64_t)num_sms ? items : 2 * (int64_t)num_sms;
-    chunk_intra_kernel<<<(unsigned)grid, 128, kIntraSmem, stream>>>(mq, mk, mv, mwu, mmq, mul, g, beta,
-                                                                    cu, n_seq, T, Hk, Hv, ws);
-  }
+                                            reinterpret_cast<int*>(ws + L.err),
+                                            reinterpret_cast<int*>(ws + L.ctr));
+  const int user_bf = state_dtype == kBF16 ? 1 : 0;
+  const int flags = user_bf * (kStateInitBf16 | kStateFinBf16 | kStateBlocksBf16);
+  const int64_t n_chunks = (T + C - 1) / C;
+  // persistent intra-chunk grid: two CTAs per SM (shared and tensor memory allow two)
+  auto intra_grid = [&](int64_t n_slots) {
+    const int64_t items = n_slots * Hk;
+    return (unsigned)(items < 2 * (int64_t)num_sms ? items : 2 * (int64_t)num_sms);
+  };
   dim3 gc((unsigned)((int64_t)n_seq * Hv * NT));
-  chunk_chain_kernel<<<gc, kChainThreads, kChainSmem, stream>>>(
-      mq, mk, mwu, mmq, mul, mo, cu, n_seq, T, Hk, Hv, ws, reinterpret_cast<int*>(ws + L.err), init, fin,
-      state_dtype == kBF16 ? 1 : 0, static_cast<bf16*>(o), scale, blocks);
+  if (!piece_layout(T, n_seq) || (int64_t)Hv * NT > num_sms - 16) {
+    // one pass: every chunk's intra-chunk work, then the chains
+    if (T > 0)
+      chunk_intra_kernel<<<intra_grid(slots), 128, kIntraSmem, stream>>>(
+          mq, mk, mv, mwu, mmq, mul, g, beta, cu, n_seq, T, Hk, Hv, ws, 0, (int32_t)slots, 0);
+    chunk_chain_kernel<<<gc, kChainThreads, kChainSmem, stream>>>(
+        mq, mk, mwu, mmq, mul, mo, cu, n_seq, T, Hk, Hv, ws, reinterpret_cast<int*>(ws + L.err), init, fin,
+        flags, static_cast<bf16*>(o), scale, blocks, 0, INT32_MAX);
+    return cudaGetLastError();
+  }
+  // One long sequence in pieces of kPieceChunks chunks. The intra-chunk kernel of every piece
+  // runs in order on a low-priority side stream; the chain kernel of piece i runs on a
+  // high-priority stream once piece i's intra-chunk work is done, beside the intra-chunk work
+  // of the pieces after it (the chain occupies 2 Hv SMs; when a chain piece ends, its SMs go
+  // to the next chain piece first). The state goes from one chain piece to the next through
+  // the workspace in fp32. Only events order the streams: no kernel waits for another.
+  const int pieces = (int)((n_chunks + kPieceChunks - 1) / kPieceChunks < kMaxPieces
+                               ? (n_chunks + kPieceChunks - 1) / kPieceChunks : kMaxPieces);
+  const int64_t per = (n_chunks + pieces - 1) / pieces;
+  PieceStreams* ps = piece_streams(dev);
+  if (ps == nullptr) return cudaErrorInitializationError;
+  std::lock_guard<std::mutex> lock(ps->mu);   // the events are reused by every call on this device
+  void* carry = ws + L.carry;
+  cudaEvent_t* ev = ps->ev;
+  if ((e = cudaEventRecord(ev[0], stream)) != cudaSuccess) return e;   // the plan is done
+  if ((e = cudaStreamWaitEvent(ps->side, ev[0], 0)) != cudaSuccess) return e;
+  if ((e = cudaStreamWaitEvent(ps->chain, ev[0], 0)) != cudaSuccess) return e;
+  for (int i = 0; i < pieces; ++i) {
+    const int64_t c0 = i * per, c1 = (i + 1) * per < n_chunks ? (i + 1) * per : n_chunks;
+    // slot s of a single sequence is its chunk s; the last piece also takes the padding slot
+    chunk_intra_kernel<<<intra_grid(c1 - c0), 128, kIntraSmem, ps->side>>>(
+        mq, mk, mv, mwu, mmq, mul, g, beta, cu, n_seq, T, Hk, Hv, ws, (int32_t)c0,
+        (int32_t)(i == pieces - 1 ? slots : c1), i);
+    if ((e = cudaEventRecord(ev[1 + i], ps->side)) != cudaSuccess) return e;
+  }
+  for (int i = 0; i < pieces; ++i) {
+    const int64_t c0 = i * per, c1 = (i + 1) * per < n_chunks ? (i + 1) * per : n_chunks;
+    if ((e = cudaStreamWaitEvent(ps->chain, ev[1 + i], 0)) != cudaSuccess) return e;
+    const bool first = i == 0, last = i == pieces - 1;
+    const int f = (first ? user_bf * kStateInitBf16 : 0) | (last ? user_bf * kStateFinBf16 : 0) |
+                  user_bf * kStateBlocksBf16;
+    chunk_chain_kernel<<<gc, kChainThreads, kChainSmem, ps->chain>>>(
+        mq, mk, mwu, mmq, mul, mo, cu, n_seq, T, Hk, Hv, ws, reinterpret_cast<int*>(ws + L.err),
+        first ? init : carry, last ? fin : carry, f, static_cast<bf16*>(o), scale, blocks,
+        (int32_t)c0, (int32_t)(last ? INT32_MAX : c1));
+  }
+  if ((e = cudaEventRecord(ev[kMaxPieces + 1], ps->chain)) != cudaSuccess) return e;
+  if ((e = cudaStreamWaitEvent(stream, ev[kMaxPieces + 1], 0)) != cudaSuccess) return e;   // join
   return cudaGetLastError();
 }
 

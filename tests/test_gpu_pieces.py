@@ -1,0 +1,90 @@
+"""A long single sequence is prefilled in pieces: the intra-chunk work of the later pieces
+runs beside the chain of the current one, and the state passes from one chain piece to the
+next in fp32. Parity against the oracle across the piece boundaries (output, final state and
+block states, fp32 and bf16 state storage), and bit-equality with the same sequence split by
+the caller at the same chunk boundaries."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import gated_deltanet_mixer_causal_b200 as gdn
+from gated_deltanet_mixer_causal_b200 import workloads as W
+import oracle
+from parity import BF16_TOL, check, np64, worst_head_o, worst_head_state
+
+pytestmark = pytest.mark.gpu
+
+SHAPE = W.LayerShape(2, 6, 128, 128)   # 12 chain CTAs: the pieces path
+T = 17000                              # 266 chunks: three pieces, the last one ragged
+BLOCK = 2048
+PIECE_CHUNKS = 128                     # the library's piece size (balanced over the pieces)
+
+
+def _piece_bounds(n_tok):
+    n_chunks = math.ceil(n_tok / 64)
+    pieces = math.ceil(n_chunks / PIECE_CHUNKS)
+    per = math.ceil(n_chunks / pieces)
+    return [min(i * per * 64, n_tok) for i in range(pieces)] + [n_tok]
+
+
+def _inputs(seed):
+    return W.make_recurrence(SHAPE, T, seed=seed, dtype=torch.bfloat16, init_std=0.02)
+
+
+@pytest.mark.parametrize("state_dtype", [torch.float32, torch.bfloat16])
+def test_pieces_against_oracle(cuda_device, state_dtype):
+    dev = cuda_device
+    r = _inputs(91)
+    sh = r.shape
+    s0 = r.initial_state.numpy()
+    if state_dtype == torch.bfloat16:
+        s0 = oracle.round_bf16(s0)
+    n_blocks = T // BLOCK
+    fin = torch.empty((1, sh.Hv, sh.dv, sh.dk), dtype=state_dtype, device=dev)
+    bs = torch.full((n_blocks + 1, sh.Hv, sh.dv, sh.dk), float("nan"), dtype=state_dtype, device=dev)
+    o = gdn.gdn_chunk_prefill(r.q.to(dev), r.k.to(dev), r.v.to(dev), r.g.to(dev), r.beta.to(dev),
+                              None, torch.from_numpy(s0).to(state_dtype).to(dev), fin,
+                              block_tokens=BLOCK, block_states=bs,
+                              block_rows=torch.zeros(1, dtype=torch.int32, device=dev), check=True)
+    torch.cuda.synchronize()
+    q, k, v = (t.float().numpy() for t in (r.q, r.k, r.v))
+    g, beta = r.g.numpy(), r.beta.numpy()
+    o_r, f_r = oracle.recurrence(q, k, v, g, beta, None, s0)
+    rnd = oracle.round_bf16 if state_dtype == torch.bfloat16 else (lambda x: x)
+    case = f"test_pieces_against_oracle[{str(state_dtype).split('.')[-1]}]"
+    check(case, "o per head", worst_head_o(np64(o), o_r, None), BF16_TOL)
+    check(case, "state per head", worst_head_state(np64(fin), rnd(f_r)), BF16_TOL)
+    # block states: the oracle chained block by block from the same initial state
+    got, s, worst = np64(bs), s0, 0.0
+    for m in range(n_blocks):
+        a, b = m * BLOCK, (m + 1) * BLOCK
+        _, s = oracle.recurrence(q[a:b], k[a:b], v[a:b], g[a:b], beta[a:b], None, s)
+        worst = max(worst, worst_head_state(got[m:m + 1], rnd(s)))
+    check(case, "block states", worst, BF16_TOL)
+    assert np.isnan(got[n_blocks]).all()
+
+
+def test_pieces_equal_the_caller_split(cuda_device):
+    """The pieces path computes exactly what consecutive calls over the same chunk ranges
+    compute, each from the previous one's fp32 final state."""
+    dev = cuda_device
+    r = _inputs(92)
+    sh = r.shape
+    q, k, v, g, beta = (t.to(dev) for t in (r.q, r.k, r.v, r.g, r.beta))
+    s0 = r.initial_state.to(dev)
+    fin = torch.empty((1, sh.Hv, sh.dv, sh.dk), dtype=torch.float32, device=dev)
+    o = gdn.gdn_chunk_prefill(q, k, v, g, beta, None, s0, fin, check=True)
+    bounds = _piece_bounds(T)
+    assert len(bounds) == 4                      # three pieces
+    parts, state = [], s0
+    for a, b in zip(bounds[:-1], bounds[1:]):
+        assert b - a < 2 * PIECE_CHUNKS * 64     # each part alone takes the one-pass path
+        nxt = torch.empty_like(fin)
+        parts.append(gdn.gdn_chunk_prefill(q[a:b], k[a:b], v[a:b], g[a:b], beta[a:b], None, state,
+                                           nxt, check=True))
+        state = nxt
+    torch.cuda.synchronize()
+    assert torch.equal(o, torch.cat(parts, 0))
+    assert torch.equal(fin, state)
