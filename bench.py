@@ -533,19 +533,20 @@ def gdn_prefill_launches() -> int:
 # of each kernel on the small case (T = 8192, decode batch 64), per unit processed (token
 # for the prefill kernels and the conv, sequence for the decode step), scaled to the
 # benchmark's launch; None when the kernel changed since the capture. The prefill figure is
-# the intra-chunk kernel's 467.18 MB plus the chain kernel's 511.14 MB.
-TRAFFIC_PER_UNIT = {"prefill": (467.18e6 + 511.14e6) / 8192, "conv": 291.25e6 / 8192,
+# the intra-chunk kernel's 469.72 MB plus the chain kernel's 512.83 MB.
+TRAFFIC_PER_UNIT = {"prefill": (469.72e6 + 512.83e6) / 8192, "conv": 291.25e6 / 8192,
                     "decode": 357.64e6 / 64}
 
 # The chunked prefill's two kernels: their share of its FLOPs (from the chunked form: the
 # intra-chunk kernel forms K K^T and Q K^T per key head, solves the triangular system and
-# builds U~ = P V, W = Pk K and Mqk; the chain applies [-W; Q] S0^T, K^T U' and Mqk U), their
-# share of its time (the ncu launch list of the 65536-token run: 1434.4 and 1977.6 us of
-# 3414.7 us, the plan kernel the rest) and their DRAM traffic per token from the same
-# captures as above.
+# builds U~ = P V, W = Pk K and Mqk; the chain applies [-W; Q] S0^T, K^T U' and Mqk U), the
+# device time of their launches in one 65536-token call from the ncu launch list (serialised
+# by ncu: eight pieces of each, 1523.1 us of intra-chunk and 2145.3 us of chain launches; in
+# the call the pieces of the two kernels overlap, so the call takes less than their sum), and
+# their DRAM traffic per token from the same captures as above.
 PREFILL_KERNELS = {
-    "chunk_intra": {"time_share": 1434.4 / 3414.7, "traffic_per_token": 467.18e6 / 8192},
-    "chunk_chain": {"time_share": 1977.6 / 3414.7, "traffic_per_token": 511.14e6 / 8192},
+    "chunk_intra": {"busy_us_64k": 1523.1, "traffic_per_token": 469.72e6 / 8192},
+    "chunk_chain": {"busy_us_64k": 2145.3, "traffic_per_token": 512.83e6 / 8192},
 }
 
 
@@ -557,16 +558,21 @@ def prefill_kernel_flops_per_token(kernel: str, sh=SHAPE, C=64):
 
 
 def prefill_kernel_split(T: int, prefill_ms: float, peak_tflops: float) -> dict:
-    """Per-kernel FLOPs and traffic of one prefill launch, with each kernel's time taken as
-    its launch-list share of the measured call time."""
+    """Per-kernel FLOPs and traffic of one prefill launch, each kernel's rate over its own
+    device time (the launch list's, scaled by tokens), and how much of the call the two
+    kernels' times overlap."""
     out = {}
+    busy = 0.0
     for k, v in PREFILL_KERNELS.items():
         flops = prefill_kernel_flops_per_token(k) * T
-        ms = prefill_ms * v["time_share"]
-        out[k] = {"flops": flops, "time_share": v["time_share"], "ms": ms,
-                  "tflops": flops / (ms / 1e3) / 1e12,
+        ms = v["busy_us_64k"] / 1e3 * T / 65536
+        busy += ms
+        out[k] = {"flops": flops, "device_ms": ms, "tflops": flops / (ms / 1e3) / 1e12,
                   "frac": flops / (ms / 1e3) / 1e12 / peak_tflops,
                   "traffic": v["traffic_per_token"] * T}
+    out["overlap"] = {"device_ms_sum": busy, "call_ms": prefill_ms,
+                      "note": "intra-chunk pieces run beside chain pieces: the call is shorter "
+                              "than the sum of its kernels' device times"}
     return out
 
 
