@@ -71,14 +71,22 @@ constexpr int kVecBytes = kVecFloats * 4;
 
 __host__ __device__ inline int64_t max_slots(int64_t T, int32_t n_seq) { return (T + C - 1) / C + n_seq; }
 
-// A long single sequence is prefilled in pieces of kPieceChunks chunks (at most kMaxPieces):
-// the intra-chunk kernel of the next pieces runs beside the chain kernel of the current one,
-// which occupies only 2 Hv of the SMs. The workspace then also holds the fp32 state handed
-// from one chain piece to the next.
-constexpr int64_t kPieceChunks = 128;
+// A long single sequence is prefilled in pieces: the intra-chunk kernel of the next pieces
+// runs beside the chain kernel of the current one, which occupies only 2 Hv of the SMs.
+// kTargetPieces pieces of at least kMinPieceChunks chunks: a chain piece costs ~15 us to
+// start, so shorter pieces lose more than the overlap gains (measured on the 27B layer: 8
+// pieces take the 65536-token prefill from 3.38 to 3.07 ms and the 32768-token one from 1.72
+// to 1.66 ms, while 16384 tokens gain nothing and 8192 tokens lose 14 %). The workspace then
+// also holds the fp32 state handed from one chain piece to the next.
+constexpr int64_t kMinPieceChunks = 64;
+constexpr int64_t kTargetPieces = 8;
 constexpr int kMaxPieces = 64;
+__host__ __device__ inline int64_t piece_chunks(int64_t n_chunks) {
+  const int64_t per = (n_chunks + kTargetPieces - 1) / kTargetPieces;
+  return per > kMinPieceChunks ? per : kMinPieceChunks;
+}
 __host__ __device__ inline bool piece_layout(int64_t T, int32_t n_seq) {
-  return n_seq == 1 && T >= 2 * kPieceChunks * C;
+  return n_seq == 1 && T >= kTargetPieces * kMinPieceChunks * C;
 }
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -1313,15 +1321,14 @@ cudaError_t launch_prefill_chunk_tc(const void* q, const void* k, const void* v,
         flags, static_cast<bf16*>(o), scale, blocks, 0, INT32_MAX);
     return cudaGetLastError();
   }
-  // One long sequence in pieces of kPieceChunks chunks. The intra-chunk kernel of every piece
+  // One long sequence in pieces of piece_chunks() chunks. The intra-chunk kernel of every piece
   // runs in order on a low-priority side stream; the chain kernel of piece i runs on a
   // high-priority stream once piece i's intra-chunk work is done, beside the intra-chunk work
   // of the pieces after it (the chain occupies 2 Hv SMs; when a chain piece ends, its SMs go
   // to the next chain piece first). The state goes from one chain piece to the next through
   // the workspace in fp32. Only events order the streams: no kernel waits for another.
-  const int pieces = (int)((n_chunks + kPieceChunks - 1) / kPieceChunks < kMaxPieces
-                               ? (n_chunks + kPieceChunks - 1) / kPieceChunks : kMaxPieces);
-  const int64_t per = (n_chunks + pieces - 1) / pieces;
+  const int64_t per = piece_chunks(n_chunks);
+  const int pieces = (int)((n_chunks + per - 1) / per);   // at most kTargetPieces + 1 <= kMaxPieces
   PieceStreams* ps = piece_streams(dev);
   if (ps == nullptr) return cudaErrorInitializationError;
   std::lock_guard<std::mutex> lock(ps->mu);   // the events are reused by every call on this device

@@ -17,15 +17,15 @@ from parity import BF16_TOL, check, np64, worst_head_o, worst_head_state
 pytestmark = pytest.mark.gpu
 
 SHAPE = W.LayerShape(2, 6, 128, 128)   # 12 chain CTAs: the pieces path
-T = 17000                              # 266 chunks: three pieces, the last one ragged
-BLOCK = 2048
-PIECE_CHUNKS = 128                     # the library's piece size (balanced over the pieces)
+T = 33000                              # 516 chunks: eight pieces, the last one ragged
+BLOCK = 4096
 
 
 def _piece_bounds(n_tok):
+    """The library's split: eight pieces of at least 64 chunks each."""
     n_chunks = math.ceil(n_tok / 64)
-    pieces = math.ceil(n_chunks / PIECE_CHUNKS)
-    per = math.ceil(n_chunks / pieces)
+    per = max(64, math.ceil(n_chunks / 8))
+    pieces = math.ceil(n_chunks / per)
     return [min(i * per * 64, n_tok) for i in range(pieces)] + [n_tok]
 
 
@@ -77,10 +77,10 @@ def test_pieces_equal_the_caller_split(cuda_device):
     fin = torch.empty((1, sh.Hv, sh.dv, sh.dk), dtype=torch.float32, device=dev)
     o = gdn.gdn_chunk_prefill(q, k, v, g, beta, None, s0, fin, check=True)
     bounds = _piece_bounds(T)
-    assert len(bounds) == 4                      # three pieces
+    assert len(bounds) == 9                      # eight pieces
     parts, state = [], s0
     for a, b in zip(bounds[:-1], bounds[1:]):
-        assert b - a < 2 * PIECE_CHUNKS * 64     # each part alone takes the one-pass path
+        assert b - a < 8 * 64 * 64               # each part alone takes the one-pass path
         nxt = torch.empty_like(fin)
         parts.append(gdn.gdn_chunk_prefill(q[a:b], k[a:b], v[a:b], g[a:b], beta[a:b], None, state,
                                            nxt, check=True))
