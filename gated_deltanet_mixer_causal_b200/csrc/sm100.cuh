@@ -70,27 +70,18 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded spin for a single thread on a latency-critical path: it polls, sleeping ~32 ns
-// between polls, so it resumes within about a hundred cycles of the phase completing while
-// leaving the issue slots to the warps it waits for. kSpinPolls polls bound the wait at
+// Bounded spin for the threads that issue on a latency-critical path: they poll, sleeping
+// ~32 ns between polls, so they resume soon after the phase completes while leaving the issue
+// slots to the warps they wait for. kSpinPolls polls bound the wait at
 // about a second.
-#ifndef GDN_SPIN_MODE
-#define GDN_SPIN_MODE 1
-#endif
 constexpr uint32_t kSpinPolls = 1u << 24;
 __device__ __forceinline__ bool mbar_spin(uint64_t* bar, uint32_t parity, int* err, int code) {
-#if GDN_SPIN_MODE == 2
-  return mbar_wait(bar, parity, err, code);
-#else
   for (uint32_t i = 0; i < kSpinPolls; ++i) {
     if (mbar_test(bar, parity)) return true;
-#if GDN_SPIN_MODE == 1
     __nanosleep(32);   // yield the issue slot to the warps that produce what is awaited
-#endif
   }
   if (err) atomicCAS(err, 0, code);
   return false;
-#endif
 }
 
 // ------------------------------------------------------------------------------ TMA
