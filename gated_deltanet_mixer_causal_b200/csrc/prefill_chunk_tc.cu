@@ -1233,12 +1233,14 @@ size_t prefill_chunk_tc_workspace(int64_t T, int32_t n_seq, int32_t Hv) {
   return ws_layout(T, n_seq, Hv).total;
 }
 
-// Per device: the two streams a prefill in pieces forks onto (intra-chunk work at the lowest
-// priority, chains at the highest) and the events that order them, created on first use and
-// kept for the life of the process. Calls on one device take the mutex while they enqueue.
+// Per device: the streams a prefill in pieces forks onto (two for the intra-chunk pieces, taken
+// in turn so that one piece's last items overlap the next piece's first, at the lowest
+// priority; one for the chains at the highest) and the events that order them, created on
+// first use and kept for the life of the process. Calls on one device take the mutex while
+// they enqueue.
 struct PieceStreams {
   std::mutex mu;
-  cudaStream_t side = nullptr, chain = nullptr;
+  cudaStream_t side[2] = {nullptr, nullptr}, chain = nullptr;
   cudaEvent_t ev[kMaxPieces + 2] = {};
 };
 
@@ -1248,16 +1250,18 @@ PieceStreams* piece_streams(int dev) {
   if (dev < 0 || dev >= 64) return nullptr;
   PieceStreams* p = &slots[dev];
   std::lock_guard<std::mutex> lock(init_mu);
-  if (p->side != nullptr) return p;
+  if (p->chain != nullptr) return p;
   int lo = 0, hi = 0;   // numerically lowest = highest priority
   if (cudaDeviceGetStreamPriorityRange(&lo, &hi) != cudaSuccess) return nullptr;
-  cudaStream_t side = nullptr, chain = nullptr;
-  if (cudaStreamCreateWithPriority(&side, cudaStreamNonBlocking, lo) != cudaSuccess) return nullptr;
-  if (cudaStreamCreateWithPriority(&chain, cudaStreamNonBlocking, hi) != cudaSuccess) return nullptr;
+  for (int i = 0; i < 2; ++i)
+    if (p->side[i] == nullptr && cudaStreamCreateWithPriority(&p->side[i], cudaStreamNonBlocking, lo) != cudaSuccess)
+      return nullptr;
   for (int i = 0; i < kMaxPieces + 2; ++i)
-    if (cudaEventCreateWithFlags(&p->ev[i], cudaEventDisableTiming) != cudaSuccess) return nullptr;
-  p->chain = chain;
-  p->side = side;
+    if (p->ev[i] == nullptr && cudaEventCreateWithFlags(&p->ev[i], cudaEventDisableTiming) != cudaSuccess)
+      return nullptr;
+  cudaStream_t chain = nullptr;
+  if (cudaStreamCreateWithPriority(&chain, cudaStreamNonBlocking, hi) != cudaSuccess) return nullptr;
+  p->chain = chain;   // set last: a non-null chain stream means the set is complete
   return p;
 }
 
@@ -1321,8 +1325,8 @@ cudaError_t launch_prefill_chunk_tc(const void* q, const void* k, const void* v,
         flags, static_cast<bf16*>(o), scale, blocks, 0, INT32_MAX);
     return cudaGetLastError();
   }
-  // One long sequence in pieces of piece_chunks() chunks. The intra-chunk kernel of every piece
-  // runs in order on a low-priority side stream; the chain kernel of piece i runs on a
+  // One long sequence in pieces of piece_chunks() chunks. The intra-chunk kernels of the pieces
+  // run on two low-priority side streams in turn; the chain kernel of piece i runs on a
   // high-priority stream once piece i's intra-chunk work is done, beside the intra-chunk work
   // of the pieces after it (the chain occupies 2 Hv SMs; when a chain piece ends, its SMs go
   // to the next chain piece first). The state goes from one chain piece to the next through
@@ -1335,15 +1339,17 @@ cudaError_t launch_prefill_chunk_tc(const void* q, const void* k, const void* v,
   void* carry = ws + L.carry;
   cudaEvent_t* ev = ps->ev;
   if ((e = cudaEventRecord(ev[0], stream)) != cudaSuccess) return e;   // the plan is done
-  if ((e = cudaStreamWaitEvent(ps->side, ev[0], 0)) != cudaSuccess) return e;
+  for (int sdx = 0; sdx < 2; ++sdx)
+    if ((e = cudaStreamWaitEvent(ps->side[sdx], ev[0], 0)) != cudaSuccess) return e;
   if ((e = cudaStreamWaitEvent(ps->chain, ev[0], 0)) != cudaSuccess) return e;
   for (int i = 0; i < pieces; ++i) {
     const int64_t c0 = i * per, c1 = (i + 1) * per < n_chunks ? (i + 1) * per : n_chunks;
     // slot s of a single sequence is its chunk s; the last piece also takes the padding slot
-    chunk_intra_kernel<<<intra_grid(c1 - c0), 128, kIntraSmem, ps->side>>>(
+    cudaStream_t side = ps->side[i & 1];
+    chunk_intra_kernel<<<intra_grid(c1 - c0), 128, kIntraSmem, side>>>(
         mq, mk, mv, mwu, mmq, mul, g, beta, cu, n_seq, T, Hk, Hv, ws, (int32_t)c0,
         (int32_t)(i == pieces - 1 ? slots : c1), i);
-    if ((e = cudaEventRecord(ev[1 + i], ps->side)) != cudaSuccess) return e;
+    if ((e = cudaEventRecord(ev[1 + i], side)) != cudaSuccess) return e;
   }
   for (int i = 0; i < pieces; ++i) {
     const int64_t c0 = i * per, c1 = (i + 1) * per < n_chunks ? (i + 1) * per : n_chunks;

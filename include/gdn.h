@@ -20,7 +20,7 @@
  * Pointers: device pointers unless stated; 16-byte aligned; tensors row-major and dense
  *   unless a stride argument says otherwise. The caller owns every buffer, including the
  *   workspace; the library allocates no device memory and keeps no state between calls,
- *   except gdn_chunk_prefill_noalloc's static scratch and, per device, two streams and a
+ *   except gdn_chunk_prefill_noalloc's static scratch and, per device, three streams and a
  *   set of events that a long single-sequence prefill forks onto and joins back from
  *   (created on first use, kept for the life of the process).
  * Streams: every call is asynchronous on `stream` (NULL = the legacy default stream) and
@@ -136,7 +136,7 @@ int32_t gdn_chunk_prefill_path(gdn_dtype_t dt, int32_t Hk, int32_t Hv, int32_t d
  * section 2 for the read-out o = S q. The kernels evaluate it chunk by chunk (the
  * WY/UT form of the same recurrence); results equal the token-by-token recurrence up to
  * rounding. On the tensor-core path a single sequence of 32768 tokens or more is run in
- * eight pieces: the call forks onto two library streams (the intra-chunk work of later
+ * eight pieces: the call forks onto library streams (the intra-chunk work of later
  * pieces beside the state pass of the current one) and joins back into `stream` with
  * events, so the call stays ordered with the rest of `stream`.
  *
