@@ -385,7 +385,7 @@ def main():
         ev[3].record(stream)
 
     # launches of this library's kernels per step: conv 1, prefill (per path), decode 1
-    launches_per_step = 1 + gdn_prefill_launches() + 1
+    launches_per_step = 1 + gdn_prefill_launches(T, 1, sh, torch.cuda.get_device_properties(dev).multi_processor_count) + 1
 
     for _ in range(args.warmup):
         step([torch.cuda.Event(enable_timing=True) for _ in range(4)])
@@ -523,9 +523,15 @@ def main():
         dist.destroy_process_group()
 
 
-def gdn_prefill_launches() -> int:
+def gdn_prefill_launches(T: int, n_seq: int = 1, sh=SHAPE, num_sms: int = 148) -> int:
     """Kernels one gdn_chunk_prefill call enqueues on the benchmark's path (bf16, d = 128):
-    the chunk plan, the intra-chunk kernel and the chain kernel."""
+    the chunk plan, then the intra-chunk and chain kernels once each, or once per piece when
+    a single sequence of 512 chunks or more is run in pieces (eight pieces of at least 64
+    chunks, while its 2 Hv chain CTAs leave at least 16 SMs free)."""
+    n_chunks = -(-T // 64)
+    if n_seq == 1 and n_chunks >= 8 * 64 and 2 * sh.Hv <= num_sms - 16:
+        per = max(64, -(-n_chunks // 8))
+        return 1 + 2 * (-(-n_chunks // per))
     return 3
 
 

@@ -119,3 +119,16 @@ def test_decode_tokens_bytes_reduce_to_one_step(bench):
     per_token = B * sh.conv_channels * 2 + B * sh.Hv * sh.dv * 2 + 2 * B * sh.Hv * 4
     for n in (2, 4, 8):
         assert bench.decode_tokens_bytes(B, n, sh) - one == (n - 1) * per_token
+
+
+def test_prefill_launch_count(bench):
+    """The plan kernel, then one intra-chunk and one chain launch per piece: eight pieces for
+    the 27B layer at 65,536 tokens, one pass below 32,768 tokens, for several sequences, or
+    when the chains would leave fewer than 16 SMs."""
+    sh = W.QWEN35_27B
+    assert bench.gdn_prefill_launches(65536, 1, sh) == 17
+    assert bench.gdn_prefill_launches(32768, 1, sh) == 17
+    assert bench.gdn_prefill_launches(33000, 1, sh) == 17     # 516 chunks in pieces of 65
+    assert bench.gdn_prefill_launches(16384, 1, sh) == 3
+    assert bench.gdn_prefill_launches(65536, 2, sh) == 3
+    assert bench.gdn_prefill_launches(65536, 1, W.LayerShape(16, 80, 128, 128)) == 3
