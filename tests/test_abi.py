@@ -194,6 +194,19 @@ def test_prefill_block_state_validation(L):
         _lib.GDN_ERR_INVALID_ARG
 
 
+def test_workspace_holds_the_piece_state_for_long_single_sequences(L):
+    """One sequence of 512 chunks or more (32,768 tokens) is prefilled in pieces, and the
+    workspace then also holds the fp32 state passed between them (Hv x d x d x 4 bytes); a
+    shorter sequence, or the same tokens as two sequences, has no such region."""
+    Hk, Hv, d = 16, 48, 128
+    size = lambda T, n: L.gdn_chunk_prefill_workspace_size(T, n, Hk, Hv, d, d, _lib.GDN_BF16)
+    per_slot = size(32767 - 64, 1) - size(32767 - 128, 1)     # one more chunk slot, no state
+    state = Hv * d * d * 4
+    assert size(32768, 1) - size(32767, 1) >= state
+    assert size(32768, 1) - size(32767, 1) < state + per_slot + 1024
+    assert size(32768, 2) - size(32767, 2) < per_slot + 1024    # two sequences: no piece state
+
+
 def test_prefill_beyond_32bit_coordinates_is_refused(L):
     """bf16 heads of 128: the tensor-core path's rows are int32 TMA coordinates, so a batch
     whose chunk rows pass 2^31 is unsupported (and says so before any launch); the same size
