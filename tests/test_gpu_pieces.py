@@ -66,16 +66,21 @@ def test_pieces_against_oracle(cuda_device, state_dtype):
     assert np.isnan(got[n_blocks]).all()
 
 
-def test_pieces_equal_the_caller_split(cuda_device):
+@pytest.mark.parametrize("form", ["initial_state", "zero_state_and_cu_seqlens"])
+def test_pieces_equal_the_caller_split(cuda_device, form):
     """The pieces path computes exactly what consecutive calls over the same chunk ranges
-    compute, each from the previous one's fp32 final state."""
+    compute, each from the previous one's fp32 final state: with an initial state, and
+    from zeros with the one sequence given through cu_seqlens."""
     dev = cuda_device
     r = _inputs(92)
     sh = r.shape
     q, k, v, g, beta = (t.to(dev) for t in (r.q, r.k, r.v, r.g, r.beta))
-    s0 = r.initial_state.to(dev)
     fin = torch.empty((1, sh.Hv, sh.dv, sh.dk), dtype=torch.float32, device=dev)
-    o = gdn.gdn_chunk_prefill(q, k, v, g, beta, None, s0, fin, check=True)
+    if form == "initial_state":
+        s0, cu = r.initial_state.to(dev), None
+    else:
+        s0, cu = None, torch.tensor([0, T], dtype=torch.int32, device=dev)
+    o = gdn.gdn_chunk_prefill(q, k, v, g, beta, cu, s0, fin, check=True)
     bounds = _piece_bounds(T)
     assert len(bounds) == 9                      # eight pieces
     parts, state = [], s0
