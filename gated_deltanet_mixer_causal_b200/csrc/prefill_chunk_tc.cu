@@ -11,20 +11,24 @@
 //
 // Three kernels:
 //  1. plan  : chunk offsets of every packed sequence (chunks never straddle sequences).
-//  2. intra : one CTA per (chunk, key head), everything that does not depend on the state:
-//             [K; Q] K^T on tcgen05 (M = 128); per value head the decay-masked A and
-//             Mqk = M o QK^T / (|q||k|), the unit lower triangular inverse Tm (fp32), then
-//             [P; Pk] V and [P; Pk] K on tcgen05 with P = Tm diag(beta),
-//             Pk = Tm diag(beta e^G / |k|), giving U~ = P V and W = Pk K. Writes -W, U~,
-//             Mqk (bf16) and the row scales to the workspace.
+//  2. intra : persistent CTAs over the (chunk, key head) items, everything that does not
+//             depend on the state: [K; Q] K^T on tcgen05 (M = 128); per value head the
+//             decay-masked A and Mqk = M o QK^T / (|q||k|), the unit lower triangular
+//             inverse Tm (16-row blocks: fp32 substitution on the diagonal, tf32 warp MMAs
+//             off it), then [P; Pk] V and [P; Pk] K on tcgen05 with P = Tm diag(beta),
+//             Pk = Tm diag(beta e^G / |k|), giving U~ = P V and W = Pk K. Writes -W, U~ and
+//             its low bf16 half, Mqk (bf16) and the row scales to the workspace.
 //  3. chain : one CTA per (sequence, value head, 64-wide slice of dv) walks the chunks in
 //             order with the fp32 state slice in registers and its bf16 copy in shared
 //             memory; per chunk only the state-dependent GEMMs remain:
 //               [-W; Q] S0^T  (U = U~ - W S0^T in rows 0..63, Q S0^T in rows 64..127)
-//               dS^T = K^T U',   O2 = Mqk U
-//             The two GEMMs on the serial path are split along K over two issuing threads
-//             (tcgen05.mma costs a fixed issue time per instruction, so two issuers halve
-//             the path); a third thread issues O2 and the TMA loads.
+//               dS^T = K^T [U' | U'lo],   O2 = Mqk U
+//             rA is split along K over two issuing warps, dS^T and O2 come from the second;
+//             a producer warp issues the TMA loads and seeds A with U~.
+// A single sequence of 512 chunks or more runs as eight pieces (ranges of chunks): the intra
+// kernel of every piece on two low-priority side streams in turn, the chain of piece i on a
+// high-priority stream once piece i's intra work is done, beside the intra work of the later
+// pieces; events alone order the streams and the state passes between chain pieces in fp32.
 // Operands are staged in shared memory in the 128-byte-swizzled layouts TMA writes; K-major
 // and MN-major descriptors read the same tiles, and stacking two 64-row tiles 8 KB apart
 // makes one M = 128 operand. Every wait is bounded.
