@@ -416,6 +416,9 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
 
   for (int j = 0; j < G; ++j) {
     const int h = hk * G + j;
+    // the next item's g, beta into registers while the last head runs (stored to shared
+    // memory once this item is done with its own)
+    if (j == G - 1 && has_next) fetch_gb(nxt);
     const float* sG = gAll + j * 64;   // cumulative log-decay of this head
     const float* sb = bAll + j * 64;
     if (tid < 64) {   // column factors of P = Tm diag(beta), Pk = Tm diag(beta e^G / |k|), A, Mqk
@@ -664,9 +667,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     tc_fence_after();
     if (j == G - 1 && has_next) {
       // every MMA of this item has read K, Q and the V tiles: fetch the next item's inputs
-      // (its g, beta into registers, stored to shared memory once this head is done)
       if (tid == 0) load_kqv(nxt);
-      fetch_gb(nxt);
     }
     uint8_t* stage_w = sm + kIPP;  // -W (rows 64..127 of the result) staged in [P | Pk], which
                                    // the MMA that produced it has finished reading

@@ -340,7 +340,8 @@ def test_decode_matches_prefill_on_gpu(cuda_device):
 
 # ------------------------------------------------------------ multi-token decode
 
-@pytest.mark.parametrize("n_tok", [1, 2, 3, 5, 8])
+# the token count is a template parameter of the kernel: every count is its own code path
+@pytest.mark.parametrize("n_tok", [1, 2, 3, 4, 5, 6, 7, 8])
 def test_decode_tokens_fp32_small(cuda_device, n_tok):
     """n_tok tokens per sequence in one call against the oracle (fp32, element by element);
     n_tok < 3 keeps old taps in the new conv state, n_tok >= 3 replaces them all."""
@@ -361,7 +362,7 @@ def test_decode_tokens_fp32_small(cuda_device, n_tok):
     np.testing.assert_array_equal(np64(cs), cs_r)
 
 
-@pytest.mark.parametrize("n_tok", [4, 8])
+@pytest.mark.parametrize("n_tok", [1, 2, 3, 4, 5, 6, 7, 8])
 def test_decode_tokens_27b_bf16(cuda_device, n_tok):
     """27B-shaped heads, 16 sequences, n_tok tokens each in one call, every head against the
     oracle (bf16 tolerance); the conv taps are copies and must match exactly."""
