@@ -380,6 +380,18 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
   if (__syncthreads_or(!ok)) { ok = false; goto teardown; }
   has_next = item_at(*next_item, nxt);   // thread 0 wrote it before the barrier above
 
+  // [K; Q] K^T -> rows 0..63: K K^T, rows 64..127: Q K^T  (M = 128, N = 64, K = 128), issued
+  // first so that it runs while the threads take the norms of the same tiles
+  if (tid == 0) {
+    tc_fence_after();
+    const uint64_t kq = smem_desc(smem_u32(sm + kIKQ), 16u, 1024u);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const uint64_t off = (uint64_t)((kk >> 2) * (16384 >> 4) + (kk & 3) * 2);
+      mma_bf16(tmem + kTKQ, kq + off, kq + off, idesc_bf16(128, 64, 0, 0), kk > 0);
+    }
+    mma_commit(bar_mma);
+  }
   {  // inverse L2 norms of the chunk's q and k rows (0 for rows past the sequence end)
     const int r = tid & 63;
     const uint8_t* tile = sm + kIKQ + (tid < 64 ? 8192 : 0);
@@ -398,16 +410,6 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     (tid < 64 ? rq : rk)[r] = inv;
   }
 
-  if (tid == 0) {   // [K; Q] K^T -> rows 0..63: K K^T, rows 64..127: Q K^T  (M = 128, N = 64, K = 128)
-    tc_fence_after();
-    const uint64_t kq = smem_desc(smem_u32(sm + kIKQ), 16u, 1024u);
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-      const uint64_t off = (uint64_t)((kk >> 2) * (16384 >> 4) + (kk & 3) * 2);
-      mma_bf16(tmem + kTKQ, kq + off, kq + off, idesc_bf16(128, 64, 0, 0), kk > 0);
-    }
-    mma_commit(bar_mma);
-  }
   ok = mbar_wait(bar_mma, ph_mma, err, kErrIntraMma);
   ph_mma ^= 1u;
   if (__syncthreads_or(!ok)) { ok = false; goto teardown; }
