@@ -539,20 +539,20 @@ def gdn_prefill_launches(T: int, n_seq: int = 1, sh=SHAPE, num_sms: int = 148) -
 # of each kernel on the small case (T = 8192, decode batch 64), per unit processed (token
 # for the prefill kernels and the conv, sequence for the decode step), scaled to the
 # benchmark's launch; None when the kernel changed since the capture. The prefill figure is
-# the intra-chunk kernel's 469.72 MB plus the chain kernel's 512.83 MB.
-TRAFFIC_PER_UNIT = {"prefill": (469.72e6 + 512.83e6) / 8192, "conv": 291.25e6 / 8192,
+# the intra-chunk kernel's 468.54 MB plus the chain kernel's 512.83 MB.
+TRAFFIC_PER_UNIT = {"prefill": (468.54e6 + 512.83e6) / 8192, "conv": 291.25e6 / 8192,
                     "decode": 357.64e6 / 64}
 
 # The chunked prefill's two kernels: their share of its FLOPs (from the chunked form: the
 # intra-chunk kernel forms K K^T and Q K^T per key head, solves the triangular system and
 # builds U~ = P V, W = Pk K and Mqk; the chain applies [-W; Q] S0^T, K^T U' and Mqk U), the
 # device time of their launches in one 65536-token call from the ncu launch list (serialised
-# by ncu: eight pieces of each, 1523.1 us of intra-chunk and 2145.3 us of chain launches; in
+# by ncu: eight pieces of each, 1527.1 us of intra-chunk and 2166.0 us of chain launches; in
 # the call the pieces of the two kernels overlap, so the call takes less than their sum), and
 # their DRAM traffic per token from the same captures as above.
 PREFILL_KERNELS = {
-    "chunk_intra": {"busy_us_64k": 1523.1, "traffic_per_token": 469.72e6 / 8192},
-    "chunk_chain": {"busy_us_64k": 2145.3, "traffic_per_token": 512.83e6 / 8192},
+    "chunk_intra": {"busy_us_64k": 1527.1, "traffic_per_token": 468.54e6 / 8192},
+    "chunk_chain": {"busy_us_64k": 2166.0, "traffic_per_token": 512.83e6 / 8192},
 }
 
 
