@@ -283,7 +283,7 @@ def parse():
     ap.add_argument("--T", type=int, default=T_PREFILL)
     ap.add_argument("--decode-batch", type=int, default=B_DECODE)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=6)
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the per-workload report (run after the timed region, N = 1 only)")
     return ap.parse_args()
@@ -452,23 +452,48 @@ def main():
         hdx = dcd.xs[0].pin_memory(); hdg = dcd.gs[0].pin_memory(); hdb = dcd.betas[0].pin_memory()
         hdo = torch.empty_like(do, device="cpu").pin_memory()
 
-        def e2e_step():
-            x.copy_(hx, non_blocking=True); g.copy_(hg, non_blocking=True)
-            beta.copy_(hb, non_blocking=True)
-            gdn.prefill_layer(x, w, g, beta, sh.Hk, sh.Hv, sh.dk, final_state=fin, y=y, o=o,
-                              workspace=ws)
-            ho.copy_(o, non_blocking=True); hfin.copy_(fin, non_blocking=True)
+        # the steps are pipelined as a serving loop runs them: step i's inputs go up on one copy
+        # stream while step i-1 computes on the compute stream and step i-2's outputs come down
+        # on another copy stream (PCIe carries both directions at once), with two sets of device
+        # buffers taken in turn; every step's copies are inside the timed region
+        up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        xb, gb, bb = [x, torch.empty_like(x)], [g, torch.empty_like(g)], [beta, torch.empty_like(beta)]
+        ob, fb = [o, torch.empty_like(o)], [fin, torch.empty_like(fin)]
+        ev_up = [torch.cuda.Event() for _ in range(2)]
+        ev_comp = [torch.cuda.Event() for _ in range(2)]
+        ev_down = [torch.cuda.Event() for _ in range(2)]
+
+        def e2e_step(i):
+            k = i % 2
+            up.wait_event(ev_comp[k])      # step i-2 no longer reads buffer set k
+            with torch.cuda.stream(up):
+                xb[k].copy_(hx, non_blocking=True); gb[k].copy_(hg, non_blocking=True)
+                bb[k].copy_(hb, non_blocking=True)
+            ev_up[k].record(up)
+            stream.wait_event(ev_up[k])
+            stream.wait_event(ev_down[k])  # step i-2's outputs have left buffer set k
+            gdn.prefill_layer(xb[k], w, gb[k], bb[k], sh.Hk, sh.Hv, sh.dk, final_state=fb[k], y=y,
+                              o=ob[k], workspace=ws)
             dx.copy_(hdx, non_blocking=True); dg.copy_(hdg, non_blocking=True)
             db.copy_(hdb, non_blocking=True)
             gdn.gdn_decode_step(dx, dw, dcs, dg, db, dst, sh.Hk, do)
             hdo.copy_(do, non_blocking=True)
+            ev_comp[k].record(stream)
+            down.wait_event(ev_comp[k])
+            with torch.cuda.stream(down):
+                ho.copy_(ob[k], non_blocking=True); hfin.copy_(fb[k], non_blocking=True)
+            ev_down[k].record(down)
 
-        e2e_step(); torch.cuda.synchronize(dev)
+        for i in range(2):
+            e2e_step(i)
+        torch.cuda.synchronize(dev)
         barrier(world)
         a = torch.cuda.Event(enable_timing=True); b = torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
+        up.wait_event(a)
+        for i in range(args.e2e_steps):
+            e2e_step(i)
+        stream.wait_event(ev_down[(args.e2e_steps - 1) % 2])
         b.record(stream)
         torch.cuda.synchronize(dev)
         e2e_ms = max_over_ranks(a.elapsed_time(b), world, dev)
@@ -476,8 +501,10 @@ def main():
         d2h = ho.numel() * 2 + hfin.numel() * 4 + hdo.numel() * 2
         e2e = {"value": world * T * args.e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "note": "prefill tokens/s with the step's x, g, beta copied in from pinned host "
-                       "memory and o + final state copied out, decode step included"}
+               "note": "prefill tokens/s with each step's x, g, beta copied in from pinned host "
+                       "memory and its o + final state copied out, decode step included; steps "
+                       "pipelined (inputs of step i up while step i-1 computes and step i-2's "
+                       "outputs come down), two device buffer sets in turn"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
