@@ -60,7 +60,7 @@ constexpr int kErrIntraTma = 11, kErrIntraMma = 12, kErrChainTma = 21, kErrChain
 // ------------------------------------------------------------------ workspace layout
 
 struct Ws {
-  size_t err, ctr, prefix, wu, ul, mq, vecs, carry, total;
+  size_t err, ctr, prefix, order, wu, ul, mq, vecs, carry, total;
 };
 
 // Per (chunk, value head): wu = [-W (64 x 128) ; U~ (64 x 128)] bf16 rows of 128 elements,
@@ -101,7 +101,8 @@ __host__ __device__ inline Ws ws_layout(int64_t T, int32_t n_seq, int32_t Hv) {
   w.err = 0;
   w.ctr = 64;      // [kMaxPieces] item counters of the intra-chunk kernel, one per piece
   w.prefix = 512;
-  w.wu = align256(w.prefix + (size_t)(n_seq + 1) * 4);
+  w.order = w.prefix + (size_t)(n_seq + 1) * 4;   // [n_seq] sequences, longest first
+  w.wu = align256(w.order + (size_t)n_seq * 4);
   w.ul = align256(w.wu + slots * Hv * kWuBytes);
   w.mq = align256(w.ul + slots * Hv * kUlBytes);
   w.vecs = align256(w.mq + slots * Hv * kMatBytes);
@@ -112,9 +113,14 @@ __host__ __device__ inline Ws ws_layout(int64_t T, int32_t n_seq, int32_t Hv) {
 
 // --------------------------------------------------------------------------- plan
 
+// Sequences ranked by chunk count (longest first, ties by index) for batches of up to this
+// many; larger batches keep their own order.
+constexpr int32_t kOrderMaxSeq = 1024;
+
 __global__ void __launch_bounds__(1024) chunk_plan_kernel(const int32_t* __restrict__ cu,
                                                           int32_t n_seq, int64_t T,
                                                           int32_t* __restrict__ prefix,
+                                                          int32_t* __restrict__ order,
                                                           int* __restrict__ err, int* __restrict__ ctr) {
   __shared__ int32_t warp_tot[32];
   __shared__ int32_t carry;
@@ -155,6 +161,19 @@ __global__ void __launch_bounds__(1024) chunk_plan_kernel(const int32_t* __restr
     __syncthreads();
   }
   if (threadIdx.x == 0) prefix[n_seq] = carry;
+  // the chain kernel takes its sequences in this order, so that the longest chains start in
+  // the first wave of CTAs instead of lengthening the last
+  __syncthreads();
+  for (int32_t n = threadIdx.x; n < n_seq; n += blockDim.x) {
+    if (n_seq > kOrderMaxSeq) { order[n] = n; continue; }
+    const int32_t len = prefix[n + 1] - prefix[n];
+    int32_t rank = 0;
+    for (int32_t m = 0; m < n_seq; ++m) {
+      const int32_t lm = prefix[m + 1] - prefix[m];
+      rank += (lm > len || (lm == len && m < n)) ? 1 : 0;
+    }
+    order[rank] = n;
+  }
 }
 
 // Largest n in [0, n_seq) with prefix[n] <= slot.
@@ -812,7 +831,7 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
   const int32_t* prefix = reinterpret_cast<const int32_t*>(ws_ro + L.prefix);
   const int tile = blockIdx.x % NT;
   const int h = (blockIdx.x / NT) % Hv;
-  const int32_t n = blockIdx.x / (NT * Hv);
+  const int32_t n = reinterpret_cast<const int32_t*>(ws_ro + L.order)[blockIdx.x / (NT * Hv)];
   const int hk = h / (Hv / Hk);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // storage of the initial, final and block states: fp32, or bf16 (kStateInitBf16 ...)
@@ -1311,6 +1330,7 @@ cudaError_t launch_prefill_chunk_tc(const void* q, const void* k, const void* v,
                 !make_map(&mo, o, (uint64_t)Hv * D, (uint64_t)T, (uint64_t)Hv * D)))
     return cudaErrorInvalidValue;
   chunk_plan_kernel<<<1, 1024, 0, stream>>>(cu, n_seq, T, reinterpret_cast<int32_t*>(ws + L.prefix),
+                                            reinterpret_cast<int32_t*>(ws + L.order),
                                             reinterpret_cast<int*>(ws + L.err),
                                             reinterpret_cast<int*>(ws + L.ctr));
   const int user_bf = state_dtype == kBF16 ? 1 : 0;
