@@ -193,6 +193,11 @@ __device__ __forceinline__ uint32_t tmem_quadrant(uint32_t tmem, int warp) {
   return tmem + ((uint32_t)(warp * 32) << 16);
 }
 
+// Barrier `id` (1..15) over `threads` threads (a multiple of 32).
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 // ------------------------------------------------------------------------ intra
 
 // Warp-level MMAs (m16n8k8, tf32 inputs, fp32 accumulate) for the 16 x 16 block products of the
@@ -233,6 +238,16 @@ __device__ __forceinline__ void block_mma16(float (&c)[2][4], const float* Xs, i
   block_mma16h(c[1], Xs, px, xr, xc, Ys, py, yr, yc, 1, lane);
 }
 
+// Stores sign * (one m16n8 accumulator fragment) into columns co .. co + 7 of a 16-row block
+// of an fp32 matrix with row pitch p.
+__device__ __forceinline__ void frag_store(float* M, int p, int co, const float (&c)[4], int lane, float sign) {
+  const int g = lane >> 2, t = lane & 3;
+  float* row0 = M + g * p + co + 2 * t;
+  float* row8 = row0 + 8 * p;
+  row0[0] = sign * c[0]; row0[1] = sign * c[1];
+  row8[0] = sign * c[2]; row8[1] = sign * c[3];
+}
+
 // shared memory of the intra kernel (offsets from a 1024-aligned base)
 constexpr int kMaxG = kPrefillTcMaxG;           // value heads per key head on this path
 constexpr int kIKQ = 0;                         // [K0 | Q0 | K1 | Q1]: [K; Q] is one 128-row operand
@@ -251,7 +266,10 @@ constexpr int kIVec = kITmp + 4 * 16 * kLd16 * 4;   // rq, rk, G, colP, colPk, c
 constexpr int kIGB = kIVec + 6 * 64 * 4;        // g, beta of every value head [2][kMaxG][64]
 constexpr int kIBar = kIGB + 2 * kMaxG * 64 * 4;    // 4 mbarriers + tmem address
 constexpr int kIntraSmem = kIBar + 64 + 1024;   // + alignment slack
-constexpr uint32_t kTKQ = 0, kTUW = 128;        // TMEM columns: [KK^T; QK^T], [P;Pk] V or K
+// TMEM columns: [KK^T; QK^T] (N = 64); [P; Pk] V (N = 128); [P; Pk] K in two N = 64 halves,
+// the first beside the other two, the second into the columns of [P; Pk] V that the U~
+// epilogue has read first
+constexpr uint32_t kTKQ = 0, kTWa = 64, kTU = 128, kTWb = 128;
 
 __global__ void __launch_bounds__(128, 2)   // two CTAs per SM (shared and tensor memory allow two)
 chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
@@ -291,6 +309,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
   uint64_t* bar_drain = bar_tma + 4;   // on an early exit: every MMA of this CTA has completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_tma + 5);
   int32_t* next_item = reinterpret_cast<int32_t*>(bar_tma + 6);   // taken by thread 0 per item
+  uint64_t* bar_mma2 = bar_tma + 7;   // the second half of [P; Pk] K has completed
   // loads issued into each barrier (thread 0 only): an early exit waits for the last of each
   uint32_t n_kq = 0, n_v0 = 0, n_v1 = 0;
 
@@ -356,6 +375,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     mbar_init(&bar_v[0], 1);
     mbar_init(&bar_v[1], 1);
     mbar_init(bar_drain, 1);
+    mbar_init(bar_mma2, 1);
     fence_mbar_init();
   }
   if (warp == 0) { tmem_alloc(tmem_slot, 256); tmem_relinquish(); }
@@ -369,7 +389,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
   store_gb();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tq = tmem_quadrant(tmem, warp);   // lanes 32 w .. 32 w + 31: rows of M = 128 results
-  uint32_t ph_mma = 0u, ph_kq = 0u;
+  uint32_t ph_mma = 0u, ph_mma2 = 0u, ph_kq = 0u;
   uint32_t vbase0 = 0u, vbase1 = 0u;   // completed loads of V buffers 0 and 1 before this item
   bool ok = true;
   __syncthreads();
@@ -501,80 +521,71 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
       }
       if (tid >= 64) fence_async_smem();
     }
-    __syncthreads();
-    if (tid == 0) {
-      tma_store_2d(&map_mq, 0, (int32_t)(((int64_t)slot * Hv + h) * C), mq_stage);
-      tma_store_commit();
-    }
-
-    // Tm = (I + A)^{-1}. Diagonal 16x16 blocks, one warp each, by fp32 forward substitution:
-    // lane j < 16 solves column j of (I + L) X = I (L the block of A, strictly lower):
+    // Tm = (I + A)^{-1}. Diagonal 16x16 blocks by the warp that wrote their rows of A (warp w,
+    // w < 2: blocks 2w and 2w + 1, one per half warp), by fp32 forward substitution: lane
+    // col of its half solves column col of (I + L) X = I (L the block of A, strictly lower):
     // x_i = delta_ij - sum_{k<i} L_ik x_k, accumulating each x_k into every later row as soon
-    // as it is known (a 15-step dependent chain; the L loads are warp broadcasts). The column
-    // stays in registers until it is complete, so no store to Tm sits between the loads of L.
-    if (lane < 16) {
-      const int b0 = warp * 16, j = lane;
+    // as it is known (a 15-step dependent chain; the L loads are half-warp broadcasts, the two
+    // halves on different banks). The column stays in registers until it is complete, so no
+    // store to Tm sits between the loads of L.
+    if (warp < 2) {
+      __syncwarp();
+      const int b0 = (2 * warp + (lane >> 4)) * 16, col = lane & 15;
       float acc[16], x[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) acc[i] = 0.f;
 #pragma unroll
       for (int k = 0; k < 16; ++k) {
-        x[k] = k == j ? 1.f : (k < j ? 0.f : -acc[k]);
+        x[k] = k == col ? 1.f : (k < col ? 0.f : -acc[k]);
 #pragma unroll
         for (int i = k + 1; i < 16; ++i) acc[i] = fmaf(Am[(b0 + i) * kLdA + b0 + k], x[k], acc[i]);   // L(i, k)
       }
 #pragma unroll
-      for (int k = 0; k < 16; ++k) Tm[(b0 + k) * kLd + b0 + j] = x[k];
+      for (int k = 0; k < 16; ++k) Tm[(b0 + k) * kLd + b0 + col] = x[k];
+      // the same warp closes its 32 x 32 diagonal block: Tm_ba = -Tm_bb A_ba Tm_aa for
+      // a = 2w, b = 2w + 1 (tf32 warp MMAs), from blocks only this warp has written
+      __syncwarp();
+      const int aa = 2 * warp, bb = aa + 1;
+      float c[2][4] = {};
+      block_mma16(c, Am, kLdA, 16 * bb, 16 * aa, Tm, kLd, 16 * aa, 16 * aa, lane);
+#pragma unroll
+      for (int nh = 0; nh < 2; ++nh) frag_store(scratch, kLd16, 8 * nh, c[nh], lane, 1.f);
+      __syncwarp();
+      float d[2][4] = {};
+      block_mma16(d, Tm, kLd, 16 * bb, 16 * bb, scratch, kLd16, 0, 0, lane);
+#pragma unroll
+      for (int nh = 0; nh < 2; ++nh)
+        frag_store(Tm + 16 * bb * kLd + 16 * aa, kLd, 8 * nh, d[nh], lane, -1.f);
     }
     __syncthreads();
-    // off-diagonal blocks by block distance: Tm_ba = -Tm_bb sum_c A_bc Tm_ca (tf32 warp MMAs).
-    // Distance 1: one warp per block; distances 2 and 3: two warps per block, one 8-column
-    // half each (a half of the result needs only the same half of the inner sum).
-    for (int dist = 1; dist < 4; ++dist) {
-      const int gq = lane >> 2, tq4 = lane & 3;
-      if (dist == 1) {
-        if (warp < 3) {
-          const int aa = warp, bb = warp + 1;
-          float c[2][4] = {};
-          block_mma16(c, Am, kLdA, 16 * bb, 16 * aa, Tm, kLd, 16 * aa, 16 * aa, lane);
-#pragma unroll
-          for (int nh = 0; nh < 2; ++nh) {
-            scratch[gq * kLd16 + 8 * nh + 2 * tq4] = c[nh][0];
-            scratch[gq * kLd16 + 8 * nh + 2 * tq4 + 1] = c[nh][1];
-            scratch[(gq + 8) * kLd16 + 8 * nh + 2 * tq4] = c[nh][2];
-            scratch[(gq + 8) * kLd16 + 8 * nh + 2 * tq4 + 1] = c[nh][3];
-          }
-          __syncwarp();
-          float d[2][4] = {};
-          block_mma16(d, Tm, kLd, 16 * bb, 16 * bb, scratch, kLd16, 0, 0, lane);
-#pragma unroll
-          for (int nh = 0; nh < 2; ++nh) {
-            float* row0 = Tm + (16 * bb + gq) * kLd + 16 * aa + 8 * nh + 2 * tq4;
-            float* row8 = row0 + 8 * kLd;
-            row0[0] = -d[nh][0]; row0[1] = -d[nh][1];
-            row8[0] = -d[nh][2]; row8[1] = -d[nh][3];
-          }
-        }
-      } else if (warp < 2 * (4 - dist)) {
-        const int aa = warp >> 1, bb = aa + dist, nh = warp & 1;
-        float c[4] = {};
-        for (int cblk = aa; cblk < bb; ++cblk)
-          block_mma16h(c, Am, kLdA, 16 * bb, 16 * cblk, Tm, kLd, 16 * cblk, 16 * aa, nh, lane);
-        scratch[gq * kLd16 + 8 * nh + 2 * tq4] = c[0];
-        scratch[gq * kLd16 + 8 * nh + 2 * tq4 + 1] = c[1];
-        scratch[(gq + 8) * kLd16 + 8 * nh + 2 * tq4] = c[2];
-        scratch[(gq + 8) * kLd16 + 8 * nh + 2 * tq4 + 1] = c[3];
-        __syncwarp();
-        float d[4] = {};
-        block_mma16h(d, Tm, kLd, 16 * bb, 16 * bb, scratch, kLd16, 0, 0, nh, lane);
-        float* row0 = Tm + (16 * bb + gq) * kLd + 16 * aa + 8 * nh + 2 * tq4;
-        float* row8 = row0 + 8 * kLd;
-        row0[0] = -d[0]; row0[1] = -d[1];
-        row8[0] = -d[2]; row8[1] = -d[3];
-      }
-      if (dist == 3 && tid == 0) tma_store_wait_read();   // Mqk left its staging tile ([P | Pk])
-      __syncthreads();
+    if (tid == 0) {
+      tma_store_2d(&map_mq, 0, (int32_t)(((int64_t)slot * Hv + h) * C), mq_stage);
+      tma_store_commit();
     }
+    // the lower-left 32 x 32 block: with X = A[32:64, 0:32] Tm[0:32, 0:32],
+    // Tm[32:64, 0:32] = -Tm[32:64, 32:64] X, i.e. per 16-column block a:
+    //   Tm_2a = -Tm_22 X_2a,  Tm_3a = -(Tm_32 X_2a + Tm_33 X_3a),  X_ba = sum_{c=a}^{1} A_bc Tm_ca.
+    // Warp w takes column block a = w / 2 and 8-column half w % 2 of both results (a half of
+    // a result needs only the same half of X), so the round needs no barrier inside it.
+    {
+      const int aa = warp >> 1, nh = warp & 1;
+      float x2[4] = {}, x3[4] = {};
+      for (int cblk = aa; cblk < 2; ++cblk) {
+        block_mma16h(x2, Am, kLdA, 32, 16 * cblk, Tm, kLd, 16 * cblk, 16 * aa, nh, lane);
+        block_mma16h(x3, Am, kLdA, 48, 16 * cblk, Tm, kLd, 16 * cblk, 16 * aa, nh, lane);
+      }
+      frag_store(scratch, kLd16, 0, x2, lane, 1.f);   // X_2a half in columns 0..7
+      frag_store(scratch, kLd16, 8, x3, lane, 1.f);   // X_3a half in columns 8..15
+      __syncwarp();
+      float t2[4] = {}, t3[4] = {};
+      block_mma16h(t2, Tm, kLd, 32, 32, scratch, kLd16, 0, 0, 0, lane);
+      block_mma16h(t3, Tm, kLd, 48, 32, scratch, kLd16, 0, 0, 0, lane);
+      block_mma16h(t3, Tm, kLd, 48, 48, scratch, kLd16, 0, 8, 0, lane);
+      frag_store(Tm + 32 * kLd + 16 * aa, kLd, 8 * nh, t2, lane, -1.f);
+      frag_store(Tm + 48 * kLd + 16 * aa, kLd, 8 * nh, t3, lane, -1.f);
+    }
+    if (tid == 0) tma_store_wait_read();   // Mqk left its staging tile ([P | Pk])
+    __syncthreads();
 
     // [P | Pk] as bf16 K-major operands: warps 0, 1 form P, warps 2, 3 Pk. A lane takes 4
     // columns (chunk c) of a row per step, a warp 8 rows x 4 chunks with the 8 rows on
@@ -617,13 +628,19 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     __syncthreads();
 
     const uint64_t dpp = smem_desc(smem_u32(sm + kIPP), 16u, 1024u);
-    if (tid == 0) {   // [P; Pk] V: rows 0..63 = U~ (M = 128, N = 128, K = 64)
+    // K as the MN-major B operand of [P; Pk] K (N = dk, K = the chunk's rows), half h at atom h
+    const uint64_t dk = smem_desc(smem_u32(sm + kIKQ), 16384u, 1024u);
+    if (tid == 0) {   // [P; Pk] V: rows 0..63 = U~ (M = 128, N = 128, K = 64), and beside it
+                      // [P; Pk] K atom 0: rows 64..127 = W columns 0..63 (N = 64)
       if (mbar_wait(&bar_v[j & 1], ((j & 1 ? vbase1 : vbase0) + (uint32_t)(j >> 1)) & 1u, err, kErrIntraTma)) {
         tc_fence_after();
         const uint64_t dv = smem_desc(smem_u32(v_tile(j & 1)), (j & 1) ? 16384u : 8192u, 1024u);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmem + kTUW, dpp + 2 * kk, dv + 128 * kk, idesc_bf16(128, 128, 0, 1), kk > 0);
+          mma_bf16(tmem + kTU, dpp + 2 * kk, dv + 128 * kk, idesc_bf16(128, 128, 0, 1), kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmem + kTWa, dpp + 2 * kk, dk + 128 * kk, idesc_bf16(128, 64, 0, 1), kk > 0);
         mma_commit(bar_mma);
       }
     }
@@ -632,17 +649,30 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     if (__syncthreads_or(!ok)) { ok = false; goto teardown; }
     tc_fence_after();
     if (tid == 0 && j + 2 < G) load_v(cur, j + 2);   // this V buffer is free
-    // U~ (rows 0..63 of the result) -> bf16 tile [64][128] in the free A region -> TMA store
-    uint8_t* stage_u = sm + kIA;   // U~: 2 swizzled atoms of [64][64]
+    uint8_t* stage_u = sm + kIA;   // U~: 2 swizzled atoms of [64][64] in the free A region
     uint8_t* stage_ul = sm + kIT;  // U~ - bf16(U~), in the Tm region (read for the last time
                                    // by the [P | Pk] build)
+    uint8_t* stage_w = sm + kIPP;  // -W, in [P | Pk] once the last MMA reading it has completed
     if (warp < 2) {
+      // U~ (rows 0..63) -> bf16 hi + lo tiles. Once its first 64 columns are in registers,
+      // thread 0 issues [P; Pk] K atom 1 into them, behind the rest of this epilogue.
 #pragma unroll
       for (int cp = 0; cp < 4; cp += 2) {
         uint32_t raw[2][32];
-        tmem_ld32_async(tq + kTUW + cp * 32, raw[0]);
-        tmem_ld32_async(tq + kTUW + cp * 32 + 32, raw[1]);
+        tmem_ld32_async(tq + kTU + cp * 32, raw[0]);
+        tmem_ld32_async(tq + kTU + cp * 32 + 32, raw[1]);
         tmem_wait_ld(raw[0], raw[1]);
+        if (cp == 0) {
+          tc_fence_before();
+          named_bar_sync(1, 64);
+          if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16(tmem + kTWb, dpp + 2 * kk, dk + (16384 >> 4) + 128 * kk, idesc_bf16(128, 64, 0, 1), kk > 0);
+            mma_commit(bar_mma2);
+          }
+        }
 #pragma unroll
         for (int hb = 0; hb < 2; ++hb) {
           const int cb = cp + hb;
@@ -661,65 +691,60 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
           }
         }
       }
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    const int32_t wrow = (int32_t)(((int64_t)slot * Hv + h) * 2 * C);
-    if (tid == 0) {
-      tma_store_2d(&map_wu, 0, wrow + C, stage_u);
-      tma_store_2d(&map_wu, 64, wrow + C, stage_u + 8192);
-      const int32_t lrow = (int32_t)(((int64_t)slot * Hv + h) * C);
-      tma_store_2d(&map_ul, 0, lrow, stage_ul);
-      tma_store_2d(&map_ul, 64, lrow, stage_ul + 8192);
-      tma_store_commit();
-    }
-    if (tid == 0) {   // [P; Pk] K: rows 64..127 = W (N = 128, K read MN-major across its atoms)
-      tc_fence_after();
-      const uint64_t dk = smem_desc(smem_u32(sm + kIKQ), 16384u, 1024u);
+    } else {
+      // -W (rows 64..127): columns 0..63 are converted while [P; Pk] K atom 1 runs, and
+      // both halves are written once it has completed
+      const int r = tid - 64;
+      auto neg_pack = [](const uint32_t (&x)[2][32], uint32_t (&p)[32]) {
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + kTUW, dpp + 2 * kk, dk + 128 * kk, idesc_bf16(128, 128, 0, 1), kk > 0);
-      mma_commit(bar_mma);
-    }
-    ok = mbar_wait(bar_mma, ph_mma, err, kErrIntraMma);
-    ph_mma ^= 1u;
-    if (__syncthreads_or(!ok)) { ok = false; goto teardown; }
-    tc_fence_after();
-    if (j == G - 1 && has_next) {
-      // every MMA of this item has read K, Q and the V tiles: fetch the next item's inputs
-      if (tid == 0) load_kqv(nxt);
-    }
-    uint8_t* stage_w = sm + kIPP;  // -W (rows 64..127 of the result) staged in [P | Pk], which
-                                   // the MMA that produced it has finished reading
-    if (warp >= 2) {
-#pragma unroll
-      for (int cp = 0; cp < 4; cp += 2) {
-        uint32_t raw[2][32];
-        tmem_ld32_async(tq + kTUW + cp * 32, raw[0]);
-        tmem_ld32_async(tq + kTUW + cp * 32 + 32, raw[1]);
-        tmem_wait_ld(raw[0], raw[1]);
-#pragma unroll
-        for (int hb = 0; hb < 2; ++hb) {
-          const int cb = cp + hb;
-          uint8_t* atom = stage_w + (cb >> 1) * 8192;
-#pragma unroll
-          for (int c8 = 0; c8 < 4; ++c8) {
-            float v8[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) v8[q] = -__uint_as_float(raw[hb][c8 * 8 + q]);
-            VecIO<bf16, 8>::store(reinterpret_cast<bf16*>(atom + sw128_off(tid - 64, (cb & 1) * 32 + c8 * 8)), v8);
-          }
+        for (int q = 0; q < 32; ++q) {
+          const __nv_bfloat162 t = __floats2bfloat162_rn(-__uint_as_float(x[q >> 4][(2 * q) & 31]),
+                                                         -__uint_as_float(x[q >> 4][(2 * q + 1) & 31]));
+          p[q] = *reinterpret_cast<const uint32_t*>(&t);
         }
+      };
+      auto store_atom = [&](const uint32_t (&p)[32], uint8_t* atom) {
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8)
+          *reinterpret_cast<uint4*>(atom + sw128_off(r, c8 * 8)) =
+              make_uint4(p[4 * c8], p[4 * c8 + 1], p[4 * c8 + 2], p[4 * c8 + 3]);
+      };
+      uint32_t wp[32];
+      {
+        uint32_t raw[2][32];
+        tmem_ld32_async(tq + kTWa, raw[0]);
+        tmem_ld32_async(tq + kTWa + 32, raw[1]);
+        tmem_wait_ld(raw[0], raw[1]);
+        neg_pack(raw, wp);
+      }
+      ok = mbar_wait(bar_mma2, ph_mma2, err, kErrIntraMma);
+      tc_fence_after();
+      if (ok) {
+        store_atom(wp, stage_w);
+        uint32_t raw[2][32];
+        tmem_ld32_async(tq + kTWb, raw[0]);
+        tmem_ld32_async(tq + kTWb + 32, raw[1]);
+        tmem_wait_ld(raw[0], raw[1]);
+        neg_pack(raw, wp);
+        store_atom(wp, stage_w + 8192);
       }
     }
+    ph_mma2 ^= 1u;
     fence_async_smem();
     tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {   // read out before the next head rewrites [P | Pk] (waited there)
-      tma_store_2d(&map_wu, 0, wrow, stage_w);
-      tma_store_2d(&map_wu, 64, wrow, stage_w + 8192);
+    if (__syncthreads_or(!ok)) { ok = false; goto teardown; }
+    if (tid == 0) {
+      const int32_t wrow = (int32_t)(((int64_t)slot * Hv + h) * 2 * C);
+      const int32_t lrow = (int32_t)(((int64_t)slot * Hv + h) * C);
+      tma_store_2d(&map_wu, 0, wrow + C, stage_u);
+      tma_store_2d(&map_wu, 64, wrow + C, stage_u + 8192);
+      tma_store_2d(&map_ul, 0, lrow, stage_ul);
+      tma_store_2d(&map_ul, 64, lrow, stage_ul + 8192);
+      tma_store_2d(&map_wu, 0, wrow, stage_w);   // read out before the next head rewrites
+      tma_store_2d(&map_wu, 64, wrow, stage_w + 8192);   // [P | Pk] (waited there)
       tma_store_commit();
+      // every MMA of this item has read K, Q and the V tiles: fetch the next item's inputs
+      if (j == G - 1 && has_next) load_kqv(nxt);
     }
     tc_fence_before();
   }
@@ -788,9 +813,6 @@ constexpr int kStateInitBf16 = 1, kStateFinBf16 = 2, kStateBlocksBf16 = 4;   // 
 // chunk c - 2's output warps had read the same buffer.
 constexpr uint32_t kTAlo = 0, kTAhi = 128, kTdS = 256, kTO2 = 384;
 
-__device__ __forceinline__ void named_bar_sync(int id, int threads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
-}
 // Barrier over `threads` threads that also returns whether any of them passed `pred`.
 __device__ __forceinline__ bool named_bar_or(int id, int threads, bool pred) {
   uint32_t r;
