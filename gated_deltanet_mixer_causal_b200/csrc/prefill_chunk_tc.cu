@@ -197,6 +197,15 @@ __device__ __forceinline__ uint32_t tmem_quadrant(uint32_t tmem, int warp) {
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
+// Barrier over `threads` threads that also returns whether any of them passed `pred`.
+__device__ __forceinline__ bool named_bar_or(int id, int threads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n"
+      " bar.red.or.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r) : "r"((uint32_t)pred), "r"(id), "r"(threads) : "memory");
+  return r != 0;
+}
 
 // ------------------------------------------------------------------------ intra
 
@@ -265,7 +274,7 @@ constexpr int kLd16 = 24;
 constexpr int kIVec = kITmp + 4 * 16 * kLd16 * 4;   // rq, rk, G, colP, colPk, colInv [6][64]
 constexpr int kIGB = kIVec + 6 * 64 * 4;        // g, beta of every value head [2][kMaxG][64]
 constexpr int kIBar = kIGB + 2 * kMaxG * 64 * 4;    // 4 mbarriers + tmem address
-constexpr int kIntraSmem = kIBar + 64 + 1024;   // + alignment slack
+constexpr int kIntraSmem = kIBar + 128 + 1024;  // + alignment slack
 // TMEM columns: [KK^T; QK^T] (N = 64); [P; Pk] V (N = 128); [P; Pk] K in two N = 64 halves,
 // the first beside the other two, the second into the columns of [P; Pk] V that the U~
 // epilogue has read first
@@ -303,20 +312,23 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
   float* colInv = rq + 320;
   float* gAll = reinterpret_cast<float*>(sm + kIGB);
   float* bAll = gAll + kMaxG * 64;
-  uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + kIBar);   // K and Q landed
+  uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + kIBar);   // K landed
   uint64_t* bar_mma = bar_tma + 1;
   uint64_t* bar_v = bar_tma + 2;   // [2] V tile of a value head landed in buffer j % 2
   uint64_t* bar_drain = bar_tma + 4;   // on an early exit: every MMA of this CTA has completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_tma + 5);
   int32_t* next_item = reinterpret_cast<int32_t*>(bar_tma + 6);   // taken by thread 0 per item
   uint64_t* bar_mma2 = bar_tma + 7;   // the second half of [P; Pk] K has completed
+  uint64_t* bar_q = bar_tma + 8;      // Q landed
   // loads issued into each barrier (thread 0 only): an early exit waits for the last of each
-  uint32_t n_kq = 0, n_v0 = 0, n_v1 = 0;
+  uint32_t n_k = 0, n_q = 0, n_v0 = 0, n_v1 = 0;   // n_k: thread 64's
 
   // The CTA is persistent: its first item is item_lo + blockIdx.x, and each further one is
   // taken from the piece's counter while the current one starts (so CTAs that become
-  // resident late, beside another kernel, take fewer). Each item's K, Q, the first V tile and
-  // its g, beta are fetched while the previous item finishes.
+  // resident late, beside another kernel, take fewer). Each item's inputs are fetched as soon
+  // as the previous item's last reader of their buffers has completed: Q and the first V tile
+  // during its last value heads, K once its last [P; Pk] K is done, g and beta during its
+  // last head.
   struct Item { int32_t slot, hk; int64_t t0; int len; };
   auto item_at = [&](int32_t it, Item& x) {
     if (it >= n_items) return false;
@@ -340,15 +352,23 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     for (int hh = 0; hh < 2; ++hh)
       tma_load_2d(dst + hh * atom, &map_v, (x.hk * G + j) * D + hh * 64, (int32_t)x.t0, &bar_v[j & 1]);
   };
-  auto load_kqv = [&](const Item& x) {   // thread 0: K, Q and the first V tile of item x
-    ++n_kq;
-    mbar_arrive_expect_tx(bar_tma, 32768);
-    for (int hh = 0; hh < 2; ++hh) {
+  // K of item x (thread 64, as soon as the last MMA reading K has completed), Q (thread 0,
+  // once the last V tile in the Q atoms has been read)
+  auto load_k = [&](const Item& x) {
+    ++n_k;
+    mbar_arrive_expect_tx(bar_tma, 16384);
+    for (int hh = 0; hh < 2; ++hh)
       tma_load_2d(sm + kIKQ + hh * 16384, &map_k, x.hk * D + hh * 64, (int32_t)x.t0, bar_tma);
-      tma_load_2d(sm + kIKQ + hh * 16384 + 8192, &map_q, x.hk * D + hh * 64, (int32_t)x.t0, bar_tma);
-    }
-    load_v(x, 0);
   };
+  auto load_q = [&](const Item& x) {
+    ++n_q;
+    mbar_arrive_expect_tx(bar_q, 16384);
+    for (int hh = 0; hh < 2; ++hh)
+      tma_load_2d(sm + kIKQ + hh * 16384 + 8192, &map_q, x.hk * D + hh * 64, (int32_t)x.t0, bar_q);
+  };
+  // the last value heads whose V tiles use buffer 1 (the Q atoms) and buffer 0: once their
+  // [P; Pk] V has completed, the next item's Q and first V tile are loaded into them
+  const int j_q = (G & 1) ? G - 2 : G - 1, j_v = (G & 1) ? G - 1 : G - 2;
   // g, beta of the G value heads of item x, this thread's share (rows past the sequence: 0)
   constexpr int kGB = kMaxG * 64 / 128;
   float gr[kGB], br[kGB];
@@ -376,6 +396,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     mbar_init(&bar_v[1], 1);
     mbar_init(bar_drain, 1);
     mbar_init(bar_mma2, 1);
+    mbar_init(bar_q, 1);
     fence_mbar_init();
   }
   if (warp == 0) { tmem_alloc(tmem_slot, 256); tmem_relinquish(); }
@@ -385,7 +406,8 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (tid == 0) load_kqv(cur);
+  if (tid == 0) { load_q(cur); load_v(cur, 0); }
+  if (tid == 64) load_k(cur);
   store_gb();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tq = tmem_quadrant(tmem, warp);   // lanes 32 w .. 32 w + 31: rows of M = 128 results
@@ -414,7 +436,7 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
       gAll[j * 64 + 2 * lane + 1] = excl + a0 + a1;
     }
   }
-  ok = mbar_wait(bar_tma, ph_kq, err, kErrIntraTma);
+  ok = mbar_wait(bar_tma, ph_kq, err, kErrIntraTma) && mbar_wait(bar_q, ph_kq, err, kErrIntraTma);
   ph_kq ^= 1u;
   if (__syncthreads_or(!ok)) { ok = false; goto teardown; }
   has_next = item_at(*next_item, nxt);   // thread 0 wrote it before the barrier above
@@ -453,7 +475,10 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
   ph_mma ^= 1u;
   if (__syncthreads_or(!ok)) { ok = false; goto teardown; }
   tc_fence_after();
-  if (tid == 0 && G > 1) load_v(cur, 1);   // into the Q atoms, which the MMA has finished reading
+  if (tid == 0) {   // into the Q atoms, which the MMA and the norms have finished reading
+    if (G > 1) load_v(cur, 1);
+    else if (has_next) load_q(nxt);
+  }
 
   for (int j = 0; j < G; ++j) {
     const int h = hk * G + j;
@@ -467,8 +492,13 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
       colPk[tid] = sb[tid] * __expf(sG[tid]) * rk[tid];
       colInv[tid] = -sG[C - 1] < 60.f ? __expf(-sG[tid]) * rk[tid] : 0.f;
     }
-    if (tid == 0) tma_store_wait_read();   // the previous head's staged tiles (A, Tm, [P | Pk])
     __syncthreads();
+    // each warp pair waits only for its own staging tiles of the previous head to be read out:
+    // warps 0, 1 for U~ (in the A and Tm regions, stored by thread 0), warps 2, 3 for -W
+    // (in [P | Pk], stored by thread 64)
+    if (tid == 0 || tid == 64) tma_store_wait_read();
+    if (warp < 2) named_bar_sync(1, 64);
+    else named_bar_sync(2, 64);
 
     // thread t < 64: row t of A from K K^T; t >= 64: row t-64 of Mqk, staged (swizzled) in
     // the [P | Pk] region, which is free until the solve is done, and stored by TMA.
@@ -648,11 +678,17 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     ph_mma ^= 1u;
     if (__syncthreads_or(!ok)) { ok = false; goto teardown; }
     tc_fence_after();
-    if (tid == 0 && j + 2 < G) load_v(cur, j + 2);   // this V buffer is free
+    if (tid == 0) {   // this V buffer is free
+      if (j + 2 < G) load_v(cur, j + 2);
+      else if (has_next && j == j_q) load_q(nxt);
+      else if (has_next && j == j_v) load_v(nxt, 0);
+    }
     uint8_t* stage_u = sm + kIA;   // U~: 2 swizzled atoms of [64][64] in the free A region
     uint8_t* stage_ul = sm + kIT;  // U~ - bf16(U~), in the Tm region (read for the last time
                                    // by the [P | Pk] build)
     uint8_t* stage_w = sm + kIPP;  // -W, in [P | Pk] once the last MMA reading it has completed
+    const int32_t wrow = (int32_t)(((int64_t)slot * Hv + h) * 2 * C);   // [-W; U~] rows
+    const int32_t lrow = (int32_t)(((int64_t)slot * Hv + h) * C);       // U~lo rows
     if (warp < 2) {
       // U~ (rows 0..63) -> bf16 hi + lo tiles. Once its first 64 columns are in registers,
       // thread 0 issues [P; Pk] K atom 1 into them, behind the rest of this epilogue.
@@ -690,6 +726,14 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
             *reinterpret_cast<uint4*>(atom_l + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
           }
         }
+        // this pass's atom of U~ and U~lo leaves at once (64 columns each)
+        fence_async_smem();
+        named_bar_sync(1, 64);
+        if (tid == 0) {
+          tma_store_2d(&map_wu, cp * 32, wrow + C, stage_u + (cp >> 1) * 8192);
+          tma_store_2d(&map_ul, cp * 32, lrow, stage_ul + (cp >> 1) * 8192);
+          tma_store_commit();
+        }
       }
     } else {
       // -W (rows 64..127): columns 0..63 are converted while [P; Pk] K atom 1 runs, and
@@ -718,6 +762,8 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
         neg_pack(raw, wp);
       }
       ok = mbar_wait(bar_mma2, ph_mma2, err, kErrIntraMma);
+      // the last MMA reading K has completed: the next item's K
+      if (tid == 64 && ok && j == G - 1 && has_next) load_k(nxt);
       tc_fence_after();
       if (ok) {
         store_atom(wp, stage_w);
@@ -728,24 +774,17 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
         neg_pack(raw, wp);
         store_atom(wp, stage_w + 8192);
       }
+      fence_async_smem();
+      if (named_bar_or(2, 64, !ok)) ok = false;
+      if (tid == 64 && ok) {   // read out before the next head's Mqk rewrites [P | Pk]
+        tma_store_2d(&map_wu, 0, wrow, stage_w);
+        tma_store_2d(&map_wu, 64, wrow, stage_w + 8192);
+        tma_store_commit();
+      }
     }
     ph_mma2 ^= 1u;
-    fence_async_smem();
     tc_fence_before();
     if (__syncthreads_or(!ok)) { ok = false; goto teardown; }
-    if (tid == 0) {
-      const int32_t wrow = (int32_t)(((int64_t)slot * Hv + h) * 2 * C);
-      const int32_t lrow = (int32_t)(((int64_t)slot * Hv + h) * C);
-      tma_store_2d(&map_wu, 0, wrow + C, stage_u);
-      tma_store_2d(&map_wu, 64, wrow + C, stage_u + 8192);
-      tma_store_2d(&map_ul, 0, lrow, stage_ul);
-      tma_store_2d(&map_ul, 64, lrow, stage_ul + 8192);
-      tma_store_2d(&map_wu, 0, wrow, stage_w);   // read out before the next head rewrites
-      tma_store_2d(&map_wu, 64, wrow, stage_w + 8192);   // [P | Pk] (waited there)
-      tma_store_commit();
-      // every MMA of this item has read K, Q and the V tiles: fetch the next item's inputs
-      if (j == G - 1 && has_next) load_kqv(nxt);
-    }
     tc_fence_before();
   }
   vbase0 += (uint32_t)(G + 1) / 2;
@@ -759,12 +798,16 @@ chunk_intra_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
 teardown:
   if (tid == 0) {
     if (!ok) {   // a wait gave up: let this CTA's loads and MMAs in flight finish (bounded)
-      if (n_kq) mbar_wait(bar_tma, (n_kq - 1) & 1u, nullptr, 0);
+      if (n_q) mbar_wait(bar_q, (n_q - 1) & 1u, nullptr, 0);
       if (n_v0) mbar_wait(&bar_v[0], (n_v0 - 1) & 1u, nullptr, 0);
       if (n_v1) mbar_wait(&bar_v[1], (n_v1 - 1) & 1u, nullptr, 0);
       mma_commit(bar_drain);
       mbar_wait(bar_drain, 0u, nullptr, 0);
     }
+    tma_store_wait_all();
+  }
+  if (tid == 64) {   // its -W stores and, after a wait gave up, its K load in flight
+    if (!ok && n_k) mbar_wait(bar_tma, (n_k - 1) & 1u, nullptr, 0);
     tma_store_wait_all();
   }
   tc_fence_before();
@@ -813,15 +856,6 @@ constexpr int kStateInitBf16 = 1, kStateFinBf16 = 2, kStateBlocksBf16 = 4;   // 
 // chunk c - 2's output warps had read the same buffer.
 constexpr uint32_t kTAlo = 0, kTAhi = 128, kTdS = 256, kTO2 = 384;
 
-// Barrier over `threads` threads that also returns whether any of them passed `pred`.
-__device__ __forceinline__ bool named_bar_or(int id, int threads, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n"
-      " bar.red.or.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}\n"
-      : "=r"(r) : "r"((uint32_t)pred), "r"(id), "r"(threads) : "memory");
-  return r != 0;
-}
 // Wait until at most one committed bulk store group of this thread still reads shared memory.
 __device__ __forceinline__ void tma_store_wait_read_le1() {
   asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
