@@ -551,15 +551,12 @@ def main():
 
 
 def gdn_prefill_launches(T: int, n_seq: int = 1, sh=SHAPE, num_sms: int = 148) -> int:
-    """Kernels one gdn_chunk_prefill call enqueues on the benchmark's path (bf16, d = 128):
-    the chunk plan, then the intra-chunk and chain kernels once each, or once per piece when
-    a single sequence of 512 chunks or more is run in pieces (eight pieces of at least 64
-    chunks, while its 2 Hv chain CTAs leave at least 16 SMs free)."""
-    n_chunks = -(-T // 64)
-    if n_seq == 1 and n_chunks >= 8 * 64 and 2 * sh.Hv <= num_sms - 16:
-        per = max(64, -(-n_chunks // 8))
-        return 1 + 2 * (-(-n_chunks // per))
-    return 3
+    """Kernels one gdn_chunk_prefill call enqueues on the benchmark's path (bf16, d = 128), as
+    the library's own schedule counts them: the chunk plan, then the intra-chunk and chain
+    kernels once each, or, for a single sequence of 512 chunks or more run in pieces, one chain
+    launch per piece and the intra-chunk launches of its schedule."""
+    import gated_deltanet_mixer_causal_b200 as gdn
+    return gdn.gdn_chunk_prefill_launches(T, n_seq, sh.Hk, sh.Hv, sh.dk, sh.dv, torch.bfloat16, num_sms)
 
 
 # DRAM traffic (bytes, dram__bytes_read.sum + dram__bytes_write.sum) from one ncu capture

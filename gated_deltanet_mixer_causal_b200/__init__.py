@@ -17,11 +17,11 @@ from typing import Optional
 import torch
 
 from ._lib import (GDNError, LIB_PATH, gdn_chunk_prefill, gdn_chunk_prefill_noalloc,
-                   gdn_chunk_prefill_path, gdn_chunk_prefill_workspace_size, gdn_conv1d_silu, gdn_decode_step,
+                   gdn_chunk_prefill_path, gdn_chunk_prefill_launches, gdn_chunk_prefill_workspace_size, gdn_conv1d_silu, gdn_decode_step,
                    gdn_decode_tokens, gdn_prefill_noalloc_status, gdn_prefill_status, lib)
 
 __all__ = ["GDNError", "LIB_PATH", "lib", "gdn_conv1d_silu", "gdn_chunk_prefill",
-           "gdn_chunk_prefill_workspace_size", "gdn_chunk_prefill_noalloc", "gdn_chunk_prefill_path", "gdn_decode_step",
+           "gdn_chunk_prefill_workspace_size", "gdn_chunk_prefill_noalloc", "gdn_chunk_prefill_path", "gdn_chunk_prefill_launches", "gdn_decode_step",
            "gdn_decode_tokens", "gdn_prefill_status", "gdn_prefill_noalloc_status",
            "prefill_layer", "qkv_views"]
 

@@ -45,6 +45,7 @@ SIGNATURES = {
     "gdn_decode_tokens_ex": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int, _P, ctypes.c_int,
                                             _I32, _I32, _I32, _I32, _I32, _I32, _F32, _P]),
     "gdn_chunk_prefill_path": (_I32, [ctypes.c_int, _I32, _I32, _I32, _I32, _I32]),
+    "gdn_chunk_prefill_launches": (_I32, [_I64, _I32, _I32, _I32, _I32, _I32, ctypes.c_int, _I32, _I32]),
     "gdn_chunk_prefill_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_int, _I64, _I32,
                                                   _I32, _I32, _I32, _I64, _I64, _P, _I32, _P, _P,
                                                   _F32, _I32, _P]),
@@ -157,6 +158,17 @@ def gdn_chunk_prefill_path(dtype: torch.dtype, Hk: int, Hv: int, dk: int, dv: in
     if p < 0:
         raise GDNError(GDN_ERR_UNSUPPORTED, "gdn_chunk_prefill_path", "unsupported shape")
     return PATH_NAMES[p]
+
+
+def gdn_chunk_prefill_launches(T: int, n_seq: int, Hk: int, Hv: int, dk: int, dv: int,
+                               dtype: torch.dtype, num_sms: int, qk_l2norm: bool = True) -> int:
+    """How many of this library's kernels one gdn_chunk_prefill call with these sizes enqueues
+    on a GPU of num_sms SMs (host-only, no GPU needed)."""
+    code = GDN_BF16 if dtype == torch.bfloat16 else GDN_F32
+    n = lib().gdn_chunk_prefill_launches(T, n_seq, Hk, Hv, dk, dv, code, int(bool(qk_l2norm)), num_sms)
+    if n < 0:
+        raise GDNError(GDN_ERR_UNSUPPORTED, "gdn_chunk_prefill_launches", "unsupported arguments")
+    return int(n)
 
 
 def _row_view(t: torch.Tensor, name: str):

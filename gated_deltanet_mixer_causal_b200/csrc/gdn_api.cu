@@ -146,6 +146,14 @@ int32_t gdn_chunk_prefill_path(gdn_dtype_t dt, int32_t Hk, int32_t Hv, int32_t d
   return use_tensor_core_prefill(dt, dk, Hk, Hv, qk_l2norm) ? GDN_PATH_CHUNKED_TC : GDN_PATH_RECURRENT;
 }
 
+int32_t gdn_chunk_prefill_launches(int64_t T, int32_t n_seq, int32_t Hk, int32_t Hv, int32_t dk,
+                                   int32_t dv, gdn_dtype_t dt, int32_t qk_l2norm, int32_t num_sms) {
+  if (gdn_chunk_prefill_path(dt, Hk, Hv, dk, dv, qk_l2norm) < 0 || T < 0 || n_seq < 1 || num_sms < 1) return -1;
+  if (!use_tensor_core_prefill(dt, dk, Hk, Hv, qk_l2norm)) return 1;
+  if (!tc_rows_fit(T, n_seq, Hv)) return -1;
+  return gdn::prefill_chunk_tc_launches(T, n_seq, Hv, num_sms);
+}
+
 gdn_status_t gdn_chunk_prefill_ex(const void* q, const void* k, const void* v, const float* g,
                                   const float* beta, void* o, gdn_dtype_t dt, int64_t T,
                                   int32_t Hk, int32_t Hv, int32_t dk, int32_t dv, int64_t qk_stride,

@@ -57,6 +57,7 @@ constexpr int kPrefillTcMaxG = 8;
 size_t prefill_chunk_tc_workspace(int64_t T, int32_t n_seq, int32_t Hv);
 // The workspace's first int: 0, or the code of a bounded wait that gave up in the last call.
 const char* prefill_chunk_tc_error_string(int code);
+int prefill_chunk_tc_launches(int64_t T, int32_t n_seq, int32_t Hv, int num_sms);
 cudaError_t launch_prefill_chunk_tc(const void* q, const void* k, const void* v, const float* g,
                                     const float* beta, void* o, int64_t T, int32_t Hk, int32_t Hv,
                                     int64_t qk_stride, int64_t v_stride, const int32_t* cu,

@@ -1315,15 +1315,48 @@ size_t prefill_chunk_tc_workspace(int64_t T, int32_t n_seq, int32_t Hv) {
   return ws_layout(T, n_seq, Hv).total;
 }
 
-// Per device: the streams a prefill in pieces forks onto (two for the intra-chunk pieces, taken
-// in turn so that one piece's last items overlap the next piece's first, at the lowest
-// priority; one for the chains at the highest) and the events that order them, created on
-// first use and kept for the life of the process. Calls on one device take the mutex while
-// they enqueue.
+// How many leading chunks of a long sequence get their intra-chunk work done up front, on the
+// whole GPU, before the first chain piece starts; the intra-chunk work of the other chunks then
+// runs on the SMs the chain leaves free, up to the end of a piece per launch. A persistent
+// intra-chunk grid holds its SMs until its items run out, so a chain piece that becomes ready
+// beside one gets only the SMs that free up whole; restricting the later grids to the chain's
+// free SMs keeps every chain piece at full width. The split (a multiple of 16 chunks)
+// minimises a model of the call: chain pieces back to back, each starting once the intra-chunk
+// work of its chunks is done, with costs measured on B200 (intra-chunk work per chunk and value
+// head: 3.60 SM-us on the whole GPU, 4.15 SM-us beside the chain; chain: 2.07 us per chunk).
+// Only the schedule depends on these figures, never the results.
+constexpr double kIntraSmUsAlone = 3.60, kIntraSmUsBeside = 4.15, kChainUsPerChunk = 2.07;
+int64_t upfront_chunks(int64_t n_chunks, int64_t per, int pieces, int32_t Hv, int num_sms, int chain_ctas) {
+  const int free_sms = num_sms - chain_ctas;
+  auto piece_end = [&](int i) { return (i + 1) * per < n_chunks ? (i + 1) * per : n_chunks; };
+  int64_t best = n_chunks;
+  double best_t = -1.0;
+  for (int64_t x = 16; x <= n_chunks; x += 16) {
+    const double t_e = kIntraSmUsAlone * Hv * (double)x / num_sms;
+    double t_intra = t_e, t = t_e;
+    int64_t done = x;   // chunks whose intra-chunk work is done by t_intra
+    for (int i = 0; i < pieces; ++i) {
+      const int64_t c0 = i * per, c1 = piece_end(i);
+      if (c1 > done) {   // the launch that completes this piece's chunks
+        t_intra += kIntraSmUsBeside * Hv * (double)(c1 - done) / free_sms;
+        done = c1;
+        t = t > t_intra ? t : t_intra;
+      }
+      t += kChainUsPerChunk * (double)(c1 - c0);
+    }
+    if (best_t < 0.0 || t < best_t) { best = x; best_t = t; }
+  }
+  return best;
+}
+
+// Per device: the streams a prefill in pieces forks onto (one for the up-front intra-chunk
+// work and one for the rest, at the lowest priority; one for the chains at the highest) and
+// the events that order them, created on first use and kept for the life of the process.
+// Calls on one device take the mutex while they enqueue.
 struct PieceStreams {
   std::mutex mu;
   cudaStream_t side[2] = {nullptr, nullptr}, chain = nullptr;
-  cudaEvent_t ev[kMaxPieces + 2] = {};
+  cudaEvent_t ev[kMaxPieces + 3] = {};   // plan, up-front work, one per piece, join
 };
 
 PieceStreams* piece_streams(int dev) {
@@ -1338,13 +1371,28 @@ PieceStreams* piece_streams(int dev) {
   for (int i = 0; i < 2; ++i)
     if (p->side[i] == nullptr && cudaStreamCreateWithPriority(&p->side[i], cudaStreamNonBlocking, lo) != cudaSuccess)
       return nullptr;
-  for (int i = 0; i < kMaxPieces + 2; ++i)
+  for (int i = 0; i < kMaxPieces + 3; ++i)
     if (p->ev[i] == nullptr && cudaEventCreateWithFlags(&p->ev[i], cudaEventDisableTiming) != cudaSuccess)
       return nullptr;
   cudaStream_t chain = nullptr;
   if (cudaStreamCreateWithPriority(&chain, cudaStreamNonBlocking, hi) != cudaSuccess) return nullptr;
   p->chain = chain;   // set last: a non-null chain stream means the set is complete
   return p;
+}
+
+// Kernels launch_prefill_chunk_tc enqueues for these sizes on a GPU of num_sms SMs: the plan,
+// then one intra-chunk and one chain launch, or in pieces one chain launch per piece and one
+// intra-chunk launch for the up-front chunks plus one per piece that ends past them.
+int prefill_chunk_tc_launches(int64_t T, int32_t n_seq, int32_t Hv, int num_sms) {
+  if (!piece_layout(T, n_seq) || (int64_t)Hv * NT > num_sms - 16) return T > 0 ? 3 : 2;
+  const int64_t n_chunks = (T + C - 1) / C;
+  const int64_t per = piece_chunks(n_chunks);
+  const int pieces = (int)((n_chunks + per - 1) / per);
+  const int64_t x = upfront_chunks(n_chunks, per, pieces, Hv, num_sms, (int)(Hv * NT));
+  int n = 2 + pieces;
+  for (int i = 0; i < pieces; ++i)
+    if (((i + 1) * per < n_chunks ? (i + 1) * per : n_chunks) > x) ++n;
+  return n;
 }
 
 cudaError_t launch_prefill_chunk_tc(const void* q, const void* k, const void* v, const float* g,
@@ -1408,35 +1456,45 @@ cudaError_t launch_prefill_chunk_tc(const void* q, const void* k, const void* v,
         flags, static_cast<bf16*>(o), scale, blocks, 0, INT32_MAX);
     return cudaGetLastError();
   }
-  // One long sequence in pieces of piece_chunks() chunks. The intra-chunk kernels of the pieces
-  // run on two low-priority side streams in turn; the chain kernel of piece i runs on a
-  // high-priority stream once piece i's intra-chunk work is done, beside the intra-chunk work
-  // of the pieces after it (the chain occupies 2 Hv SMs; when a chain piece ends, its SMs go
-  // to the next chain piece first). The state goes from one chain piece to the next through
-  // the workspace in fp32. Only events order the streams: no kernel waits for another.
+  // One long sequence in pieces of piece_chunks() chunks. The intra-chunk work of the first x
+  // chunks (upfront_chunks) runs first as one launch on the whole GPU; then the chain pieces
+  // run back to back on a high-priority stream, piece i once the intra-chunk work of its
+  // chunks is done, beside the intra-chunk work of the rest on a low-priority stream, one
+  // launch up to the end of each piece, each with a persistent grid sized to the SMs the chain
+  // leaves free (the chain takes 2 Hv SMs). The state goes from one chain piece to the next
+  // through the workspace in fp32. Only events order the streams: no kernel waits for another.
   const int64_t per = piece_chunks(n_chunks);
   const int pieces = (int)((n_chunks + per - 1) / per);   // at most kTargetPieces + 1 <= kMaxPieces
+  const int chain_ctas = (int)gc.x;
+  const int64_t x = upfront_chunks(n_chunks, per, pieces, Hv, num_sms, chain_ctas);
   PieceStreams* ps = piece_streams(dev);
   if (ps == nullptr) return cudaErrorInitializationError;
   std::lock_guard<std::mutex> lock(ps->mu);   // the events are reused by every call on this device
   void* carry = ws + L.carry;
   cudaEvent_t* ev = ps->ev;
+  // slot s of a single sequence is its chunk s; the padding slot goes with the last chunk
+  auto slot_end = [&](int64_t c) { return (int32_t)(c == n_chunks ? slots : c); };
   if ((e = cudaEventRecord(ev[0], stream)) != cudaSuccess) return e;   // the plan is done
-  for (int sdx = 0; sdx < 2; ++sdx)
-    if ((e = cudaStreamWaitEvent(ps->side[sdx], ev[0], 0)) != cudaSuccess) return e;
-  if ((e = cudaStreamWaitEvent(ps->chain, ev[0], 0)) != cudaSuccess) return e;
-  for (int i = 0; i < pieces; ++i) {
-    const int64_t c0 = i * per, c1 = (i + 1) * per < n_chunks ? (i + 1) * per : n_chunks;
-    // slot s of a single sequence is its chunk s; the last piece also takes the padding slot
-    cudaStream_t side = ps->side[i & 1];
-    chunk_intra_kernel<<<intra_grid(c1 - c0), 128, kIntraSmem, side>>>(
-        mq, mk, mv, mwu, mmq, mul, g, beta, cu, n_seq, T, Hk, Hv, ws, (int32_t)c0,
-        (int32_t)(i == pieces - 1 ? slots : c1), i);
-    if ((e = cudaEventRecord(ev[1 + i], side)) != cudaSuccess) return e;
+  if ((e = cudaStreamWaitEvent(ps->side[0], ev[0], 0)) != cudaSuccess) return e;
+  chunk_intra_kernel<<<intra_grid(slot_end(x)), 128, kIntraSmem, ps->side[0]>>>(
+      mq, mk, mv, mwu, mmq, mul, g, beta, cu, n_seq, T, Hk, Hv, ws, 0, slot_end(x), 0);
+  if ((e = cudaEventRecord(ev[1], ps->side[0])) != cudaSuccess) return e;   // chunks 0 .. x-1
+  if ((e = cudaStreamWaitEvent(ps->chain, ev[1], 0)) != cudaSuccess) return e;
+  if ((e = cudaStreamWaitEvent(ps->side[1], ev[1], 0)) != cudaSuccess) return e;
+  const int64_t free_ctas = 2 * (int64_t)(num_sms - chain_ctas);
+  int64_t done = x;
+  for (int i = 0; i < pieces; ++i) {   // the rest, up to the end of each piece
+    const int64_t c1 = (i + 1) * per < n_chunks ? (i + 1) * per : n_chunks;
+    if (c1 <= done) continue;
+    const unsigned grid = intra_grid(slot_end(c1) - done);
+    chunk_intra_kernel<<<(unsigned)(grid < free_ctas ? grid : free_ctas), 128, kIntraSmem, ps->side[1]>>>(
+        mq, mk, mv, mwu, mmq, mul, g, beta, cu, n_seq, T, Hk, Hv, ws, (int32_t)done, slot_end(c1), 1 + i);
+    if ((e = cudaEventRecord(ev[2 + i], ps->side[1])) != cudaSuccess) return e;
+    done = c1;
   }
   for (int i = 0; i < pieces; ++i) {
     const int64_t c0 = i * per, c1 = (i + 1) * per < n_chunks ? (i + 1) * per : n_chunks;
-    if ((e = cudaStreamWaitEvent(ps->chain, ev[1 + i], 0)) != cudaSuccess) return e;
+    if (c1 > x && (e = cudaStreamWaitEvent(ps->chain, ev[2 + i], 0)) != cudaSuccess) return e;
     const bool first = i == 0, last = i == pieces - 1;
     const int f = (first ? user_bf * kStateInitBf16 : 0) | (last ? user_bf * kStateFinBf16 : 0) |
                   user_bf * kStateBlocksBf16;
@@ -1445,8 +1503,8 @@ cudaError_t launch_prefill_chunk_tc(const void* q, const void* k, const void* v,
         first ? init : carry, last ? fin : carry, f, static_cast<bf16*>(o), scale, blocks,
         (int32_t)c0, (int32_t)(last ? INT32_MAX : c1));
   }
-  if ((e = cudaEventRecord(ev[kMaxPieces + 1], ps->chain)) != cudaSuccess) return e;
-  if ((e = cudaStreamWaitEvent(stream, ev[kMaxPieces + 1], 0)) != cudaSuccess) return e;   // join
+  if ((e = cudaEventRecord(ev[kMaxPieces + 2], ps->chain)) != cudaSuccess) return e;
+  if ((e = cudaStreamWaitEvent(stream, ev[kMaxPieces + 2], 0)) != cudaSuccess) return e;   // join
   return cudaGetLastError();
 }
 

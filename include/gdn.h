@@ -128,6 +128,16 @@ int32_t gdn_chunk_prefill_path(gdn_dtype_t dt, int32_t Hk, int32_t Hv, int32_t d
                                int32_t qk_l2norm);
 
 /*
+ * gdn_chunk_prefill_launches -- how many kernels of this library one gdn_chunk_prefill call
+ * with these arguments enqueues on a GPU of num_sms SMs (host-only: no CUDA call is made):
+ * 1 on the token-recurrent path; on the tensor-core path the plan, then one intra-chunk and
+ * one chain launch, or, for one long sequence run in pieces, one chain launch per piece and
+ * the intra-chunk launches of its schedule. Returns -1 for arguments the prefill rejects.
+ */
+int32_t gdn_chunk_prefill_launches(int64_t T, int32_t n_seq, int32_t Hk, int32_t Hv, int32_t dk,
+                                   int32_t dv, gdn_dtype_t dt, int32_t qk_l2norm, int32_t num_sms);
+
+/*
  * gdn_chunk_prefill -- the gated delta rule over packed sequences (prefill).
  *
  * Defined by the Qwen3.5 page, section 5: S <- alpha S + beta (v - S k) k^T read as

@@ -13,7 +13,9 @@ import importlib.util
 import os
 
 import pytest
+import torch
 
+import gated_deltanet_mixer_causal_b200 as gdn
 from gated_deltanet_mixer_causal_b200 import workloads as W
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -122,13 +124,21 @@ def test_decode_tokens_bytes_reduce_to_one_step(bench):
 
 
 def test_prefill_launch_count(bench):
-    """The plan kernel, then one intra-chunk and one chain launch per piece: eight pieces for
-    the 27B layer at 65,536 tokens, one pass below 32,768 tokens, for several sequences, or
-    when the chains would leave fewer than 16 SMs."""
+    """The plan kernel, then one intra-chunk and one chain launch; a single sequence of 512
+    chunks or more runs in eight pieces: one chain launch per piece, one intra-chunk launch for
+    the chunks done up front (544 of 1024 for the 27B layer at 65,536 tokens, 272 of 512 at
+    32,768) and one for the rest of each later piece. One pass below 32,768 tokens, for several
+    sequences, or when the chains would leave fewer than 16 SMs."""
     sh = W.QWEN35_27B
-    assert bench.gdn_prefill_launches(65536, 1, sh) == 17
-    assert bench.gdn_prefill_launches(32768, 1, sh) == 17
-    assert bench.gdn_prefill_launches(33000, 1, sh) == 17     # 516 chunks in pieces of 65
+    assert bench.gdn_prefill_launches(65536, 1, sh) == 1 + 1 + 4 + 8
+    assert bench.gdn_prefill_launches(32768, 1, sh) == 1 + 1 + 4 + 8
+    assert bench.gdn_prefill_launches(33000, 1, sh) == 1 + 1 + 4 + 8   # 516 chunks, pieces of 65
     assert bench.gdn_prefill_launches(16384, 1, sh) == 3
     assert bench.gdn_prefill_launches(65536, 2, sh) == 3
     assert bench.gdn_prefill_launches(65536, 1, W.LayerShape(16, 80, 128, 128)) == 3
+    # the 9B layer (Hv 32): its chains leave 84 SMs, enough for the intra-chunk work of every
+    # piece after the first to keep up with them
+    assert bench.gdn_prefill_launches(65536, 1, W.QWEN35_9B) == 1 + 1 + 7 + 8
+    assert bench.gdn_prefill_launches(0, 1, sh) == 2
+    assert gdn.gdn_chunk_prefill_launches(4096, 1, 2, 2, 16, 16, torch.float32, 148) == 1
+    assert gdn.gdn_chunk_prefill_launches(65536, 1, 16, 48, 128, 128, torch.bfloat16, 148, qk_l2norm=False) == 1
