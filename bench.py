@@ -530,6 +530,7 @@ def main():
                        "global_batch": world, "seq_len": T, "parallelism": f"dp{world}",
                        "l2": "inputs larger than L2 (126 MB); no flush"},
             "prefill": {"tokens_per_s": value, "conv_ms": conv_avg, "chunk_prefill_ms": pre_avg,
+                        "chunk_prefill_ms_steps": [round(t, 4) for t in pre_ms],
                         "chunk_prefill_tflops": pre_tflops,
                         "flops_per_token": prefill_flops_per_token(),
                         "layer_ms": (conv_avg + pre_avg),

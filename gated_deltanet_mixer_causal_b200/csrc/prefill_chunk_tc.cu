@@ -1320,8 +1320,8 @@ size_t prefill_chunk_tc_workspace(int64_t T, int32_t n_seq, int32_t Hv) {
 // runs on the SMs the chain leaves free, up to the end of a piece per launch. A persistent
 // intra-chunk grid holds its SMs until its items run out, so a chain piece that becomes ready
 // beside one gets only the SMs that free up whole; restricting the later grids to the chain's
-// free SMs keeps every chain piece at full width. The split (a multiple of 16 chunks)
-// minimises a model of the call: chain pieces back to back, each starting once the intra-chunk
+// free SMs keeps every chain piece at full width. The split (a multiple of 16 chunks, at least
+// the first piece) minimises a model of the call: chain pieces back to back, each starting once the intra-chunk
 // work of its chunks is done, with costs measured on B200 (intra-chunk work per chunk and value
 // head: 3.60 SM-us on the whole GPU, 4.15 SM-us beside the chain; chain: 2.07 us per chunk).
 // Only the schedule depends on these figures, never the results.
@@ -1331,7 +1331,8 @@ int64_t upfront_chunks(int64_t n_chunks, int64_t per, int pieces, int32_t Hv, in
   auto piece_end = [&](int i) { return (i + 1) * per < n_chunks ? (i + 1) * per : n_chunks; };
   int64_t best = n_chunks;
   double best_t = -1.0;
-  for (int64_t x = 16; x <= n_chunks; x += 16) {
+  for (int64_t x = (per + 15) / 16 * 16; x <= n_chunks; x += 16) {   // x >= per: chain 0 needs
+                                                                     // only the up-front launch
     const double t_e = kIntraSmUsAlone * Hv * (double)x / num_sms;
     double t_intra = t_e, t = t_e;
     int64_t done = x;   // chunks whose intra-chunk work is done by t_intra
@@ -1356,7 +1357,7 @@ int64_t upfront_chunks(int64_t n_chunks, int64_t per, int pieces, int32_t Hv, in
 struct PieceStreams {
   std::mutex mu;
   cudaStream_t side[2] = {nullptr, nullptr}, chain = nullptr;
-  cudaEvent_t ev[kMaxPieces + 3] = {};   // plan, up-front work, one per piece, join
+  cudaEvent_t ev[kMaxPieces + 3] = {};   // plan, up-front work, one per piece, chain start, join
 };
 
 PieceStreams* piece_streams(int dev) {
@@ -1480,7 +1481,35 @@ cudaError_t launch_prefill_chunk_tc(const void* q, const void* k, const void* v,
       mq, mk, mv, mwu, mmq, mul, g, beta, cu, n_seq, T, Hk, Hv, ws, 0, slot_end(x), 0);
   if ((e = cudaEventRecord(ev[1], ps->side[0])) != cudaSuccess) return e;   // chunks 0 .. x-1
   if ((e = cudaStreamWaitEvent(ps->chain, ev[1], 0)) != cudaSuccess) return e;
-  if ((e = cudaStreamWaitEvent(ps->side[1], ev[1], 0)) != cudaSuccess) return e;
+  auto chain_piece = [&](int i, cudaEvent_t started) {
+    const int64_t c0 = i * per, c1 = (i + 1) * per < n_chunks ? (i + 1) * per : n_chunks;
+    const bool first = i == 0, last = i == pieces - 1;
+    const int f = (first ? user_bf * kStateInitBf16 : 0) | (last ? user_bf * kStateFinBf16 : 0) |
+                  user_bf * kStateBlocksBf16;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = gc;
+    cfg.blockDim = dim3(kChainThreads);
+    cfg.dynamicSmemBytes = kChainSmem;
+    cfg.stream = ps->chain;
+    cudaLaunchAttribute attr[1];
+    if (started != nullptr) {   // fires once the piece's CTAs have all begun (at worst at its end)
+      attr[0].id = cudaLaunchAttributeLaunchCompletionEvent;
+      attr[0].val.launchCompletionEvent.event = started;
+      attr[0].val.launchCompletionEvent.flags = 0;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+    }
+    return cudaLaunchKernelEx(&cfg, chunk_chain_kernel, mq, mk, mwu, mmq, mul, mo, cu, n_seq, T, Hk, Hv,
+                              (const uint8_t*)ws, reinterpret_cast<int*>(ws + L.err), first ? init : carry,
+                              last ? fin : carry, f, static_cast<bf16*>(o), scale, blocks, (int32_t)c0,
+                              (int32_t)(last ? INT32_MAX : c1));
+  };
+  // chain piece 0 first: the intra-chunk work beside the chains starts only once its CTAs have
+  // all begun, so that they take whole SMs before the intra-chunk grid spreads over the GPU
+  // (x >= the first piece: chain piece 0 waits for nothing on that stream, so no cycle)
+  if ((e = chain_piece(0, ev[kMaxPieces + 1])) != cudaSuccess) return e;
+  if ((e = cudaStreamWaitEvent(ps->side[1], ev[0], 0)) != cudaSuccess) return e;   // the plan
+  if ((e = cudaStreamWaitEvent(ps->side[1], ev[kMaxPieces + 1], 0)) != cudaSuccess) return e;
   const int64_t free_ctas = 2 * (int64_t)(num_sms - chain_ctas);
   int64_t done = x;
   for (int i = 0; i < pieces; ++i) {   // the rest, up to the end of each piece
@@ -1492,16 +1521,10 @@ cudaError_t launch_prefill_chunk_tc(const void* q, const void* k, const void* v,
     if ((e = cudaEventRecord(ev[2 + i], ps->side[1])) != cudaSuccess) return e;
     done = c1;
   }
-  for (int i = 0; i < pieces; ++i) {
-    const int64_t c0 = i * per, c1 = (i + 1) * per < n_chunks ? (i + 1) * per : n_chunks;
+  for (int i = 1; i < pieces; ++i) {   // after the records above: each wait is on this call's
+    const int64_t c1 = (i + 1) * per < n_chunks ? (i + 1) * per : n_chunks;
     if (c1 > x && (e = cudaStreamWaitEvent(ps->chain, ev[2 + i], 0)) != cudaSuccess) return e;
-    const bool first = i == 0, last = i == pieces - 1;
-    const int f = (first ? user_bf * kStateInitBf16 : 0) | (last ? user_bf * kStateFinBf16 : 0) |
-                  user_bf * kStateBlocksBf16;
-    chunk_chain_kernel<<<gc, kChainThreads, kChainSmem, ps->chain>>>(
-        mq, mk, mwu, mmq, mul, mo, cu, n_seq, T, Hk, Hv, ws, reinterpret_cast<int*>(ws + L.err),
-        first ? init : carry, last ? fin : carry, f, static_cast<bf16*>(o), scale, blocks,
-        (int32_t)c0, (int32_t)(last ? INT32_MAX : c1));
+    if ((e = chain_piece(i, nullptr)) != cudaSuccess) return e;
   }
   if ((e = cudaEventRecord(ev[kMaxPieces + 2], ps->chain)) != cudaSuccess) return e;
   if ((e = cudaStreamWaitEvent(stream, ev[kMaxPieces + 2], 0)) != cudaSuccess) return e;   // join
