@@ -564,20 +564,20 @@ def gdn_prefill_launches(T: int, n_seq: int = 1, sh=SHAPE, num_sms: int = 148) -
 # of each kernel on the small case (T = 8192, decode batch 64), per unit processed (token
 # for the prefill kernels and the conv, sequence for the decode step), scaled to the
 # benchmark's launch; None when the kernel changed since the capture. The prefill figure is
-# the intra-chunk kernel's 468.54 MB plus the chain kernel's 512.83 MB.
-TRAFFIC_PER_UNIT = {"prefill": (468.54e6 + 512.83e6) / 8192, "conv": 291.25e6 / 8192,
+# the intra-chunk kernel's 468.19 MB plus the chain kernel's 512.32 MB.
+TRAFFIC_PER_UNIT = {"prefill": (468.19e6 + 512.32e6) / 8192, "conv": 291.25e6 / 8192,
                     "decode": 357.64e6 / 64}
 
 # The chunked prefill's two kernels: their share of its FLOPs (from the chunked form: the
 # intra-chunk kernel forms K K^T and Q K^T per key head, solves the triangular system and
 # builds U~ = P V, W = Pk K and Mqk; the chain applies [-W; Q] S0^T, K^T U' and Mqk U), the
-# device time of their launches in one 65536-token call from the ncu launch list (serialised
-# by ncu: eight pieces of each, 1527.1 us of intra-chunk and 2166.0 us of chain launches; in
-# the call the pieces of the two kernels overlap, so the call takes less than their sum), and
-# their DRAM traffic per token from the same captures as above.
+# device time each takes alone for a 65536-token call's work (its ncu capture at T = 8192,
+# one launch on the whole GPU, scaled by tokens: 168.54 us -> 1348.4 us of intra-chunk work,
+# 266.94 us -> 2135.6 us of chain; in the call the two run side by side, so the call takes
+# less than their sum), and their DRAM traffic per token from the same captures.
 PREFILL_KERNELS = {
-    "chunk_intra": {"busy_us_64k": 1527.1, "traffic_per_token": 468.54e6 / 8192},
-    "chunk_chain": {"busy_us_64k": 2166.0, "traffic_per_token": 512.83e6 / 8192},
+    "chunk_intra": {"busy_us_64k": 1348.4, "traffic_per_token": 468.19e6 / 8192},
+    "chunk_chain": {"busy_us_64k": 2135.6, "traffic_per_token": 512.32e6 / 8192},
 }
 
 
@@ -602,8 +602,9 @@ def prefill_kernel_split(T: int, prefill_ms: float, peak_tflops: float) -> dict:
                   "frac": flops / (ms / 1e3) / 1e12 / peak_tflops,
                   "traffic": v["traffic_per_token"] * T}
     out["overlap"] = {"device_ms_sum": busy, "call_ms": prefill_ms,
-                      "note": "intra-chunk pieces run beside chain pieces: the call is shorter "
-                              "than the sum of its kernels' device times"}
+                      "note": "each kernel's device time alone for the call's work; in the call "
+                              "the intra-chunk work of later pieces runs beside the chain "
+                              "pieces, so the call is shorter than the sum"}
     return out
 
 
