@@ -865,10 +865,11 @@ __device__ __forceinline__ void tma_store_wait_read_le1() {
 //   issuers : rA(c) = [-W; Q] S0^T in two K halves (dk rows 0..63 after the state warps of
 //             quadrants 0, 1 are done, 64..127 after quadrants 2, 3), the lo half on top of
 //             [I; 0] U~ (issued as soon as the stage lands, off the serial path);
-//             dS^T = K^T [U' | U'lo] once all of U is written (U' is carried as a bf16
+//             dS^T = K^T [U' | U'lo] once all of U' is written (U' is carried as a bf16
 //             hi + lo pair on the state path, where a chunk that rewrites one key
 //             telescopes U's rows), then O2 = [K atom1; Mqk] U behind it (second issuer)
-//   compute : U = rows 0..63 of rA -> U (bf16), U' (hi + lo) (quadrants 0, 1)   -> "U ready"
+//   compute : U = rows 0..63 of rA -> U' (hi + lo) -> "U' ready", U (bf16) -> "U ready"
+//             (quadrants 0, 1)
 //             S^T <- e^{G_L} S^T + dS^T, bf16 copy (all 8 warps)               -> "S ready"
 //             o = scale (e^{G_r}/|q_r| rows 64..127 of rA + O2) (quadrants 2, 3): a full
 //             chunk is staged in shared memory and leaves by one TMA store     -> "stage free"
@@ -915,8 +916,10 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
   uint64_t* bar_A1 = bars + 9;
   uint64_t* bar_B = bars + 10;     // dS^T complete
   uint64_t* bar_O = bars + 12;
-  uint64_t* bar_U0 = bars + 13;    // U, U' rows 0..31 written (the 2 warps of quadrant 0)
+  uint64_t* bar_U0 = bars + 13;    // U rows 0..31 written (the 2 warps of quadrant 0)
   uint64_t* bar_U1 = bars + 14;    // rows 32..63 (quadrant 1)
+  uint64_t* bar_Up0 = bars + 23;   // U' (hi + lo) rows 0..31 written, before U itself
+  uint64_t* bar_Up1 = bars + 24;   // rows 32..63
   uint64_t* bar_S0 = bars + 15;    // state bf16 rows 0..63 written (quadrants 0, 1: 4 warps)
   uint64_t* bar_S1 = bars + 16;    // rows 64..127 (quadrants 2, 3)
   uint64_t* bar_drain = bars + 17; // [3] on an early exit: each issuing thread's MMAs have completed
@@ -933,6 +936,8 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     for (int i = 8; i < 13; ++i) mbar_init(&bars[i], 1);
     mbar_init(bar_U0, 2);
     mbar_init(bar_U1, 2);
+    mbar_init(bar_Up0, 2);
+    mbar_init(bar_Up1, 2);
     mbar_init(bar_S0, 4);
     mbar_init(bar_S1, 4);
     for (int i = 0; i < 3; ++i) mbar_init(&bar_drain[i], 1);
@@ -1072,15 +1077,18 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     issue_rA(0);
     for (int c = 0; c < nc; ++c) {
       const int b = c & 1;
-      if (part == 1) {   // once all of U is written: dS^T, then O2 behind it in the queue
-        if (__any_sync(0xffffffffu, !mbar_spin(bar_U1, (uint32_t)c & 1u, err_word, kErrChainMma) ||
-                                        !mbar_spin(bar_U0, (uint32_t)c & 1u, err_word, kErrChainMma) ||
+      if (part == 1) {   // once all of U' is written: dS^T; once U is: O2 behind it in the queue
+        if (__any_sync(0xffffffffu, !mbar_spin(bar_Up1, (uint32_t)c & 1u, err_word, kErrChainMma) ||
+                                        !mbar_spin(bar_Up0, (uint32_t)c & 1u, err_word, kErrChainMma) ||
                                         !mbar_spin(&bar_tmb[b], (uint32_t)(c >> 1) & 1u, err_word, kErrChainTma))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)   // dS^T = K^T [U' | U'lo]: N = 128, the two halves summed later
           mma_bf16_warp(tmem + kTdS, dK + soff(b) + 128 * kk, dUp + 128 * kk, kIB, kk > 0);
         mma_commit_warp(bar_B);
+        if (__any_sync(0xffffffffu, !mbar_spin(bar_U1, (uint32_t)c & 1u, err_word, kErrChainMma) ||
+                                        !mbar_spin(bar_U0, (uint32_t)c & 1u, err_word, kErrChainMma))) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)   // rows 64..127 of [K atom1; Mqk] U
           mma_bf16_warp(tmem + kTO2 + 64 * b, dUM + soff(b) + 2 * kk, dU + 128 * kk, kIA, kk > 0);
@@ -1156,21 +1164,31 @@ chunk_chain_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
         tmem_ld32_async(tq + kTAhi + 64 * b + half * 32, a1);
         tmem_wait_ld(a0, a1);
 #pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8) {   // U in bf16; U' as a hi + lo bf16 pair
-          uint32_t u[4], hi[4], lo[4];
+        // U' (a hi + lo bf16 pair) first: dS^T, on the serial path, needs only U'; then U in
+        // bf16 for O2
+        uint32_t u[4][4];
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8) {
+          uint32_t hi[4], lo[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const float x0 = __uint_as_float(a0[c8 * 8 + 2 * q]) + __uint_as_float(a1[c8 * 8 + 2 * q]);
             const float x1 = __uint_as_float(a0[c8 * 8 + 2 * q + 1]) + __uint_as_float(a1[c8 * 8 + 2 * q + 1]);
             __nv_bfloat162 ub = __floats2bfloat162_rn(x0, x1);
-            u[q] = *reinterpret_cast<uint32_t*>(&ub);
+            u[c8][q] = *reinterpret_cast<uint32_t*>(&ub);
             split_bf16x2_alu(us * x0, us * x1, hi[q], lo[q]);
           }
           const uint32_t off = sw128_off(r, half * 32 + c8 * 8);
-          *reinterpret_cast<uint4*>(sm + kCU + off) = make_uint4(u[0], u[1], u[2], u[3]);
           *reinterpret_cast<uint4*>(sm + kCUp + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
           *reinterpret_cast<uint4*>(sm + kCUpl + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
+        fence_async_smem();
+        tc_fence_before();
+        warp_arrive(quad == 0 ? bar_Up0 : bar_Up1);
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8)
+          *reinterpret_cast<uint4*>(sm + kCU + sw128_off(r, half * 32 + c8 * 8)) =
+              make_uint4(u[c8][0], u[c8][1], u[c8][2], u[c8][3]);
         fence_async_smem();
         tc_fence_before();
         warp_arrive(quad == 0 ? bar_U0 : bar_U1);
