@@ -564,8 +564,8 @@ def gdn_prefill_launches(T: int, n_seq: int = 1, sh=SHAPE, num_sms: int = 148) -
 # of each kernel on the small case (T = 8192, decode batch 64), per unit processed (token
 # for the prefill kernels and the conv, sequence for the decode step), scaled to the
 # benchmark's launch; None when the kernel changed since the capture. The prefill figure is
-# the intra-chunk kernel's 468.19 MB plus the chain kernel's 512.32 MB.
-TRAFFIC_PER_UNIT = {"prefill": (468.19e6 + 512.32e6) / 8192, "conv": 291.25e6 / 8192,
+# the intra-chunk kernel's 468.19 MB plus the chain kernel's 509.36 MB.
+TRAFFIC_PER_UNIT = {"prefill": (468.19e6 + 509.36e6) / 8192, "conv": 291.25e6 / 8192,
                     "decode": 357.64e6 / 64}
 
 # The chunked prefill's two kernels: their share of its FLOPs (from the chunked form: the
@@ -573,11 +573,11 @@ TRAFFIC_PER_UNIT = {"prefill": (468.19e6 + 512.32e6) / 8192, "conv": 291.25e6 / 
 # builds U~ = P V, W = Pk K and Mqk; the chain applies [-W; Q] S0^T, K^T U' and Mqk U), the
 # device time each takes alone for a 65536-token call's work (its ncu capture at T = 8192,
 # one launch on the whole GPU, scaled by tokens: 168.54 us -> 1348.4 us of intra-chunk work,
-# 266.94 us -> 2135.6 us of chain; in the call the two run side by side, so the call takes
+# 265.18 us -> 2121.5 us of chain; in the call the two run side by side, so the call takes
 # less than their sum), and their DRAM traffic per token from the same captures.
 PREFILL_KERNELS = {
     "chunk_intra": {"busy_us_64k": 1348.4, "traffic_per_token": 468.19e6 / 8192},
-    "chunk_chain": {"busy_us_64k": 2135.6, "traffic_per_token": 512.32e6 / 8192},
+    "chunk_chain": {"busy_us_64k": 2121.5, "traffic_per_token": 509.36e6 / 8192},
 }
 
 
