@@ -93,3 +93,36 @@ def test_pieces_equal_the_caller_split(cuda_device, form):
     torch.cuda.synchronize()
     assert torch.equal(o, torch.cat(parts, 0))
     assert torch.equal(fin, state)
+
+
+@pytest.mark.parametrize("T_call", [16384, 65536])
+def test_launch_count_is_what_runs(cuda_device, T_call):
+    """gdn_chunk_prefill_launches, which the benchmark reports as its kernel count, equals the
+    number of this library's kernels one call runs (CUPTI trace): one pass at 16,384 tokens
+    of the 27B layer, the up-front, beside-the-chain and chain launches at 65,536."""
+    from torch.profiler import ProfilerActivity, profile
+    dev = cuda_device
+    sh = W.QWEN35_27B
+    gen = torch.Generator(device="cpu").manual_seed(5)
+    q = torch.randn((T_call, sh.Hk, sh.dk), generator=gen).to(torch.bfloat16).to(dev)
+    k = torch.randn((T_call, sh.Hk, sh.dk), generator=gen).to(torch.bfloat16).to(dev)
+    v = torch.randn((T_call, sh.Hv, sh.dv), generator=gen).to(torch.bfloat16).to(dev)
+    g = (-0.3 * torch.rand((T_call, sh.Hv), generator=gen)).to(dev)
+    beta = torch.sigmoid(torch.randn((T_call, sh.Hv), generator=gen)).to(dev)
+    fin = torch.empty((1, sh.Hv, sh.dv, sh.dk), device=dev)
+    o = torch.empty((T_call, sh.Hv, sh.dv), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(gdn.gdn_chunk_prefill_workspace_size(T_call, 1, sh.Hk, sh.Hv, sh.dk, sh.dv, torch.bfloat16),
+                     dtype=torch.uint8, device=dev)
+    run = lambda: gdn.gdn_chunk_prefill(q, k, v, g, beta, None, None, fin, 1.0, True, o, ws)
+    run()
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        run()
+        torch.cuda.synchronize()
+    ours = [e.name for e in prof.events()
+            if e.device_type == torch.autograd.DeviceType.CUDA and "chunk_" in e.name]
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    expect = gdn.gdn_chunk_prefill_launches(T_call, 1, sh.Hk, sh.Hv, sh.dk, sh.dv, torch.bfloat16, sms)
+    assert len(ours) == expect, ours
+    assert sum("chunk_plan" in n for n in ours) == 1
+    assert sum("chunk_chain" in n for n in ours) == (1 if expect == 3 else 8)
